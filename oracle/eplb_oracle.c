@@ -307,9 +307,9 @@ int oracle_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P,
   if (R < 0 || E <= 0 || P <= 0 || G <= 0 || N <= 0 || gpus <= 0 || X <= 0)
     return ORACLE_ERR_SHAPE;
   if (P < E) return ORACLE_ERR_SHAPE;
-  if (E % G != 0 || gpus % N != 0 || P % gpus != 0) return ORACLE_ERR_DIVISIBILITY;
+  if (E % G != 0 || P % gpus != 0) return ORACLE_ERR_DIVISIBILITY;
   int g = G, n = N;
-  if (G % N != 0) { g = 1; n = 1; } /* global policy */
+  if (G % N != 0) { g = 1; n = 1; } /* global policy: gpus % N is not needed */
   for (int64_t r = 0; r < R; ++r) {
     const int64_t *w = loads + r * E;
     for (int e = 0; e < E; ++e)

@@ -315,6 +315,10 @@ def test_rebalance_errors():
         oracle.rebalance(w, 18, 4, 2, 8)            # 18 % 8 != 0
     assert e.value.code == oracle.ERR_DIVISIBILITY
     with pytest.raises(oracle.OracleError) as e:
+        oracle.rebalance(w, 18, 4, 4, 6)            # hierarchical needs gpus % nodes == 0
+    assert e.value.code == oracle.ERR_DIVISIBILITY
+    oracle.rebalance(w, 18, 3, 2, 3)                # global: 3 % 2 != 0 is fine
+    with pytest.raises(oracle.OracleError) as e:
         oracle.rebalance(w, 8, 4, 2, 8)             # fewer replicas than experts
     assert e.value.code == oracle.ERR_SHAPE
     with pytest.raises(oracle.OracleError) as e:
