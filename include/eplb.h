@@ -1,0 +1,161 @@
+/*
+ * eplb.h -- C ABI of libeplb.so, the B200 (sm_100a) hot path of the
+ * Expert-Parallelism Load Balancer: count expert loads, accumulate them over
+ * a sliding window, rebalance every MoE layer into a replica/placement plan,
+ * and redirect token indices to physical replicas.
+ *
+ * Sources cited below:
+ *   [EPLB] page "DualPipe и EPLB: конвейер в обе стороны и балансировщик
+ *          экспертов", Part 2 "EPLB": section "Алгоритм" (hierarchical and
+ *          global policies, moving-average load prediction), box
+ *          "От переводчика: термины" (load = routed tokens), section
+ *          "Интерфейс и пример" and the appendix eplb.py (rebalance_experts,
+ *          balanced_packing, replicate_experts).
+ *   [LPLB] page "DeepSeek开源LPLB：基于线性规划的MoE负载均衡器...", usage
+ *          example: a planner maps the router's logical indices to physical
+ *          indices.
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" are caller-owned global memory on the current
+ *     CUDA device; the library allocates nothing and keeps no state besides
+ *     a per-device cache of launch limits.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *     The return value covers host-side argument checks and launch errors.
+ *     Data-dependent errors (an index or load out of range, a wait that ran
+ *     out) are reported through the optional device word `status`: when it
+ *     is non-NULL the first error code of the call is stored there with an
+ *     atomic compare-and-swap from EPLB_OK; callers clear it beforehand.
+ *   - Layouts are dense row-major (C order), element strides as stated.
+ *   - Integer indices are int32; loads and counts are int64.
+ */
+#ifndef EPLB_H_
+#define EPLB_H_
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum eplb_status {
+  EPLB_OK = 0,
+  EPLB_ERR_NULL = 1,          /* a required pointer is NULL */
+  EPLB_ERR_SHAPE = 2,         /* negative or inconsistent sizes, P < E */
+  EPLB_ERR_DIVISIBILITY = 3,  /* E % G, gpus % N or P % gpus is not 0 */
+  EPLB_ERR_RANGE = 4,         /* a load outside [0, 2^40), an exact ratio too wide,
+                                 a logcnt outside [1, X] given to redirect */
+  EPLB_ERR_SLOTS = 5,         /* an expert got more replicas than log2phy slots X */
+  EPLB_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed */
+  EPLB_ERR_TIMEOUT = 7,       /* an in-kernel wait gave up (bounded, ~2 s) */
+  EPLB_ERR_ALIGN = 8,         /* a pointer lacks the alignment stated below */
+  EPLB_ERR_LIMIT = 9          /* a size beyond this build's stated limits */
+} eplb_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *eplb_status_string(int32_t status);
+
+/* Message of the last CUDA error seen by a call on this host thread. */
+const char *eplb_last_cuda_error(void);
+
+/* ABI version of this library: (major << 16) | minor. */
+int32_t eplb_abi_version(void);
+
+/*
+ * S1 -- load counting.  [EPLB] "От переводчика: термины": the load of an
+ * expert is the number of tokens the router sent it.
+ *
+ *   counts[l, e] (+)= #{ (t, k) : idx[l, t, k] == e }
+ *
+ * idx      device int32 [L, T, K] (16-byte aligned); values outside [0, E)
+ *          are skipped and their number is added to *bad.
+ * counts   device int64 [L, E]; overwritten (accumulate == 0) or added to.
+ * bad      device uint64 word, nullable; added to, never cleared.
+ * status   device int32 word, nullable (EPLB_ERR_TIMEOUT only).
+ * Limits:  1 <= E <= 1024, K >= 1, L, T >= 0.
+ * Integer atomics make the result independent of scheduling.
+ */
+eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K,
+                             int32_t E, int64_t *counts, int32_t accumulate,
+                             unsigned long long *bad, int32_t *status,
+                             cudaStream_t stream);
+
+/*
+ * S2 -- sliding-window accumulation.  [EPLB] "Алгоритм": expert load is
+ * commonly predicted by a moving average over historical statistics; the
+ * window sum is that average times W.
+ *
+ *   snaps[s - s_first, l, e] = sum_{u = max(0, s-W+1)}^{s} steps[u, l, e],
+ *   for s_first <= s < S.
+ *
+ * steps    device int64 [S, L, E].
+ * snaps    device int64 [S - s_first, L, E]; must not overlap steps.
+ * W >= 1 (W >= S gives running totals); 0 <= s_first < S.
+ * Sums are exact; wrap-around of int64 is the caller's concern.
+ * With a ring buffer of the last W per-step counts, s_first = S - 1 = W - 1
+ * returns the current window sum (row order does not change a full sum).
+ */
+eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, int32_t E,
+                                   int64_t W, int64_t s_first, int64_t *snaps,
+                                   int32_t *status, cudaStream_t stream);
+
+/*
+ * S3/S4 -- rebalance_experts over R independent rows ([EPLB] "Алгоритм",
+ * appendix rebalance_experts / rebalance_experts_hierarchical /
+ * balanced_packing / replicate_experts).  Policy: hierarchical when
+ * G % N == 0, otherwise the same procedure with one group on one node
+ * (global).  Per row:
+ *   1. group loads -> balanced_packing over N nodes (G/N groups each);
+ *   2. replicate_experts inside every node (E/N -> P/N replicas, each extra
+ *      replica to the largest load per replica, lowest index on ties);
+ *   3. replica loads w/cnt -> balanced_packing over the node's gpus/N GPUs
+ *      (P/gpus replicas each; heaviest first, stable; lightest non-full
+ *      GPU, lowest index on ties);
+ * all comparisons exact (integer cross-products, sums of w/cnt over a
+ * common denominator).  Outputs:
+ *   phy2log[r, p]  logical expert of physical slot p (slot p lives on GPU
+ *                  p / (P/gpus), node p / (P/N));
+ *   phyrank[r, p]  replica rank of slot p among its expert's replicas;
+ *   logcnt[r, e]   replicas of expert e;
+ *   log2phy[r, e, k] = physical slot of replica k of e, -1 for k >= logcnt.
+ *
+ * loads    device int64 [R, E], each in [0, 2^40) (else the row's outputs
+ *          are -1 / 0 and *status = EPLB_ERR_RANGE).
+ * phy2log, phyrank  device int32 [R, P]; logcnt device int32 [R, E];
+ * log2phy  device int32 [R, E, X].  X = (P - E) / N + 1 (hierarchical) or
+ *          P - E + 1 (global) always suffices; with a smaller X, replicas of
+ *          rank >= X are left out of log2phy and *status = EPLB_ERR_SLOTS.
+ * Limits:  1 <= E <= 1024, E <= P <= 2048, G | E, gpus | P, N | gpus (hierarchical),
+ *          X >= 1, R >= 0.
+ */
+eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P,
+                           int32_t G, int32_t N, int32_t gpus, int32_t X,
+                           int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
+                           int32_t *log2phy, int32_t *status, cudaStream_t stream);
+
+/*
+ * S5 -- redirect logical expert indices to physical replicas ([LPLB] usage
+ * example: logical indices in, physical indices out).  Replica rule (this
+ * library's fixed choice; the pages leave it open): token t of the call is
+ * global token t0 + t and uses replica (t0 + t) mod logcnt[l, e] for every
+ * one of its K slots, so shards of one batch redirect consistently.
+ *
+ *   out[l, t, k] = log2phy[l, e, (t0 + t) mod logcnt[l, e]],  e = idx[l, t, k]
+ *
+ * idx, out device int32 [L, T, K], both 16-byte aligned, not overlapping.
+ *          An index outside [0, E) gives -1 and is added to *bad; a logcnt
+ *          outside [1, X] gives -1 and *status = EPLB_ERR_RANGE.
+ * log2phy  device int32 [L, E, X]; logcnt device int32 [L, E].
+ * Limits:  1 <= E <= 1024, 1 <= X, E * X <= 32768, T * K < 2^31,
+ *          0 <= t0, t0 + T < 2^31.
+ */
+eplb_status eplb_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                          const int32_t *log2phy, int32_t X, const int32_t *logcnt,
+                          int64_t t0, int32_t *out, unsigned long long *bad,
+                          int32_t *status, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EPLB_H_ */

@@ -1,0 +1,214 @@
+"""B200-native EPLB hot path: Python binding of libeplb.so.
+
+The four stages of the Expert-Parallelism Load Balancer's data path run in
+hand-written sm_100a kernels behind a C ABI (``include/eplb.h``); this module
+only marshals torch CUDA tensors (pointers, sizes, the current stream) into
+those calls.  There is no fallback: if ``libeplb.so`` is missing or no CUDA
+device is present, every call raises.
+
+    counts  = count_loads(idx, E)                        # S1  int64 [L, E]
+    snaps   = window_accumulate(steps, W)                # S2  int64 [S, L, E]
+    plan    = rebalance(loads, P, G, N, gpus)            # S3/S4 Plan(phy2log, phyrank, logcnt, log2phy)
+    phys    = redirect(idx, plan.log2phy, plan.logcnt)   # S5  int32 [L, T, K]
+
+Sources: page "DualPipe и EPLB: конвейер в обе стороны и балансировщик
+экспертов" (EPLB README translation with the eplb.py appendix) and the LPLB
+usage example (page "DeepSeek开源LPLB：基于线性规划的MoE负载均衡器").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import NamedTuple, Optional
+
+import torch
+
+__all__ = [
+    "EplbError", "Plan", "count_loads", "window_accumulate", "rebalance", "redirect",
+    "default_slots", "lib_path", "load_library", "STATUS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libeplb.so")
+
+STATUS = {
+    0: "EPLB_OK", 1: "EPLB_ERR_NULL", 2: "EPLB_ERR_SHAPE", 3: "EPLB_ERR_DIVISIBILITY",
+    4: "EPLB_ERR_RANGE", 5: "EPLB_ERR_SLOTS", 6: "EPLB_ERR_CUDA", 7: "EPLB_ERR_TIMEOUT",
+    8: "EPLB_ERR_ALIGN", 9: "EPLB_ERR_LIMIT",
+}
+
+
+class EplbError(RuntimeError):
+    """A non-zero eplb_status returned by the C ABI (or read from a status word)."""
+
+    def __init__(self, code: int, where: str, detail: str = ""):
+        self.code = int(code)
+        msg = f"{where}: {STATUS.get(self.code, self.code)}"
+        super().__init__(msg + (f" ({detail})" if detail else ""))
+
+
+class Plan(NamedTuple):
+    phy2log: torch.Tensor   # int32 [R, P]
+    phyrank: torch.Tensor   # int32 [R, P]
+    logcnt: torch.Tensor    # int32 [R, E]
+    log2phy: torch.Tensor   # int32 [R, E, X]
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libeplb.so (built by ``python -m moe_expert_load_eplb_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m moe_expert_load_eplb_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
+    sig = {
+        "eplb_status_string": ([i32], ctypes.c_char_p),
+        "eplb_last_cuda_error": ([], ctypes.c_char_p),
+        "eplb_abi_version": ([], i32),
+        "eplb_count_loads": ([p, i64, i64, i32, i32, p, i32, p, p, p], i32),
+        "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, p, p], i32),
+        "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p], i32),
+        "eplb_redirect": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, p], i32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        detail = load_library().eplb_last_cuda_error().decode() if code == 6 else ""
+        raise EplbError(code, where, detail)
+
+
+def _cuda(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def count_loads(idx: torch.Tensor, num_experts: int, counts: Optional[torch.Tensor] = None,
+                accumulate: bool = False, bad: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """S1: counts[l, e] (+)= #{(t, k): idx[l, t, k] == e} for int32 idx [L, T, K]."""
+    _cuda(idx, torch.int32, "idx")
+    if idx.dim() != 3:
+        raise ValueError("idx must be [L, T, K]")
+    L, T, K = idx.shape
+    if counts is None:
+        counts = torch.empty((L, num_experts), dtype=torch.int64, device=idx.device)
+        accumulate = False
+    _cuda(counts, torch.int64, "counts")
+    if tuple(counts.shape) != (L, num_experts):
+        raise ValueError("counts must be [L, E]")
+    with torch.cuda.device(idx.device):
+        _check(load_library().eplb_count_loads(
+            _ptr(idx), L, T, K, num_experts, _ptr(counts), int(bool(accumulate)),
+            _ptr(bad), _ptr(status), _stream(idx.device)), "eplb_count_loads")
+    return counts
+
+
+def window_accumulate(steps: torch.Tensor, window: int, s_first: int = 0,
+                      out: Optional[torch.Tensor] = None,
+                      status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """S2: out[s - s_first] = sum of steps[max(0, s-window+1) .. s] (int64 [S, L, E])."""
+    _cuda(steps, torch.int64, "steps")
+    if steps.dim() != 3:
+        raise ValueError("steps must be [S, L, E]")
+    S, L, E = steps.shape
+    if out is None:
+        out = torch.empty((max(S - s_first, 0), L, E), dtype=torch.int64, device=steps.device)
+    _cuda(out, torch.int64, "out")
+    if tuple(out.shape) != (S - s_first, L, E):
+        raise ValueError("out must be [S - s_first, L, E]")
+    with torch.cuda.device(steps.device):
+        _check(load_library().eplb_window_accumulate(
+            _ptr(steps), S, L, E, window, s_first, _ptr(out), _ptr(status),
+            _stream(steps.device)), "eplb_window_accumulate")
+    return out
+
+
+def default_slots(num_logical: int, num_replicas: int, num_groups: int, num_nodes: int) -> int:
+    """log2phy width that always suffices: the most replicas one expert can get."""
+    nodes = num_nodes if num_nodes > 0 and num_groups % num_nodes == 0 else 1
+    return max(1, (num_replicas - num_logical) // nodes + 1)
+
+
+def rebalance(loads: torch.Tensor, num_replicas: int, num_groups: int, num_nodes: int,
+              num_gpus: int, slots: Optional[int] = None, out: Optional[Plan] = None,
+              status: Optional[torch.Tensor] = None) -> Plan:
+    """S3/S4: rebalance_experts for every row of int64 loads [R, E] (hierarchical
+    policy when num_groups % num_nodes == 0, else global)."""
+    _cuda(loads, torch.int64, "loads")
+    if loads.dim() != 2:
+        raise ValueError("loads must be [R, E]")
+    R, E = loads.shape
+    P = num_replicas
+    X = default_slots(E, P, num_groups, num_nodes) if slots is None else slots
+    dev = loads.device
+    if out is None:
+        out = Plan(torch.empty((R, P), dtype=torch.int32, device=dev),
+                   torch.empty((R, P), dtype=torch.int32, device=dev),
+                   torch.empty((R, E), dtype=torch.int32, device=dev),
+                   torch.empty((R, E, X), dtype=torch.int32, device=dev))
+    for name, t, shape in (("phy2log", out.phy2log, (R, P)), ("phyrank", out.phyrank, (R, P)),
+                           ("logcnt", out.logcnt, (R, E)), ("log2phy", out.log2phy, (R, E, X))):
+        _cuda(t, torch.int32, name)
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be {shape}")
+    with torch.cuda.device(dev):
+        _check(load_library().eplb_rebalance(
+            _ptr(loads), R, E, P, num_groups, num_nodes, num_gpus, X,
+            _ptr(out.phy2log), _ptr(out.phyrank), _ptr(out.logcnt), _ptr(out.log2phy),
+            _ptr(status), _stream(dev)), "eplb_rebalance")
+    return out
+
+
+def redirect(idx: torch.Tensor, log2phy: torch.Tensor, logcnt: torch.Tensor, token_offset: int = 0,
+             out: Optional[torch.Tensor] = None, bad: Optional[torch.Tensor] = None,
+             status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """S5: out[l, t, k] = log2phy[l, e, (token_offset + t) mod logcnt[l, e]], e = idx[l, t, k]."""
+    _cuda(idx, torch.int32, "idx")
+    _cuda(log2phy, torch.int32, "log2phy")
+    _cuda(logcnt, torch.int32, "logcnt")
+    if idx.dim() != 3 or log2phy.dim() != 3 or logcnt.dim() != 2:
+        raise ValueError("idx [L, T, K], log2phy [L, E, X], logcnt [L, E] expected")
+    L, T, K = idx.shape
+    _, E, X = log2phy.shape
+    if log2phy.shape[0] != L or tuple(logcnt.shape) != (L, E):
+        raise ValueError("table shapes do not match idx")
+    if out is None:
+        out = torch.empty_like(idx)
+    _cuda(out, torch.int32, "out")
+    if out.shape != idx.shape:
+        raise ValueError("out must match idx")
+    with torch.cuda.device(idx.device):
+        _check(load_library().eplb_redirect(
+            _ptr(idx), L, T, K, E, _ptr(log2phy), X, _ptr(logcnt), int(token_offset),
+            _ptr(out), _ptr(bad), _ptr(status), _stream(idx.device)), "eplb_redirect")
+    return out

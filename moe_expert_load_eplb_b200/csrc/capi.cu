@@ -1,0 +1,168 @@
+// capi.cu -- the exported C ABI of libeplb.so: argument checks, policy
+// choice and launches.  Declarations and contracts are in include/eplb.h.
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace eplb {
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_once[kMaxDevices];
+DeviceInfo g_info[kMaxDevices];
+bool g_ok[kMaxDevices];
+
+thread_local char g_last_error[256] = "no error";
+
+int bit_width(int64_t v) {  // bits needed to write v >= 0 (0 -> 0)
+  int b = 0;
+  while (v > 0) {
+    ++b;
+    v >>= 1;
+  }
+  return b;
+}
+
+int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+bool device_info(DeviceInfo *out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::call_once(g_once[dev], [dev]() {
+    DeviceInfo d;
+    g_ok[dev] = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+                cudaDeviceGetAttribute(&d.max_smem_optin,
+                                       cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
+    g_info[dev] = d;
+  });
+  *out = g_info[dev];
+  return g_ok[dev];
+}
+
+eplb_status cuda_fail(cudaError_t err) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(err),
+                cudaGetErrorString(err));
+  return EPLB_ERR_CUDA;
+}
+
+}  // namespace eplb
+
+using namespace eplb;
+
+extern "C" {
+
+const char *eplb_status_string(int32_t status) {
+  switch (status) {
+    case EPLB_OK: return "EPLB_OK";
+    case EPLB_ERR_NULL: return "EPLB_ERR_NULL";
+    case EPLB_ERR_SHAPE: return "EPLB_ERR_SHAPE";
+    case EPLB_ERR_DIVISIBILITY: return "EPLB_ERR_DIVISIBILITY";
+    case EPLB_ERR_RANGE: return "EPLB_ERR_RANGE";
+    case EPLB_ERR_SLOTS: return "EPLB_ERR_SLOTS";
+    case EPLB_ERR_CUDA: return "EPLB_ERR_CUDA";
+    case EPLB_ERR_TIMEOUT: return "EPLB_ERR_TIMEOUT";
+    case EPLB_ERR_ALIGN: return "EPLB_ERR_ALIGN";
+    case EPLB_ERR_LIMIT: return "EPLB_ERR_LIMIT";
+    default: return "EPLB_ERR_UNKNOWN";
+  }
+}
+
+const char *eplb_last_cuda_error(void) { return g_last_error; }
+
+int32_t eplb_abi_version(void) { return (1 << 16) | 0; }
+
+eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                             int64_t *counts, int32_t accumulate, unsigned long long *bad,
+                             int32_t *status, cudaStream_t stream) {
+  if (L < 0 || T < 0 || K < 1 || E < 1) return EPLB_ERR_SHAPE;
+  if (E > 1024 || T > (int64_t(1) << 31) / K) return EPLB_ERR_LIMIT;
+  if (L == 0) return EPLB_OK;
+  if (counts == nullptr) return EPLB_ERR_NULL;
+  if (T > 0 && idx == nullptr) return EPLB_ERR_NULL;
+  if (T > 0 && !aligned16(idx)) return EPLB_ERR_ALIGN;
+  if (!accumulate) {
+    const cudaError_t err =
+        cudaMemsetAsync(counts, 0, static_cast<size_t>(L) * E * sizeof(int64_t), stream);
+    if (err != cudaSuccess) return cuda_fail(err);
+  }
+  if (T == 0) return EPLB_OK;
+  return launch_count_loads(idx, L, T * K, E, counts, bad, status, stream);
+}
+
+eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, int32_t E,
+                                   int64_t W, int64_t s_first, int64_t *snaps, int32_t *status,
+                                   cudaStream_t stream) {
+  (void)status;
+  if (S < 0 || L < 0 || E < 1 || W < 1 || s_first < 0) return EPLB_ERR_SHAPE;
+  if (S == 0 || L == 0) return s_first == 0 ? EPLB_OK : EPLB_ERR_SHAPE;
+  if (s_first >= S) return EPLB_ERR_SHAPE;
+  if (steps == nullptr || snaps == nullptr) return EPLB_ERR_NULL;
+  const int64_t C = L * E;
+  if (C > (int64_t(1) << 34)) return EPLB_ERR_LIMIT;
+  return launch_window(steps, S, C, W, s_first, snaps, stream);
+}
+
+eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P, int32_t G,
+                           int32_t N, int32_t gpus, int32_t X, int32_t *phy2log,
+                           int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
+                           cudaStream_t stream) {
+  if (R < 0 || E < 1 || P < 1 || G < 1 || N < 1 || gpus < 1 || X < 1) return EPLB_ERR_SHAPE;
+  if (P < E) return EPLB_ERR_SHAPE;
+  if (E > 1024 || P > 2048 || R > 0x7fffffffLL) return EPLB_ERR_LIMIT;
+  if (E % G != 0 || P % gpus != 0) return EPLB_ERR_DIVISIBILITY;
+  RebalanceShape sh;
+  sh.E = E;
+  sh.P = P;
+  sh.gpus = gpus;
+  sh.X = X;
+  if (G % N == 0) {  // hierarchical policy
+    if (gpus % N != 0) return EPLB_ERR_DIVISIBILITY;
+    sh.G = G;
+    sh.N = N;
+  } else {  // global policy: one group on one node
+    sh.G = 1;
+    sh.N = 1;
+  }
+  if (static_cast<int64_t>(E) * X > (int64_t(1) << 26)) return EPLB_ERR_LIMIT;
+  sh.gs = E / sh.G;
+  sh.gpn = sh.G / sh.N;
+  sh.lpn = E / sh.N;
+  sh.ppn = P / sh.N;
+  sh.ppg = P / gpus;
+  sh.mpn = gpus / sh.N;
+  sh.npad = next_pow2(sh.ppn);
+  sh.gpad = next_pow2(sh.G);
+  sh.ibits = bit_width(sh.ppn);
+  sh.qbits = bit_width(sh.mpn - 1);
+  sh.gibits = bit_width(sh.G);
+  sh.nqbits = bit_width(sh.N - 1);
+  if (R == 0) return EPLB_OK;
+  if (!loads || !phy2log || !phyrank || !logcnt || !log2phy) return EPLB_ERR_NULL;
+  return launch_rebalance(loads, R, sh, phy2log, phyrank, logcnt, log2phy, status, stream);
+}
+
+eplb_status eplb_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                          const int32_t *log2phy, int32_t X, const int32_t *logcnt, int64_t t0,
+                          int32_t *out, unsigned long long *bad, int32_t *status,
+                          cudaStream_t stream) {
+  if (L < 0 || T < 0 || K < 1 || E < 1 || X < 1 || t0 < 0) return EPLB_ERR_SHAPE;
+  if (E > 1024 || static_cast<int64_t>(E) * X > 32768) return EPLB_ERR_LIMIT;
+  if (T >= (int64_t(1) << 31) / K || t0 + T >= (int64_t(1) << 31)) return EPLB_ERR_LIMIT;
+  if (L == 0 || T == 0) return EPLB_OK;
+  if (!idx || !log2phy || !logcnt || !out) return EPLB_ERR_NULL;
+  if (!aligned16(idx) || !aligned16(out)) return EPLB_ERR_ALIGN;
+  return launch_redirect(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, status, stream);
+}
+
+}  // extern "C"

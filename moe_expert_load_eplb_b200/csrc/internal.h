@@ -1,0 +1,46 @@
+// internal.h -- launchers behind the C ABI (host side, not exported).
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/eplb.h"
+
+namespace eplb {
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem_optin = 0;
+};
+
+// Cached per device; returns false when the runtime query fails.
+bool device_info(DeviceInfo *out);
+
+// Records a CUDA error message for eplb_last_cuda_error() and maps it.
+eplb_status cuda_fail(cudaError_t err);
+
+eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer, int32_t E,
+                               int64_t *counts, unsigned long long *bad, int32_t *status,
+                               cudaStream_t stream);
+
+eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
+                          int64_t *snaps, cudaStream_t stream);
+
+struct RebalanceShape {
+  int32_t E, P, G, N, gpus, X;   // G, N after the policy choice
+  int32_t gs, gpn, lpn, ppn, ppg, mpn;
+  int32_t npad, gpad;
+  int32_t ibits, qbits, gibits, nqbits;
+};
+
+eplb_status launch_rebalance(const int64_t *loads, int64_t R, const RebalanceShape &sh,
+                             int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
+                             int32_t *log2phy, int32_t *status, cudaStream_t stream);
+
+eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                            const int32_t *log2phy, int32_t X, const int32_t *logcnt, int64_t t0,
+                            int32_t *out, unsigned long long *bad, int32_t *status,
+                            cudaStream_t stream);
+
+}  // namespace eplb

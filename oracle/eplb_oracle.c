@@ -252,22 +252,21 @@ static int rebalance_hierarchical_row(const int64_t *weight, int E, int P,
     const int *cnt = mlogcnt + n * lpn;
 
     /* step 3: replicas -> GPUs of node n, load of replica j is
-       tokens_per_mlog[phy2mlog[j]] / cnt[phy2mlog[j]], scaled by LAMBDA */
-    i128 lambda = 1;
-    for (int i = 0; i < lpn; ++i) {
-      lambda = lambda / gcd128(lambda, cnt[i]) * cnt[i];
-      if (lambda > ((i128)1 << 62)) { rc = ORACLE_ERR_RANGE; goto done; }
-    }
-    int64_t wmax = 0;
-    for (int i = 0; i < lpn; ++i) if (tokens_per_mlog[i] > wmax) wmax = tokens_per_mlog[i];
-    /* every pack sum must stay below 2^126 */
-    if ((i128)wmax * lambda > (((i128)1) << 126) / (ppg > 0 ? ppg : 1)) {
-      rc = ORACLE_ERR_RANGE;
-      goto done;
-    }
-    for (int j = 0; j < ppn; ++j) {
-      int i = phy2mlog[j];
-      tokens_per_phy[j] = (i128)tokens_per_mlog[i] * (lambda / cnt[i]);
+       tokens_per_mlog[phy2mlog[j]] / cnt[phy2mlog[j]], scaled by LAMBDA.
+       With one replica per GPU balanced_packing returns the identity
+       without reading the loads, so they are not formed then.  A row whose
+       LAMBDA exceeds 2^62 cannot be held exactly and is rejected. */
+    for (int j = 0; j < ppn; ++j) tokens_per_phy[j] = 0;
+    if (ppg > 1) {
+      i128 lambda = 1;
+      for (int i = 0; i < lpn; ++i) {
+        lambda = lambda / gcd128(lambda, cnt[i]) * cnt[i];
+        if (lambda > ((i128)1 << 62)) { rc = ORACLE_ERR_RANGE; goto done; }
+      }
+      for (int j = 0; j < ppn; ++j) {
+        int i = phy2mlog[j];
+        tokens_per_phy[j] = (i128)tokens_per_mlog[i] * (lambda / cnt[i]);
+      }
     }
     rc = balanced_packing(tokens_per_phy, ppn, gpus_per_node, pack, rank_in_pack);
     if (rc) goto done;

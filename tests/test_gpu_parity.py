@@ -1,0 +1,386 @@
+"""GPU parity: every CUDA stage against the CPU oracle, bit for bit.
+
+All comparisons are exact (integer and index work).  Inputs come from the
+seeded generators in ``workloads``; the oracle consumes the same bytes copied
+to the host.  Calls go through the C ABI (ctypes binding).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests._invariants import check_plan
+
+pytestmark = pytest.mark.gpu
+
+eplb = pytest.importorskip("moe_expert_load_eplb_b200")
+DEV = "cuda:0"
+
+
+def _np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().numpy()
+
+
+def _status():
+    return torch.zeros(1, dtype=torch.int32, device=DEV)
+
+
+def _oracle_rows(loads_np, P, G, N, gpus, X):
+    """Oracle plan; rows the oracle rejects as not exactly representable
+    (status RANGE) come back as error rows (-1 / 0), the GPU's convention."""
+    try:
+        return oracle.rebalance(loads_np, P, G, N, gpus, slots=X), 0
+    except oracle.OracleError as err:
+        if err.code != oracle.ERR_RANGE:
+            raise
+    R, E = loads_np.shape
+    out = [np.full((R, P), -1, np.int32), np.full((R, P), -1, np.int32),
+           np.zeros((R, E), np.int32), np.full((R, E, X), -1, np.int32)]
+    for r in range(R):
+        try:
+            row = oracle.rebalance(loads_np[r:r + 1], P, G, N, gpus, slots=X)
+        except oracle.OracleError as err:
+            assert err.code == oracle.ERR_RANGE
+            continue
+        for o, x in zip(out, row):
+            o[r] = x[0]
+    return tuple(out), oracle.ERR_RANGE
+
+
+def _rebalance_both(loads_np, P, G, N, gpus, slots=None):
+    loads = torch.from_numpy(np.ascontiguousarray(loads_np)).to(DEV)
+    st = _status()
+    plan = eplb.rebalance(loads, P, G, N, gpus, slots=slots, status=st)
+    torch.cuda.synchronize()
+    ref, ref_status = _oracle_rows(np.ascontiguousarray(loads_np, dtype=np.int64), P, G, N, gpus,
+                                   plan.log2phy.shape[2])
+    got_status = int(st.item())
+    assert got_status == ref_status, (got_status, ref_status)
+    return plan, ref, got_status
+
+
+def _assert_plan_equal(plan, ref):
+    for name, got, want in zip(("phy2log", "phyrank", "logcnt", "log2phy"), plan, ref):
+        g = _np(got)
+        if not np.array_equal(g, want):
+            bad = np.argwhere(g != want)
+            raise AssertionError(f"{name} differs at {len(bad)} places, first {bad[:5].tolist()}")
+
+
+# ---------------------------------------------------------------- fixtures --
+
+@pytest.fixture(scope="module")
+def c1_idx():
+    return W.c1_indices(device=DEV)
+
+
+@pytest.fixture(scope="module")
+def c2_idx():
+    return W.routed_indices(2, device=DEV)
+
+
+@pytest.fixture(scope="module")
+def c5_idx():
+    torch.cuda.empty_cache()
+    return W.routed_indices(5, device=DEV)
+
+
+# ------------------------------------------------------------------ count --
+
+@pytest.mark.parametrize("cfg", [1, 2, 5])
+def test_count_configs(cfg, request):
+    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
+    E = W.CONFIGS[cfg].E
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    counts = eplb.count_loads(idx, E, bad=bad)
+    ref, nbad = oracle.count_loads(_np(idx), E)
+    assert np.array_equal(_np(counts), ref)
+    assert int(bad.item()) == nbad == 0
+    assert int(counts.sum()) == idx.numel()
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 1001, 3), (2, 4097, 8), (5, 3, 7), (4, 4096, 1),
+                                   (1, 70001, 5), (2, 0, 8), (7, 12345, 2)])
+@pytest.mark.parametrize("E", [1, 12, 256, 1024])
+def test_count_ragged_and_bad(shape, E):
+    L, T, K = shape
+    g = torch.Generator(device=DEV).manual_seed(L * 131 + T * 7 + K + E)
+    idx = torch.randint(-2, E + 2, (L, T, K), generator=g, device=DEV, dtype=torch.int32)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    counts = eplb.count_loads(idx, E, bad=bad)
+    ref, nbad = oracle.count_loads(_np(idx), E)
+    assert np.array_equal(_np(counts), ref)
+    assert int(bad.item()) == nbad
+    again = eplb.count_loads(idx, E, counts=counts, accumulate=True, bad=bad)
+    assert np.array_equal(_np(again), 2 * ref)
+    assert int(bad.item()) == 2 * nbad
+
+
+def test_count_skewed_single_expert():
+    # every index equal: the worst case for same-address atomics
+    idx = torch.full((3, 50000, 8), 7, dtype=torch.int32, device=DEV)
+    counts = eplb.count_loads(idx, 256)
+    ref, _ = oracle.count_loads(_np(idx), 256)
+    assert np.array_equal(_np(counts), ref)
+
+
+def test_count_misaligned_pointer_rejected():
+    base = torch.zeros(1 + 4 * 16, dtype=torch.int32, device=DEV)
+    with pytest.raises(eplb.EplbError) as e:
+        eplb.count_loads(base[1:].view(1, 16, 4), 8)
+    assert e.value.code == 8
+
+
+# ----------------------------------------------------------------- window --
+
+@pytest.fixture(scope="module")
+def c4_steps():
+    return W.c4_steps(device=DEV)
+
+
+@pytest.mark.parametrize("window", [1000, 128, 1])
+def test_window_c4(c4_steps, window):
+    snaps = eplb.window_accumulate(c4_steps, window)
+    ref = oracle.window(_np(c4_steps), window)
+    assert np.array_equal(_np(snaps), ref)
+
+
+@pytest.mark.parametrize("S,L,E,window,s_first", [(1, 1, 1, 1, 0), (7, 3, 5, 2, 0), (100, 2, 12, 7, 0),
+                                                  (33, 1, 1, 100, 10), (65, 58, 256, 16, 64),
+                                                  (16, 58, 256, 16, 15), (300, 3, 3, 40, 299),
+                                                  (129, 5, 77, 64, 1)])
+def test_window_shapes(S, L, E, window, s_first):
+    g = torch.Generator(device=DEV).manual_seed(S * 1000 + E)
+    steps = torch.randint(0, 1 << 40, (S, L, E), generator=g, device=DEV, dtype=torch.int64)
+    snaps = eplb.window_accumulate(steps, window, s_first=s_first)
+    ref = oracle.window(_np(steps), window, s_first)
+    assert np.array_equal(_np(snaps), ref)
+
+
+# -------------------------------------------------------------- rebalance --
+
+def test_rebalance_readme_example():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "eplb_readme_example.json")) as f:
+        ex = json.load(f)
+    w = np.array(ex["weight"], dtype=np.int64)
+    for G in (4, 3):
+        plan, ref, st = _rebalance_both(w, 16, G, 2, 8)
+        assert st == 0
+        _assert_plan_equal(plan, ref)
+    plan, _, _ = _rebalance_both(w, 16, 4, 2, 8)
+    assert _np(plan.phy2log).tolist() == ex["phy2log"]["value"]
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 5])
+def test_rebalance_on_counted_loads(cfg, request):
+    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
+    c = W.CONFIGS[cfg]
+    loads = _np(eplb.count_loads(idx, c.E))
+    plan, ref, st = _rebalance_both(loads, c.P, c.G, c.N, c.gpus)
+    assert st == 0
+    _assert_plan_equal(plan, ref)
+    check_plan(loads[:4], *(p[:4] for p in ref), c.P, c.G, c.N, c.gpus)
+
+
+def test_rebalance_c3_global():
+    c = W.CONFIGS[3]
+    loads = W.c3_loads()
+    plan, ref, st = _rebalance_both(loads, c.P, c.G, c.N, c.gpus)
+    assert st == 0
+    _assert_plan_equal(plan, ref)
+
+
+def test_rebalance_c4_sweep(c4_steps):
+    c = W.CONFIGS[4]
+    snaps = eplb.window_accumulate(c4_steps, c.W)
+    loads = _np(snaps).reshape(-1, c.E)
+    plan, ref, st = _rebalance_both(loads, c.P, c.G, c.N, c.gpus)
+    assert st == 0
+    _assert_plan_equal(plan, ref)
+
+
+SHAPES = [
+    (12, 4, 16, 2, 8), (12, 3, 16, 2, 8), (16, 4, 16, 2, 4), (16, 4, 32, 4, 8), (8, 2, 16, 2, 16),
+    (24, 6, 36, 3, 6), (256, 8, 288, 4, 32), (256, 1, 288, 2, 144), (64, 8, 96, 8, 16),
+    (1, 1, 1, 1, 1), (1, 1, 64, 1, 4), (2, 2, 2, 2, 2), (1024, 32, 2048, 8, 64), (1024, 1, 1024, 1, 1),
+    (384, 12, 448, 4, 64), (160, 10, 200, 5, 40), (128, 16, 160, 16, 32), (256, 8, 320, 1, 160),
+    (96, 3, 2048, 2, 8), (300, 5, 602, 7, 7),
+]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("dist", ["uniform", "ties", "zeros", "huge", "skew", "onehot"])
+def test_rebalance_shapes(shape, dist):
+    E, G, P, N, gpus = shape
+    rng = np.random.default_rng(abs(hash((E, G, P, N, gpus))) % (1 << 31) + len(dist))
+    R = 5
+    if dist == "uniform":
+        w = rng.integers(0, 5000, (R, E))
+    elif dist == "ties":
+        w = rng.integers(0, 3, (R, E)) * 12
+    elif dist == "zeros":
+        w = np.zeros((R, E), dtype=np.int64)
+    elif dist == "huge":
+        w = rng.integers((1 << 40) - 100000, 1 << 40, (R, E))
+    elif dist == "skew":
+        w = np.round(1e4 * (rng.pareto(1.1, (R, E)) + 1)).astype(np.int64)
+    else:
+        w = np.zeros((R, E), dtype=np.int64)
+        w[np.arange(R), rng.integers(0, E, R)] = (1 << 40) - 1
+    plan, ref, st = _rebalance_both(w.astype(np.int64), P, G, N, gpus)
+    assert st in (0, 4)
+    _assert_plan_equal(plan, ref)
+
+
+def _random_shape(rng):
+    while True:
+        N = int(rng.choice([1, 2, 3, 4, 5, 8]))
+        hier = rng.random() < 0.7
+        G = N * int(rng.integers(1, 5)) if hier else int(rng.choice([3, 5, 7, 9])) * (1 if N == 1 else 1)
+        if not hier and G % N == 0:
+            G += 1
+        gs = int(rng.integers(1, 9))
+        E = G * gs
+        gpus = (N if hier else 1) * int(rng.integers(1, 9))
+        ppg = int(rng.integers(1, 6))
+        P = gpus * ppg
+        while P < E:
+            P += gpus
+        if E <= 1024 and P <= 2048:
+            return E, G, P, N, gpus
+
+
+@pytest.mark.parametrize("seed", range(60))
+def test_rebalance_fuzz(seed):
+    rng = np.random.default_rng(1000 + seed)
+    E, G, P, N, gpus = _random_shape(rng)
+    R = int(rng.integers(1, 6))
+    kind = seed % 4
+    if kind == 0:
+        w = rng.integers(0, 100, (R, E))
+    elif kind == 1:
+        w = rng.integers(0, 1 << 40, (R, E))
+    elif kind == 2:
+        w = rng.integers(0, 4, (R, E)) * int(rng.integers(1, 1000))
+    else:
+        w = np.round(1e3 * (rng.pareto(1.2, (R, E)) + 1)).astype(np.int64)
+    plan, ref, st = _rebalance_both(w.astype(np.int64), P, G, N, gpus)
+    assert st in (0, 4), (E, G, P, N, gpus)
+    _assert_plan_equal(plan, ref)
+
+
+def test_rebalance_range_error_row():
+    w = np.full((3, 12), 10, dtype=np.int64)
+    w[1, 5] = 1 << 40
+    loads = torch.from_numpy(w).to(DEV)
+    st = _status()
+    plan = eplb.rebalance(loads, 16, 4, 2, 8, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+    assert (_np(plan.phy2log[1]) == -1).all() and (_np(plan.logcnt[1]) == 0).all()
+    ref, code = _oracle_rows(w, 16, 4, 2, 8, plan.log2phy.shape[2])
+    assert code == 4
+    _assert_plan_equal(plan, ref)
+
+
+def test_rebalance_slots_error():
+    w = np.array([[1000, 1, 1, 1]], dtype=np.int64)
+    loads = torch.from_numpy(w).to(DEV)
+    st = _status()
+    plan = eplb.rebalance(loads, 8, 1, 1, 4, slots=2, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 5
+    ref = oracle.rebalance(w, 8, 1, 1, 4)  # full width
+    assert np.array_equal(_np(plan.phy2log), ref[0])
+    assert np.array_equal(_np(plan.log2phy), ref[3][:, :, :2])
+
+
+def test_rebalance_host_errors():
+    loads = torch.ones((1, 12), dtype=torch.int64, device=DEV)
+    for args, code in [((16, 5, 2, 8), 3), ((18, 4, 2, 8), 3), ((8, 4, 2, 8), 2), ((16, 4, 4, 6), 3)]:
+        with pytest.raises(eplb.EplbError) as e:
+            eplb.rebalance(loads, *args)
+        assert e.value.code == code
+
+
+# --------------------------------------------------------------- redirect --
+
+@pytest.mark.parametrize("cfg", [1, 2, 5])
+def test_redirect_configs(cfg, request):
+    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
+    c = W.CONFIGS[cfg]
+    counts = eplb.count_loads(idx, c.E)
+    plan = eplb.rebalance(counts, c.P, c.G, c.N, c.gpus)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    st = _status()
+    out = eplb.redirect(idx, plan.log2phy, plan.logcnt, bad=bad, status=st)
+    ref, nbad = oracle.redirect(_np(idx), _np(plan.log2phy), _np(plan.logcnt))
+    assert np.array_equal(_np(out), ref)
+    assert int(bad.item()) == nbad == 0 and int(st.item()) == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 1001, 3), (2, 4097, 8), (5, 3, 7), (2, 70001, 5),
+                                   (1, 9999, 1), (4, 2048, 6)])
+@pytest.mark.parametrize("t0", [0, 17, (1 << 31) - 80000])
+def test_redirect_ragged(shape, t0):
+    L, T, K = shape
+    E, P, G, N, gpus = 24, 40, 6, 2, 4
+    rng = np.random.default_rng(L + T + K)
+    w = rng.integers(0, 1000, (L, E))
+    ref_plan = oracle.rebalance(w, P, G, N, gpus)
+    l2p = torch.from_numpy(ref_plan[3]).to(DEV)
+    cnt = torch.from_numpy(ref_plan[2]).to(DEV)
+    g = torch.Generator(device=DEV).manual_seed(T)
+    idx = torch.randint(-1, E + 1, (L, T, K), generator=g, device=DEV, dtype=torch.int32)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    out = eplb.redirect(idx, l2p, cnt, token_offset=t0, bad=bad)
+    ref, nbad = oracle.redirect(_np(idx), ref_plan[3], ref_plan[2], t0)
+    assert np.array_equal(_np(out), ref)
+    assert int(bad.item()) == nbad
+
+
+def test_redirect_invalid_logcnt_reports_range():
+    idx = torch.zeros((1, 8, 4), dtype=torch.int32, device=DEV)
+    l2p = torch.zeros((1, 4, 2), dtype=torch.int32, device=DEV)
+    cnt = torch.tensor([[0, 1, 3, 1]], dtype=torch.int32, device=DEV)
+    st = _status()
+    out = eplb.redirect(idx, l2p, cnt, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4 and (_np(out) == -1).all()
+
+
+def test_redirect_sharded_equals_whole(c2_idx):
+    c = W.CONFIGS[2]
+    counts = eplb.count_loads(c2_idx, c.E)
+    plan = eplb.rebalance(counts, c.P, c.G, c.N, c.gpus)
+    whole = eplb.redirect(c2_idx, plan.log2phy, plan.logcnt)
+    h = c.T // 2
+    a = eplb.redirect(c2_idx[:, :h].contiguous(), plan.log2phy, plan.logcnt, 0)
+    b = eplb.redirect(c2_idx[:, h:].contiguous(), plan.log2phy, plan.logcnt, h)
+    assert torch.equal(torch.cat([a, b], dim=1), whole)
+
+
+# --------------------------------------------------------------- pipeline --
+
+def test_pipeline_step_c2(c2_idx):
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+    c = W.CONFIGS[2]
+    hist = W.histogram_steps(15, c.L, c.E, c.T * c.K, 2, device=DEV)
+    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=16, device=DEV)
+    step.ring[:15].copy_(hist)
+    step.steps_done = 15
+    plan, out = step(c2_idx)
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    counts, _ = oracle.count_loads(_np(c2_idx), c.E)
+    ring = np.concatenate([_np(hist), counts[None]], axis=0)
+    loads = oracle.window(ring, 16, 15)[0]
+    ref = oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=step.X)
+    _assert_plan_equal(plan, ref)
+    red, _ = oracle.redirect(_np(c2_idx), ref[3], ref[2])
+    assert np.array_equal(_np(out), red)
