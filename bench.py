@@ -1,0 +1,395 @@
+"""Benchmark of the EPLB hot path on B200: one step = count -> window ->
+rebalance -> redirect over the DeepSeek-V3-shaped prefill workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (per rank): 58 MoE layers x 65,536 tokens x top-8 group-limited
+routed int32 indices over 256 experts in 8 groups (popularity log-normal,
+seeded, synthetic), a 16-step load window, plans of 288 physical experts
+over 4 nodes x 8 GPUs.  Metric: layer-rebalances per second of the whole
+step; the load-count and redirect kernels are reported against the measured
+HBM bandwidth.  Rank 0 prints one JSON line.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronisation; each step is timed on its stream with CUDA events
+(one between every two stages); L2 is flushed (a 512 MB write) between steps,
+outside the events.  With N > 1 (torchrun) every rank counts and redirects
+its own 65,536 tokens per layer and the per-step counts are summed with one
+NCCL all-reduce; every rank then computes the same plan.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+CFG = W.CONFIGS[2]
+WINDOW = 16
+METRIC = "EPLB layer-rebalances/sec on 1 B200 + load-count GB/s vs HBM peak"
+UNIT = "layer-rebalances/s"
+FLUSH_BYTES = 512 << 20
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def _config(world: int) -> dict:
+    return {"workload": CFG.name, "layers": CFG.L, "experts": CFG.E, "groups": CFG.G,
+            "replicas": CFG.P, "nodes": CFG.N, "plan_gpus": CFG.gpus,
+            "tokens_per_layer_per_rank": CFG.T, "top_k": CFG.K, "window": WINDOW,
+            "l2": "flushed between steps (512 MB write)", "parallelism": f"dp{world}"}
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    NAMES = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+             0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+             0x10: "sync_boost", 0x100: "display_clock"}
+
+    def __init__(self, device: int, period: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop, self.ok = period, threading.Event(), False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device)
+            uuid = getattr(props, "uuid", None)
+            h = None
+            if uuid is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    h = None
+            if h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+                phys = int(vis.split(",")[device]) if vis and vis.split(",")[device].isdigit() else device
+                h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.h, self.nv = h, pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.NAMES.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------- profiles --
+
+def _kernel_sha(name: str) -> str:
+    path = os.path.join(ROOT, "moe_expert_load_eplb_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def _traffic(kernel_file: str, profile: str, scale: float):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", profile)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != _kernel_sha(kernel_file):
+        return None
+    return float(m_b.group(1)) * scale
+
+
+# --------------------------------------------------------------------- ours --
+
+def run_ours(args, rank: int, world: int, group):
+    import moe_expert_load_eplb_b200 as eplb  # noqa: F401  (fails loudly without libeplb.so)
+    from moe_expert_load_eplb_b200 import count_loads, rebalance, redirect, window_accumulate
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    c = CFG
+    idx = W.routed_indices(2, device=dev, shard=rank)
+    hist = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K * world, 2, device=dev)
+    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=WINDOW, device=dev,
+                    token_offset=rank * c.T, group=group)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def one(i, marks=None):
+        row = step.ring[step.steps_done % WINDOW]
+        rec = (lambda k: marks[k].record()) if marks else (lambda k: None)
+        rec(0)
+        count_loads(idx, c.E, counts=row, bad=step.bad, status=step.status)
+        rec(1)
+        if group is not None:
+            torch.distributed.all_reduce(row, group=group)
+        rec(2)
+        window_accumulate(step.ring, WINDOW, s_first=WINDOW - 1, out=step.loads, status=step.status)
+        rec(3)
+        rebalance(step.loads[0], c.P, c.G, c.N, c.gpus, slots=step.X, out=step.plan, status=step.status)
+        rec(4)
+        redirect(idx, step.plan.log2phy, step.plan.logcnt, step.token_offset, out=step.out,
+                 bad=step.bad, status=step.status)
+        rec(5)
+        step.steps_done += 1
+
+    step.ring[:WINDOW - 1].copy_(hist)
+    step.steps_done = WINDOW - 1
+    for i in range(args.warmup):
+        flush.fill_(i & 0xff)
+        one(i)
+    torch.cuda.synchronize()
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {eplb.STATUS.get(int(step.status.item()))} in warm-up")
+
+    K = args.steps
+    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
+    if group is not None:
+        torch.distributed.barrier(group=group)
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        for i in range(K):
+            flush.fill_(i & 0xff)
+            one(i, marks[i])
+        torch.cuda.synchronize()
+    if group is not None:
+        torch.distributed.barrier(group=group)
+    if int(step.status.item()) != 0:
+        raise RuntimeError(f"device status {eplb.STATUS.get(int(step.status.item()))}")
+
+    stage_names = ["count", "allreduce", "window", "rebalance", "redirect"]
+    per_stage = {n: [] for n in stage_names}
+    totals = []
+    for m in marks:
+        for k, n in enumerate(stage_names):
+            per_stage[n].append(m[k].elapsed_time(m[k + 1]))
+        totals.append(m[0].elapsed_time(m[5]))
+    total_ms = torch.tensor([sum(totals)], dtype=torch.float64, device=dev)
+    if group is not None:
+        torch.distributed.all_reduce(total_ms, op=torch.distributed.ReduceOp.MAX, group=group)
+    total_ms = float(total_ms.item())
+    ms_per_step = total_ms / K
+    value = c.L * K / (total_ms / 1e3)
+
+    hbm_peak, peak_kind = _peaks()
+    n_idx = c.L * c.T * c.K
+    algo = {"count": 4.0 * n_idx, "redirect": 8.0 * n_idx,
+            "window": 8.0 * WINDOW * c.L * c.E + 8.0 * c.L * c.E,
+            "rebalance": 8.0 * c.L * c.E + 4.0 * c.L * (2 * c.P + c.E + c.E * step.X)}
+    stages = {}
+    for n in ["count", "window", "rebalance", "redirect"] + (["allreduce"] if group is not None else []):
+        ms = statistics.mean(per_stage[n])
+        d = {"ms": round(ms, 5)}
+        if n in algo:
+            gbs = algo[n] / (ms / 1e3) / 1e9 if ms > 0 else None
+            d["algo_bytes"] = algo[n]
+            d["gbs"] = round(gbs, 1) if gbs else None
+            if n in ("count", "redirect", "window"):
+                d["frac_hbm"] = round(gbs / hbm_peak, 4) if gbs else None
+        stages[n] = d
+    stages["rebalance"]["rows_per_s"] = round(c.L / (stages["rebalance"]["ms"] / 1e3), 1)
+    stages["rebalance"]["us_per_call"] = round(stages["rebalance"]["ms"] * 1e3, 2)
+
+    dominant = max(["count", "window", "rebalance", "redirect"], key=lambda n: stages[n]["ms"])
+    if dominant in ("count", "redirect", "window"):
+        kfile = {"count": "count.cu", "redirect": "redirect.cu", "window": "window.cu"}[dominant]
+        roof = {"kernel": dominant, "bound": "hbm", "achieved": stages[dominant]["gbs"],
+                "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": stages[dominant]["frac_hbm"],
+                "traffic": _traffic(kfile, f"{dominant}_dsv3_prefill.md", 1.0)}
+    else:
+        roof = {"kernel": "rebalance", "bound": "alu", "achieved": None, "peak": None,
+                "unit": "GB/s", "frac": None, "traffic": None}
+
+    out = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+           "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+           "data": "synthetic (seeded group-limited routing, log-normal popularity)",
+           "config": _config(world), "gpu_launches": 4 * K,
+           "tokens_per_s": round(world * c.T * K / (total_ms / 1e3), 1),
+           "load_count_gbs": stages["count"]["gbs"],
+           "load_count_frac_hbm": stages["count"]["frac_hbm"],
+           "stages": stages, "roofline": roof, "clocks": clocks.summary()}
+
+    # ---- e2e: the same step through the public API with host buffers ------
+    Ke = max(5, min(K, 50))
+    idx_host = idx.cpu().pin_memory()
+    out_host = torch.empty(step.out.shape, dtype=torch.int32).pin_memory()
+    plan_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.plan]
+    idx_dev = torch.empty_like(idx)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+    if group is not None:
+        torch.distributed.barrier(group=group)
+    torch.cuda.synchronize()
+    for i in range(Ke):
+        flush.fill_(i & 0xff)
+        ev[i][0].record()
+        idx_dev.copy_(idx_host, non_blocking=True)
+        step(idx_dev)
+        out_host.copy_(step.out, non_blocking=True)
+        for h, d in zip(plan_host, step.plan):
+            h.copy_(d, non_blocking=True)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
+    if group is not None:
+        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX, group=group)
+    e2e_ms = float(e2e_ms.item())
+    out["e2e"] = {"value": round(c.L * Ke / (e2e_ms / 1e3), 1), "unit": UNIT,
+                  "h2d_bytes_per_step": idx.numel() * 4,
+                  "d2h_bytes_per_step": out_host.numel() * 4 + sum(t.numel() * 4 for t in plan_host),
+                  "steps": Ke, "ms_per_step": round(e2e_ms / Ke, 4)}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(idx.cpu().numpy(), hist.cpu().numpy(), args.cpu_seconds)
+    return out
+
+
+# ------------------------------------------------------------ the oracle --
+
+def _oracle_step(idx_h, hist_h, layers):
+    """One step of the oracle on the first `layers` layers: count, window,
+    rebalance, redirect (the same work per layer as the GPU step)."""
+    import numpy as np
+    import oracle
+    c = CFG
+    sub = idx_h[:layers]
+    counts, _ = oracle.count_loads(sub, c.E)
+    ring = np.concatenate([hist_h[:, :layers], counts[None]], axis=0)
+    loads = oracle.window(ring, WINDOW, WINDOW - 1)[0]
+    X = (c.P - c.E) // c.N + 1
+    plan = oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=X)
+    oracle.redirect(sub, plan[3], plan[2])
+
+
+def cpu_baseline(idx_h, hist_h, seconds: float):
+    _oracle_step(idx_h, hist_h, 1)  # load / build the oracle library outside the timing
+    n, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_step(idx_h, hist_h, CFG.L)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": round(CFG.L * n / el, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} full steps (58 layers x 65,536 tokens x top-8: count, 16-step window, "
+                      f"rebalance, redirect), single-thread plain C, {el:.1f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle timed as the reference arm on this host's cores."""
+    c = CFG
+    idx_h = W.routed_indices(2, device="cpu", T=c.T).numpy()
+    hist_h = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K, 2).numpy()
+    t0 = time.perf_counter()
+    _oracle_step(idx_h, hist_h, 1)
+    t_layer = max(time.perf_counter() - t0, 1e-4)
+    budget = 60.0
+    layers = int(max(1, min(c.L, budget / ((args.steps + args.warmup) * t_layer))))
+    for _ in range(args.warmup):
+        _oracle_step(idx_h, hist_h, layers)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(idx_h, hist_h, layers)
+    el = time.perf_counter() - t0
+    value = layers * args.steps / el
+    sample = (f"{layers} of 58 layers per step (count, 16-step window, rebalance, redirect over "
+              f"65,536 tokens x top-8 each), single-thread plain C oracle")
+    return {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+            "config": _config(1), "impl": "reference",
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = _args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    torch.cuda.set_device(local)
+    group = None
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+        group = torch.distributed.group.WORLD
+    try:
+        res = run_ours(args, rank, world, group)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if group is not None:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -117,12 +117,15 @@ def group_limited_indices(popularity: torch.Tensor, T: int, K: int, G: int, grou
     return out
 
 
-def routed_indices(config: int, device="cpu", T: int | None = None, L: int | None = None) -> torch.Tensor:
+def routed_indices(config: int, device="cpu", T: int | None = None, L: int | None = None,
+                   shard: int = 0) -> torch.Tensor:
     """Routed indices of configs 2 and 5 (optionally with fewer tokens / layers).
 
     Config 2: popularity LogNormal(mu=0, sigma=1) per expert per layer.
     Config 5: popularity ∝ rank^-1.0 (Zipf s=1.0) through a seeded permutation.
-    Both: 8 groups of 32, 4 groups per token, top-8.
+    Both: 8 groups of 32, 4 groups per token, top-8.  ``shard`` selects an
+    independent token stream with the same popularity (one per data-parallel
+    rank).
     """
     c = CONFIGS[config]
     L = c.L if L is None else L
@@ -135,7 +138,8 @@ def routed_indices(config: int, device="cpu", T: int | None = None, L: int | Non
         pop = torch.stack([base[torch.randperm(c.E, generator=g)] for _ in range(L)])
     else:
         raise ValueError("routed indices exist for configs 2 and 5")
-    return group_limited_indices(pop.float(), T, c.K, c.G, 4, seed_for(config, 0), device)
+    return group_limited_indices(pop.float(), T, c.K, c.G, 4, seed_for(config, 0) + 100000 * shard,
+                                 device)
 
 
 def c3_loads(L: int = 58, E: int = 256) -> np.ndarray:
