@@ -162,47 +162,12 @@ def _traffic(kernel_file: str, profile: str, scale: float):
 
 # --------------------------------------------------------------------- ours --
 
-def run_ours(args, rank: int, world: int, group):
-    import moe_expert_load_eplb_b200 as eplb  # noqa: F401  (fails loudly without libeplb.so)
-    from moe_expert_load_eplb_b200 import count_loads, rebalance, redirect, window_accumulate
-    from moe_expert_load_eplb_b200.pipeline import EplbStep
+STAGES = ("count", "allreduce", "window", "rebalance", "redirect")
 
-    dev = torch.device("cuda", torch.cuda.current_device())
-    c = CFG
-    idx = W.routed_indices(2, device=dev, shard=rank)
-    hist = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K * world, 2, device=dev)
-    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=WINDOW, device=dev,
-                    token_offset=rank * c.T, group=group)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
-    def one(i, marks=None):
-        row = step.ring[step.steps_done % WINDOW]
-        rec = (lambda k: marks[k].record()) if marks else (lambda k: None)
-        rec(0)
-        count_loads(idx, c.E, counts=row, bad=step.bad, status=step.status)
-        rec(1)
-        if group is not None:
-            torch.distributed.all_reduce(row, group=group)
-        rec(2)
-        window_accumulate(step.ring, WINDOW, s_first=WINDOW - 1, out=step.loads, status=step.status)
-        rec(3)
-        rebalance(step.loads[0], c.P, c.G, c.N, c.gpus, slots=step.X, out=step.plan, status=step.status)
-        rec(4)
-        redirect(idx, step.plan.log2phy, step.plan.logcnt, step.token_offset, out=step.out,
-                 bad=step.bad, status=step.status)
-        rec(5)
-        step.steps_done += 1
-
-    step.ring[:WINDOW - 1].copy_(hist)
-    step.steps_done = WINDOW - 1
-    for i in range(args.warmup):
-        flush.fill_(i & 0xff)
-        one(i)
-    torch.cuda.synchronize()
-    if int(step.status.item()) != 0:
-        raise RuntimeError(f"device status {eplb.STATUS.get(int(step.status.item()))} in warm-up")
-
-    K = args.steps
+def _timed_steps(step, idx, flush, K, group, dev):
+    """Runs K steps with events between stages; returns (total ms max over
+    ranks, per-stage mean ms, clock summary)."""
     marks = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
     if group is not None:
         torch.distributed.barrier(group=group)
@@ -210,74 +175,133 @@ def run_ours(args, rank: int, world: int, group):
     with ClockSampler(dev.index) as clocks:
         for i in range(K):
             flush.fill_(i & 0xff)
-            one(i, marks[i])
+            step(idx, marks[i])
         torch.cuda.synchronize()
     if group is not None:
         torch.distributed.barrier(group=group)
-    if int(step.status.item()) != 0:
-        raise RuntimeError(f"device status {eplb.STATUS.get(int(step.status.item()))}")
-
-    stage_names = ["count", "allreduce", "window", "rebalance", "redirect"]
-    per_stage = {n: [] for n in stage_names}
-    totals = []
-    for m in marks:
-        for k, n in enumerate(stage_names):
-            per_stage[n].append(m[k].elapsed_time(m[k + 1]))
-        totals.append(m[0].elapsed_time(m[5]))
-    total_ms = torch.tensor([sum(totals)], dtype=torch.float64, device=dev)
+    per_stage = {n: statistics.mean(m[k].elapsed_time(m[k + 1]) for m in marks)
+                 for k, n in enumerate(STAGES)}
+    total = torch.tensor([sum(m[0].elapsed_time(m[5]) for m in marks)], dtype=torch.float64,
+                         device=dev)
     if group is not None:
-        torch.distributed.all_reduce(total_ms, op=torch.distributed.ReduceOp.MAX, group=group)
-    total_ms = float(total_ms.item())
+        torch.distributed.all_reduce(total, op=torch.distributed.ReduceOp.MAX, group=group)
+    return float(total.item()), per_stage, clocks.summary()
+
+
+def _stage_report(per_stage, fused, X, world, hbm_peak):
+    c = CFG
+    n_idx = c.L * c.T * c.K
+    algo = {"window": 8.0 * WINDOW * c.L * c.E + 8.0 * c.L * c.E,
+            "rebalance": 8.0 * c.L * c.E + 4.0 * c.L * (2 * c.P + c.E + c.E * X)}
+    if fused:
+        algo["count"] = 8.0 * n_idx + 8.0 * c.L * c.E  # indices in, physical indices + counts out
+    else:
+        algo["count"] = 4.0 * n_idx
+        algo["redirect"] = 8.0 * n_idx
+    stages = {}
+    names = ["count", "window", "rebalance"] + ([] if fused else ["redirect"])
+    names += ["allreduce"] if world > 1 else []
+    for n in names:
+        ms = per_stage[n]
+        d = {"ms": round(ms, 5)}
+        if n in algo and ms > 0:
+            gbs = algo[n] / (ms / 1e3) / 1e9
+            d.update(algo_bytes=algo[n], gbs=round(gbs, 1))
+            if n != "rebalance":
+                d["frac_hbm"] = round(gbs / hbm_peak, 4)
+        stages[n] = d
+    if fused:
+        stages["count"]["kernel"] = "count_redirect (S1+S5 fused)"
+    stages["rebalance"]["us_per_call"] = round(per_stage["rebalance"] * 1e3, 2)
+    stages["rebalance"]["rows_per_s"] = round(c.L / (per_stage["rebalance"] / 1e3), 1)
+    return stages
+
+
+def run_ours(args, rank: int, world: int, group):
+    import moe_expert_load_eplb_b200 as eplb
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    c = CFG
+    idx = W.routed_indices(2, device=dev, shard=rank)
+    hist = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K * world, 2, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    hbm_peak, peak_kind = _peaks()
+
+    def make(fused):
+        st = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=WINDOW, device=dev,
+                      token_offset=rank * c.T, group=group, fused=fused)
+        st.fill_history(hist)
+        return st
+
+    def check(st, where):
+        torch.cuda.synchronize()
+        code = int(st.status.item())
+        if code != 0:
+            raise RuntimeError(f"device status {eplb.STATUS.get(code)} in {where}")
+
+    # ---- the timed step: serving order (count+redirect fused, then plan) ----
+    step = make(True)
+    for i in range(args.warmup):
+        flush.fill_(i & 0xff)
+        step(idx)
+    check(step, "warm-up")
+    K = args.steps
+    total_ms, per_stage, clocks = _timed_steps(step, idx, flush, K, group, dev)
+    check(step, "timed steps")
     ms_per_step = total_ms / K
     value = c.L * K / (total_ms / 1e3)
+    stages = _stage_report(per_stage, True, step.X, world, hbm_peak)
 
-    hbm_peak, peak_kind = _peaks()
-    n_idx = c.L * c.T * c.K
-    algo = {"count": 4.0 * n_idx, "redirect": 8.0 * n_idx,
-            "window": 8.0 * WINDOW * c.L * c.E + 8.0 * c.L * c.E,
-            "rebalance": 8.0 * c.L * c.E + 4.0 * c.L * (2 * c.P + c.E + c.E * step.X)}
-    stages = {}
-    for n in ["count", "window", "rebalance", "redirect"] + (["allreduce"] if group is not None else []):
-        ms = statistics.mean(per_stage[n])
-        d = {"ms": round(ms, 5)}
-        if n in algo:
-            gbs = algo[n] / (ms / 1e3) / 1e9 if ms > 0 else None
-            d["algo_bytes"] = algo[n]
-            d["gbs"] = round(gbs, 1) if gbs else None
-            if n in ("count", "redirect", "window"):
-                d["frac_hbm"] = round(gbs / hbm_peak, 4) if gbs else None
-        stages[n] = d
-    stages["rebalance"]["rows_per_s"] = round(c.L / (stages["rebalance"]["ms"] / 1e3), 1)
-    stages["rebalance"]["us_per_call"] = round(stages["rebalance"]["ms"] * 1e3, 2)
-
-    dominant = max(["count", "window", "rebalance", "redirect"], key=lambda n: stages[n]["ms"])
-    if dominant in ("count", "redirect", "window"):
-        kfile = {"count": "count.cu", "redirect": "redirect.cu", "window": "window.cu"}[dominant]
-        roof = {"kernel": dominant, "bound": "hbm", "achieved": stages[dominant]["gbs"],
+    dominant = max(("count", "window", "rebalance"), key=lambda n: stages[n]["ms"])
+    if dominant == "count":
+        roof = {"kernel": "count_redirect", "bound": "hbm", "achieved": stages["count"]["gbs"],
                 "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                "frac": stages[dominant]["frac_hbm"],
-                "traffic": _traffic(kfile, f"{dominant}_dsv3_prefill.md", 1.0)}
+                "frac": stages["count"]["frac_hbm"],
+                "traffic": _traffic("redirect.cu", "count_redirect_dsv3_prefill.md", 1.0)}
+    elif dominant == "window":
+        roof = {"kernel": "window", "bound": "hbm", "achieved": stages["window"]["gbs"],
+                "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": stages["window"]["frac_hbm"],
+                "traffic": _traffic("window.cu", "window_dsv3_prefill.md", 1.0)}
     else:
         roof = {"kernel": "rebalance", "bound": "alu", "achieved": None, "peak": None,
-                "unit": "GB/s", "frac": None, "traffic": None}
+                "unit": None, "frac": None, "traffic": None}
 
     out = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
            "data": "synthetic (seeded group-limited routing, log-normal popularity)",
-           "config": _config(world), "gpu_launches": 4 * K,
+           "config": dict(_config(world), step_order="serving: count+redirect with the plan in "
+                          "force (fused, one pass over the indices) -> window -> rebalance"),
+           "gpu_launches": step.launches_per_step * K,
            "tokens_per_s": round(world * c.T * K / (total_ms / 1e3), 1),
-           "load_count_gbs": stages["count"]["gbs"],
-           "load_count_frac_hbm": stages["count"]["frac_hbm"],
-           "stages": stages, "roofline": roof, "clocks": clocks.summary()}
+           "stages": stages, "roofline": roof, "clocks": clocks}
 
-    # ---- e2e: the same step through the public API with host buffers ------
+    # ---- the same four stages in the fresh-plan order, for comparison -----
+    fresh = make(False)
+    for i in range(max(3, args.warmup // 4)):
+        flush.fill_(i & 0xff)
+        fresh(idx)
+    check(fresh, "fresh-order warm-up")
+    Kf = max(3, min(K, 500))
+    f_total, f_stage, _ = _timed_steps(fresh, idx, flush, Kf, group, dev)
+    check(fresh, "fresh-order steps")
+    fstages = _stage_report(f_stage, False, fresh.X, world, hbm_peak)
+    out["fresh_order"] = {"steps": Kf, "ms_per_step": round(f_total / Kf, 5),
+                          "value": round(c.L * Kf / (f_total / 1e3), 1), "stages": fstages}
+    out["load_count_gbs"] = fstages["count"]["gbs"]
+    out["load_count_frac_hbm"] = fstages["count"]["frac_hbm"]
+    del fresh
+
+    # ---- e2e: the serving step through the public API with host buffers --
     Ke = max(5, min(K, 50))
     idx_host = idx.cpu().pin_memory()
     out_host = torch.empty(step.out.shape, dtype=torch.int32).pin_memory()
     plan_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.plan]
     idx_dev = torch.empty_like(idx)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(Ke)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(Ke)]
     if group is not None:
         torch.distributed.barrier(group=group)
     torch.cuda.synchronize()
@@ -290,7 +314,7 @@ def run_ours(args, rank: int, world: int, group):
         for h, d in zip(plan_host, step.plan):
             h.copy_(d, non_blocking=True)
         ev[i][1].record()
-    torch.cuda.synchronize()
+    check(step, "e2e steps")
     e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
     if group is not None:
         torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX, group=group)
@@ -307,33 +331,41 @@ def run_ours(args, rank: int, world: int, group):
 
 # ------------------------------------------------------------ the oracle --
 
-def _oracle_step(idx_h, hist_h, layers):
-    """One step of the oracle on the first `layers` layers: count, window,
-    rebalance, redirect (the same work per layer as the GPU step)."""
+def _oracle_plan(hist_h, layers):
+    import numpy as np
+    import oracle
+    c = CFG
+    ring = np.concatenate([hist_h[:, :layers], np.zeros((1, layers, c.E), np.int64)], axis=0)
+    loads = oracle.window(ring, WINDOW, WINDOW - 1)[0]
+    return oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=(c.P - c.E) // c.N + 1)
+
+
+def _oracle_step(idx_h, hist_h, layers, plan):
+    """One serving step of the oracle on the first `layers` layers: count and
+    redirect with the plan in force, window, rebalance (the GPU step's work)."""
     import numpy as np
     import oracle
     c = CFG
     sub = idx_h[:layers]
     counts, _ = oracle.count_loads(sub, c.E)
+    oracle.redirect(sub, plan[3], plan[2])
     ring = np.concatenate([hist_h[:, :layers], counts[None]], axis=0)
     loads = oracle.window(ring, WINDOW, WINDOW - 1)[0]
-    X = (c.P - c.E) // c.N + 1
-    plan = oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=X)
-    oracle.redirect(sub, plan[3], plan[2])
+    return oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=(c.P - c.E) // c.N + 1)
 
 
 def cpu_baseline(idx_h, hist_h, seconds: float):
-    _oracle_step(idx_h, hist_h, 1)  # load / build the oracle library outside the timing
+    plan = _oracle_plan(hist_h, CFG.L)  # also loads the oracle library, outside the timing
     n, t0 = 0, time.perf_counter()
     while True:
-        _oracle_step(idx_h, hist_h, CFG.L)
+        _oracle_step(idx_h, hist_h, CFG.L, plan)
         n += 1
         el = time.perf_counter() - t0
         if el >= seconds:
             break
     return {"value": round(CFG.L * n / el, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{n} full steps (58 layers x 65,536 tokens x top-8: count, 16-step window, "
-                      f"rebalance, redirect), single-thread plain C, {el:.1f} s"}
+            "sample": f"{n} full serving steps (58 layers x 65,536 tokens x top-8: count and "
+                      f"redirect, 16-step window, rebalance), single-thread plain C, {el:.1f} s"}
 
 
 def run_reference(args):
@@ -341,20 +373,22 @@ def run_reference(args):
     c = CFG
     idx_h = W.routed_indices(2, device="cpu", T=c.T).numpy()
     hist_h = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K, 2).numpy()
+    plan1 = _oracle_plan(hist_h, 1)
     t0 = time.perf_counter()
-    _oracle_step(idx_h, hist_h, 1)
+    _oracle_step(idx_h, hist_h, 1, plan1)
     t_layer = max(time.perf_counter() - t0, 1e-4)
     budget = 60.0
     layers = int(max(1, min(c.L, budget / ((args.steps + args.warmup) * t_layer))))
+    plan = _oracle_plan(hist_h, layers)
     for _ in range(args.warmup):
-        _oracle_step(idx_h, hist_h, layers)
+        _oracle_step(idx_h, hist_h, layers, plan)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_step(idx_h, hist_h, layers)
+        _oracle_step(idx_h, hist_h, layers, plan)
     el = time.perf_counter() - t0
     value = layers * args.steps / el
-    sample = (f"{layers} of 58 layers per step (count, 16-step window, rebalance, redirect over "
-              f"65,536 tokens x top-8 each), single-thread plain C oracle")
+    sample = (f"{layers} of 58 layers per step (count and redirect 65,536 tokens x top-8, "
+              f"16-step window, rebalance), single-thread plain C oracle")
     return {"metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(el / args.steps * 1e3, 4), "higher_is_better": True,

@@ -154,6 +154,22 @@ eplb_status eplb_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, i
                           int64_t t0, int32_t *out, unsigned long long *bad,
                           int32_t *status, cudaStream_t stream);
 
+/*
+ * S1 + S5 fused -- count the loads of a batch and redirect it in one pass over
+ * its indices (each index read from HBM once: 8 bytes per index instead of
+ * 4 + 8).  Same contracts as eplb_count_loads for idx / counts / accumulate /
+ * bad and as eplb_redirect for log2phy / X / logcnt / t0 / out / status; an
+ * index outside [0, E) is added to *bad once.  This is the serving order the
+ * EPLB pages describe ([EPLB] "Алгоритм": the plan comes from a moving
+ * average of past loads): the tables are the plan in force, built from
+ * earlier steps, while this batch's counts feed the next plan.
+ * Limits:  those of both calls.
+ */
+eplb_status eplb_count_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                                int64_t *counts, int32_t accumulate, const int32_t *log2phy,
+                                int32_t X, const int32_t *logcnt, int64_t t0, int32_t *out,
+                                unsigned long long *bad, int32_t *status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -24,7 +24,7 @@ from typing import NamedTuple, Optional
 import torch
 
 __all__ = [
-    "EplbError", "Plan", "count_loads", "window_accumulate", "rebalance", "redirect",
+    "EplbError", "Plan", "count_loads", "window_accumulate", "rebalance", "redirect", "count_redirect",
     "default_slots", "lib_path", "load_library", "STATUS",
 ]
 
@@ -79,6 +79,7 @@ def load_library():
         "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, p, p], i32),
         "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p], i32),
         "eplb_redirect": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, p], i32),
+        "eplb_count_redirect": ([p, i64, i64, i32, i32, p, i32, p, i32, p, i64, p, p, p, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -212,3 +213,38 @@ def redirect(idx: torch.Tensor, log2phy: torch.Tensor, logcnt: torch.Tensor, tok
             _ptr(idx), L, T, K, E, _ptr(log2phy), X, _ptr(logcnt), int(token_offset),
             _ptr(out), _ptr(bad), _ptr(status), _stream(idx.device)), "eplb_redirect")
     return out
+
+
+def count_redirect(idx: torch.Tensor, num_experts: int, log2phy: torch.Tensor, logcnt: torch.Tensor,
+                   token_offset: int = 0, counts: Optional[torch.Tensor] = None,
+                   accumulate: bool = False, out: Optional[torch.Tensor] = None,
+                   bad: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None):
+    """S1 + S5 in one pass over idx: counts (+)= histogram of idx and
+    out = redirect(idx, log2phy, logcnt, token_offset).  Returns (counts, out)."""
+    _cuda(idx, torch.int32, "idx")
+    _cuda(log2phy, torch.int32, "log2phy")
+    _cuda(logcnt, torch.int32, "logcnt")
+    if idx.dim() != 3 or log2phy.dim() != 3 or logcnt.dim() != 2:
+        raise ValueError("idx [L, T, K], log2phy [L, E, X], logcnt [L, E] expected")
+    L, T, K = idx.shape
+    _, E, X = log2phy.shape
+    if E != num_experts or log2phy.shape[0] != L or tuple(logcnt.shape) != (L, E):
+        raise ValueError("table shapes do not match idx / num_experts")
+    if counts is None:
+        counts = torch.empty((L, E), dtype=torch.int64, device=idx.device)
+        accumulate = False
+    _cuda(counts, torch.int64, "counts")
+    if tuple(counts.shape) != (L, E):
+        raise ValueError("counts must be [L, E]")
+    if out is None:
+        out = torch.empty_like(idx)
+    _cuda(out, torch.int32, "out")
+    if out.shape != idx.shape:
+        raise ValueError("out must match idx")
+    with torch.cuda.device(idx.device):
+        _check(load_library().eplb_count_redirect(
+            _ptr(idx), L, T, K, E, _ptr(counts), int(bool(accumulate)), _ptr(log2phy), X,
+            _ptr(logcnt), int(token_offset), _ptr(out), _ptr(bad), _ptr(status),
+            _stream(idx.device)), "eplb_count_redirect")
+    return counts, out

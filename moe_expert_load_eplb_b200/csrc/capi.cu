@@ -147,6 +147,21 @@ eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P
   sh.qbits = bit_width(sh.mpn - 1);
   sh.gibits = bit_width(sh.G);
   sh.nqbits = bit_width(sh.N - 1);
+  sh.cmax = sh.ppn - sh.lpn + 1;
+  {
+    unsigned __int128 lam = 1;
+    for (int c = 2; c <= sh.cmax && lam != 0; ++c) {
+      unsigned __int128 a = lam, b = static_cast<unsigned __int128>(c);
+      while (b != 0) {
+        const unsigned __int128 t = a % b;
+        a = b;
+        b = t;
+      }
+      lam = lam / a * c;
+      if (lam > (static_cast<unsigned __int128>(1) << 62)) lam = 0;
+    }
+    sh.lam_fixed = static_cast<uint64_t>(lam);
+  }
   if (R == 0) return EPLB_OK;
   if (!loads || !phy2log || !phyrank || !logcnt || !log2phy) return EPLB_ERR_NULL;
   return launch_rebalance(loads, R, sh, phy2log, phyrank, logcnt, log2phy, status, stream);
@@ -162,7 +177,29 @@ eplb_status eplb_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, i
   if (L == 0 || T == 0) return EPLB_OK;
   if (!idx || !log2phy || !logcnt || !out) return EPLB_ERR_NULL;
   if (!aligned16(idx) || !aligned16(out)) return EPLB_ERR_ALIGN;
-  return launch_redirect(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, status, stream);
+  return launch_redirect(idx, L, T, K, E, log2phy, X, logcnt, t0, out, nullptr, bad, status,
+                         stream);
+}
+
+eplb_status eplb_count_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                                int64_t *counts, int32_t accumulate, const int32_t *log2phy,
+                                int32_t X, const int32_t *logcnt, int64_t t0, int32_t *out,
+                                unsigned long long *bad, int32_t *status, cudaStream_t stream) {
+  if (L < 0 || T < 0 || K < 1 || E < 1 || X < 1 || t0 < 0) return EPLB_ERR_SHAPE;
+  if (E > 1024 || static_cast<int64_t>(E) * X > 32768) return EPLB_ERR_LIMIT;
+  if (T >= (int64_t(1) << 31) / K || t0 + T >= (int64_t(1) << 31)) return EPLB_ERR_LIMIT;
+  if (L == 0) return EPLB_OK;
+  if (counts == nullptr) return EPLB_ERR_NULL;
+  if (T > 0 && (!idx || !log2phy || !logcnt || !out)) return EPLB_ERR_NULL;
+  if (T > 0 && (!aligned16(idx) || !aligned16(out))) return EPLB_ERR_ALIGN;
+  if (!accumulate) {
+    const cudaError_t err =
+        cudaMemsetAsync(counts, 0, static_cast<size_t>(L) * E * sizeof(int64_t), stream);
+    if (err != cudaSuccess) return cuda_fail(err);
+  }
+  if (T == 0) return EPLB_OK;
+  return launch_redirect(idx, L, T, K, E, log2phy, X, logcnt, t0, out, counts, bad, status,
+                         stream);
 }
 
 }  // extern "C"

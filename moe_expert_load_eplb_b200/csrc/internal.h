@@ -32,15 +32,18 @@ struct RebalanceShape {
   int32_t gs, gpn, lpn, ppn, ppg, mpn;
   int32_t npad, gpad;
   int32_t ibits, qbits, gibits, nqbits;
+  int32_t cmax;                  // most replicas one expert can get: ppn - lpn + 1
+  uint64_t lam_fixed;            // lcm(1..cmax) when <= 2^62, else 0
 };
 
 eplb_status launch_rebalance(const int64_t *loads, int64_t R, const RebalanceShape &sh,
                              int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
                              int32_t *log2phy, int32_t *status, cudaStream_t stream);
 
+// Redirect; with counts != nullptr the same pass also adds the load histogram.
 eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
                             const int32_t *log2phy, int32_t X, const int32_t *logcnt, int64_t t0,
-                            int32_t *out, unsigned long long *bad, int32_t *status,
-                            cudaStream_t stream);
+                            int32_t *out, int64_t *counts, unsigned long long *bad,
+                            int32_t *status, cudaStream_t stream);
 
 }  // namespace eplb

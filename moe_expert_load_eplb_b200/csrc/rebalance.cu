@@ -10,19 +10,32 @@
 //           ties);
 //   step 3  replica loads w/c -> balanced_packing over the node's GPUs
 //           (P/gpus each); sums of w/c are held as integers w * (Lambda/c),
-//           Lambda = lcm of the node's replica counts;
+//           Lambda a common multiple of the node's replica counts;
 //   then the index bookkeeping and log2phy.
 // balanced_packing visits items heaviest first with ties by ascending index
 // and puts each into the lightest non-full pack (lowest pack index on ties).
 //
-// Latency-bound design: the row lives in shared memory; sorts are CTA-wide
-// bitonic networks on composite keys (load << b | (mask - index)), which
-// turns the stable (load desc, index asc) order into a plain descending sort
-// of distinct integers; each node's serial greedy chains run in one warp
-// (node n on warp n mod 4) as xor-butterfly argmax / argmin reductions with
-// no block-wide barrier per step.  Keys are 64-bit when the row's magnitudes
-// allow and 128-bit otherwise; both are exact, so the choice never changes
-// the result.
+// Latency-bound design, measured phase by phase with clock64 probes:
+//   * the row lives in shared memory; every sort key is a composite integer
+//     (load << b | (mask - index)), so the stable (load desc, index asc)
+//     order is a plain descending order of distinct integers;
+//   * sorts count ranks CTA-wide (a key's rank is the number of larger keys
+//     in its segment); threads are grouped by segment and rank several keys
+//     against each loaded key; segments longer than 512 use a bitonic network;
+//   * replicate_experts: an expert outside the top R = P/N - E/N experts of
+//     its node (by load, ties by index) has at least R quotients ahead of it,
+//     so it never gets an extra replica; the R candidates are selected by
+//     rank and the greedy runs on them alone -- in one lane's registers for
+//     R <= 8, one candidate per lane with an xor-butterfly argmax for R <= 32;
+//   * balanced_packing keeps a node's packs (<= 16) sorted by composite key
+//     (weight << 12 | pack) in one lane's registers: each item takes the
+//     first (lightest, lowest index) pack and re-inserts it with one parallel
+//     compare and two selects, with no shuffle, barrier or memory access on
+//     the chain; wider nodes use one warp per node and a butterfly argmin;
+//   * Lambda is lcm(1..cmax) from the host when 64-bit keys can hold it, else
+//     the lcm of the counts present in the node; keys are 64-bit when the
+//     row's magnitudes allow and 128-bit otherwise.  All paths are exact, so
+//     none changes the result.
 #include <algorithm>
 
 #include "common.cuh"
@@ -31,10 +44,21 @@
 namespace eplb {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kWarps = kThreads / 32;
+// CTA size is chosen per launch: 512 threads when there are few rows (each
+// row's parallel phases then spread over 4 warps per scheduler), 128 when
+// many rows share every SM.
+constexpr int kMaxThreads = 512;
+constexpr int kFewRowThreads = 512;
+constexpr int kManyRowThreads = 128;
+__device__ __forceinline__ int nthr() { return static_cast<int>(blockDim.x); }
+__device__ __forceinline__ int nwarps() { return static_cast<int>(blockDim.x) >> 5; }
 constexpr int64_t kLoadLimit = int64_t(1) << 40;
-constexpr uint32_t kNone = 0xffffffffu;
+constexpr int kRankSortMax = 512;        // longer segments use the bitonic network
+constexpr int kTableMaxEntries = 16384;  // log2phy rows up to this size are built in smem
+// Every composite key keeps an index (item, pack, group or expert, all < 4096)
+// in its low kIdxBits bits, so keys are combined with constant shifts only.
+constexpr int kIdxBits = 12;
+constexpr uint64_t kIdxMask = (uint64_t(1) << kIdxBits) - 1;
 
 typedef unsigned __int128 u128;
 
@@ -43,24 +67,40 @@ struct RbArgs {
   int32_t *phy2log, *phyrank, *logcnt, *log2phy, *status;
   RebalanceShape s;
   uint32_t x_magic;
+  int table_vec4;  // log2phy rows may be written as 16-byte vectors
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+__host__ __device__ inline int bitmap_words(const RebalanceShape &s) { return (s.cmax + 32) / 32; }
+__host__ __device__ inline bool table_in_smem(const RebalanceShape &s) {
+  return static_cast<int64_t>(s.E) * s.X <= kTableMaxEntries;
+}
+// experts per node that can receive extra replicas
+__host__ __device__ inline int num_cand(const RebalanceShape &s) {
+  return min(s.ppn - s.lpn, s.lpn);
+}
 
 // Shared-memory carve-up of one row (byte offsets), identical on host and device.
 struct Layout {
-  size_t keys, pw, w, wm, gkey, npw, lam, mlog2log, cnt, lc, p2m, rrank, ipack, irank, outp, outr,
-      gpack, grank, npc, pc, total;
+  size_t keys, sorted, pw, w, wm, gkey, gsorted, npw, lam, cand_w, table, mlog2log, cnt, lc, p2m,
+      rrank, ipack, irank, outp, outr, gpack, grank, npc, pc, cand_i, cand_c, bitmap, total;
   __host__ __device__ explicit Layout(const RebalanceShape &s) {
+    const int nc = num_cand(s);
     size_t o = 0;
-    keys = o; o += size_t(s.N) * s.npad * 16;  // u128 or u64 sort keys
-    pw = o; o += size_t(s.gpus) * 16;          // pack weights of step 3 (N * mpn)
+    keys = o; o += size_t(s.N) * max(s.npad, s.lpn) * 16;  // u128/u64 keys, stride npad (or lpn)
+    sorted = o; o += size_t(s.N) * s.npad * 16;
+    pw = o; o += size_t(s.gpus) * 16;                       // pack weights of the warp fallback
     o = align16(o);
     w = o; o += size_t(s.E) * 8;
     wm = o; o += size_t(s.E) * 8;
     gkey = o; o += size_t(s.gpad) * 8;
+    gsorted = o; o += size_t(s.gpad) * 8;
     npw = o; o += size_t(s.N) * 8;
     lam = o; o += size_t(s.N) * 8;
+    cand_w = o; o += size_t(s.N) * nc * 8;
+    o = align16(o);
+    table = o; o += table_in_smem(s) ? size_t(s.E) * s.X * 4 : 0;
+    o = align16(o);
     mlog2log = o; o += size_t(s.E) * 4;
     cnt = o; o += size_t(s.E) * 4;
     lc = o; o += size_t(s.E) * 4;
@@ -74,6 +114,9 @@ struct Layout {
     grank = o; o += size_t(s.G) * 4;
     npc = o; o += size_t(s.N) * 4;
     pc = o; o += size_t(s.gpus) * 4;
+    cand_i = o; o += size_t(s.N) * nc * 4;
+    cand_c = o; o += size_t(s.N) * nc * 4;
+    bitmap = o; o += size_t(s.N) * bitmap_words(s) * 4;
     total = align16(o);
   }
 };
@@ -86,16 +129,20 @@ __device__ __forceinline__ u128 shfl_xor(u128 v, int off) {
   const uint64_t hi = shfl_xor(static_cast<uint64_t>(v >> 64), off);
   return (static_cast<u128>(hi) << 64) | lo;
 }
+template <typename K>
+__device__ __forceinline__ K kmin(K a, K b) {
+  return b < a ? b : a;
+}
 
-__device__ __forceinline__ uint64_t gcd_u64(uint64_t a, uint64_t b) {  // binary gcd
+__device__ __forceinline__ uint32_t gcd_u32(uint32_t a, uint32_t b) {  // binary gcd
   if (a == 0) return b;
   if (b == 0) return a;
-  const int shift = __ffsll(static_cast<long long>(a | b)) - 1;
-  a >>= __ffsll(static_cast<long long>(a)) - 1;
+  const int shift = __ffs(a | b) - 1;
+  a >>= __ffs(a) - 1;
   do {
-    b >>= __ffsll(static_cast<long long>(b)) - 1;
+    b >>= __ffs(b) - 1;
     if (a > b) {
-      const uint64_t t = a;
+      const uint32_t t = a;
       a = b;
       b = t;
     }
@@ -104,27 +151,65 @@ __device__ __forceinline__ uint64_t gcd_u64(uint64_t a, uint64_t b) {  // binary
   return a << shift;
 }
 
-// lcm with overflow detection (results above 2^62 flag `ovf`).
-__device__ __forceinline__ uint64_t lcm_u64(uint64_t a, uint64_t b, bool &ovf) {
-  if (a == b || b <= 1) return a;
-  if (a <= 1) return b;
-  const uint64_t q = a / gcd_u64(a, b);
-  const u128 r = static_cast<u128>(q) * b;
-  if (r > (static_cast<u128>(1) << 62)) {
-    ovf = true;
-    return 1;
-  }
-  return static_cast<uint64_t>(r);
+// lcm(lam, c) with lam <= 2^62; false when the result would exceed 2^62.
+__device__ __forceinline__ bool lcm_into(uint64_t &lam, uint32_t c) {
+  if (c < 2) return true;
+  const uint32_t rem = lam >> 32 ? static_cast<uint32_t>(lam % c)
+                                 : static_cast<uint32_t>(lam) % c;
+  const uint32_t g = gcd_u32(rem, c);
+  const u128 next = static_cast<u128>(lam) * (c / g);
+  if (next > (static_cast<u128>(1) << 62)) return false;
+  lam = static_cast<uint64_t>(next);
+  return true;
 }
 
-// CTA-wide bitonic sort, descending, of nseg independent segments of npad
-// (power of two) keys each.  Ends with a barrier.
+// ---------------------------------------------------------------------------
+// Descending ranks of n distinct keys in each of nseg segments (segment g at
+// key + g * stride).  Threads are grouped by segment (nthr() / nseg per
+// segment); each ranks up to 4 keys per pass against every key it loads.
+// emit(g, j, rank, key) receives every key.
+template <typename K, typename Emit>
+__device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit emit) {
+  constexpr int Q = 4;
+  const int tps = nseg >= nthr() ? 1 : nthr() / nseg;
+  const int segs_per_pass = nthr() / tps;
+  const int sub = threadIdx.x % tps;
+  for (int g0 = 0; g0 < nseg; g0 += segs_per_pass) {
+    const int g = g0 + static_cast<int>(threadIdx.x) / tps;
+    if (static_cast<int>(threadIdx.x) / tps >= segs_per_pass || g >= nseg) continue;
+    const K *seg = key + g * stride;
+    for (int j0 = sub; j0 < n; j0 += tps * Q) {
+      K me[Q];
+      int r[Q];
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const int j = j0 + q * tps;
+        me[q] = j < n ? seg[j] : ~K(0);
+        r[q] = 0;
+      }
+#pragma unroll 4
+      for (int i = 0; i < n; ++i) {
+        const K kk = seg[i];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) r[q] += kk > me[q] ? 1 : 0;
+      }
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const int j = j0 + q * tps;
+        if (j < n) emit(g, j, r[q], me[q]);
+      }
+    }
+  }
+}
+
+// CTA-wide bitonic sort, descending, of nseg segments of npad (power of two)
+// keys each, in place; padding keys must be 0.
 template <typename K>
 __device__ void bitonic_desc(K *key, int npad, int nseg) {
   const int half = (npad * nseg) >> 1;
   for (int k = 2; k <= npad; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int t = threadIdx.x; t < half; t += kThreads) {
+      for (int t = threadIdx.x; t < half; t += nthr()) {
         const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1));
         const int p = i | j;
         const bool desc = ((i & (npad - 1)) & k) == 0;
@@ -139,117 +224,300 @@ __device__ void bitonic_desc(K *key, int npad, int nseg) {
   }
 }
 
-// balanced_packing's greedy, run by one warp over items already sorted as
-// composite keys (load << ibits | (imask - item)), descending.  Pack q is
-// owned by lane q % 32; each lane caches the composite key
-// (weight << qbits | q) of its lightest non-full pack and the warp takes
-// the minimum with an xor butterfly, so ties go to the lowest pack index.
+// ---------------------------------------------------------------------------
+// balanced_packing's greedy over items sorted as composite keys
+// (load << 12 | (4095 - item)), descending.  One lane runs one segment.
+// Its m <= MAXM packs are kept sorted ascending by ck = weight << 12 | pack
+// (all ones once full), with each pack's item count alongside; the lightest
+// non-full pack (lowest index on ties) is ck[0], and adding an item's load is
+// one 64- or 128-bit add of (key & ~4095).  After an item is added the pack
+// is re-inserted: lt[k] = ck[k] < new is a prefix, and slot i takes ck[i+1]
+// where lt[i+1], the new key where the prefix ends, else ck[i].
+template <typename K, int MAXM>
+__device__ void pack_lane(const K *skey, int n, int m, int cap, int32_t *ipack, int32_t *irank) {
+  if (n <= 0) return;
+  const K imask = K(kIdxMask);
+  const K kmax = ~K(0);
+  K ck[MAXM];
+  int pc[MAXM];
+#pragma unroll
+  for (int k = 0; k < MAXM; ++k) {
+    ck[k] = k < m ? K(k) : kmax;
+    pc[k] = 0;
+  }
+  K nxt = skey[0];
+  for (int j = 0; j < n; ++j) {
+    const K c = nxt;
+    if (j + 1 < n) nxt = skey[j + 1];
+    const K best = ck[0];
+    const int r = pc[0];
+    const K nk = r + 1 < cap ? best + (c & ~imask) : kmax;
+    bool lt[MAXM + 1];
+    lt[0] = true;
+    lt[MAXM] = false;
+#pragma unroll
+    for (int k = 1; k < MAXM; ++k) lt[k] = ck[k] < nk;
+#pragma unroll
+    for (int i = 0; i < MAXM; ++i) {
+      const bool here = lt[i] && !lt[i + 1];
+      const K up = i + 1 < MAXM ? ck[i + 1] : kmax;
+      const int upc = i + 1 < MAXM ? pc[i + 1] : 0;
+      ck[i] = lt[i + 1] ? up : (here ? nk : ck[i]);
+      pc[i] = lt[i + 1] ? upc : (here ? r + 1 : pc[i]);
+    }
+    const int item = static_cast<int>(imask - (c & imask));
+    ipack[item] = static_cast<int>(best & imask);
+    irank[item] = r;
+  }
+}
+
+// Same greedy for wide segments, one warp per segment: pack q is owned by
+// lane q % 32 (state in shared memory); each lane caches the composite key
+// of its lightest non-full pack; the warp takes the minimum with an xor
+// butterfly.
 template <typename K>
-__device__ void warp_pack(const K *skey, int n, int m, int cap, int ibits, int qbits, K *pw,
-                          int32_t *pc, int32_t *ipack, int32_t *irank) {
+__device__ void pack_warp(const K *skey, int n, int m, int cap, K *pw, int32_t *pc,
+                          int32_t *ipack, int32_t *irank) {
   const int lane = threadIdx.x & 31;
-  const K imask = (K(1) << ibits) - 1;
-  const K qmask = (K(1) << qbits) - 1;
+  const K imask = K(kIdxMask);
   const K kmax = ~K(0);
   for (int q = lane; q < m; q += 32) {
     pw[q] = 0;
     pc[q] = 0;
   }
   __syncwarp();
-  K best = lane < m ? K(lane) : kmax;  // every pack empty: lowest owned index
+  K best = lane < m ? K(lane) : kmax;
   int rounds = 0;
   while ((1 << rounds) < min(m, 32)) ++rounds;
   for (int j = 0; j < n; ++j) {
     const K ck = skey[j];
-    const K v = ck >> ibits;
-    const int item = static_cast<int>(imask - (ck & imask));
     K b = best;
-    for (int r = rounds - 1; r >= 0; --r) {
-      const K o = shfl_xor(b, 1 << r);
-      b = o < b ? o : b;
-    }
-    const int q = static_cast<int>(b & qmask);
+    for (int r = rounds - 1; r >= 0; --r) b = kmin(b, shfl_xor(b, 1 << r));
+    const int q = static_cast<int>(b & imask);
     if (b != kmax && lane == (q & 31)) {
       const int rk = pc[q];
       pc[q] = rk + 1;
-      pw[q] += v;
+      pw[q] += ck & ~imask;  // weights kept pre-shifted
+      const int item = static_cast<int>(imask - (ck & imask));
       ipack[item] = q;
       irank[item] = rk;
       K nb = kmax;
       for (int qq = lane; qq < m; qq += 32)
-        if (pc[qq] < cap) {
-          const K kk = (pw[qq] << qbits) | K(qq);
-          nb = kk < nb ? kk : nb;
-        }
+        if (pc[qq] < cap) nb = kmin(nb, pw[qq] | K(qq));
       best = nb;
     }
     __syncwarp();
   }
 }
 
-// a beats b in replicate_experts' argmax: larger w/c, then lower index.
-// ci packs (count << 16 | index); kNone marks "no candidate".
-__device__ __forceinline__ bool rep_better(int64_t aw, uint32_t aci, int64_t bw, uint32_t bci) {
-  if (aci == kNone) return false;
-  if (bci == kNone) return true;
-  const int64_t lhs = aw * static_cast<int64_t>(bci >> 16);
-  const int64_t rhs = bw * static_cast<int64_t>(aci >> 16);
-  return lhs > rhs || (lhs == rhs && (aci & 0xffffu) < (bci & 0xffffu));
+// Packs nseg segments (segment g: n sorted keys at skey + g * stride, results
+// at ipack/irank + g * out_stride) into m packs of cap items each.
+template <typename K>
+__device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
+                              int32_t *pc, int32_t *ipack, int32_t *irank, int out_stride) {
+  // 128-bit keys keep the register variant to 8 packs (register pressure)
+  if (m <= 8 || (m <= 16 && sizeof(K) == 8)) {
+    for (int g = threadIdx.x; g < nseg; g += nthr()) {
+      if (m <= 8)
+        pack_lane<K, 8>(skey + g * stride, n, m, cap, ipack + g * out_stride, irank + g * out_stride);
+      else
+        pack_lane<K, (sizeof(K) == 8 ? 16 : 8)>(skey + g * stride, n, m, cap, ipack + g * out_stride,
+                                                irank + g * out_stride);
+    }
+  } else {
+    for (int g = threadIdx.x >> 5; g < nseg; g += nwarps())
+      pack_warp<K>(skey + g * stride, n, m, cap, pw + g * m, pc + g * m, ipack + g * out_stride,
+                   irank + g * out_stride);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// replicate_experts.  a beats b on a larger w/c, then a lower index.
+__device__ __forceinline__ bool rep_better(int64_t aw, int ac, int ai, int64_t bw, int bc, int bi) {
+  const int64_t lhs = aw * static_cast<int64_t>(bc);
+  const int64_t rhs = bw * static_cast<int64_t>(ac);
+  return lhs > rhs || (lhs == rhs && ai < bi);
+}
+
+// D'Hondt form of the greedy: the extra replicas, in order, are the R best
+// (candidate k, divisor d) pairs by w_k / d desc, expert index asc, d asc
+// (each step takes the largest current quotient, and an expert's quotients
+// w/1, w/2, ... only decrease).  Pair (k, d) has at least k + d - 1 pairs
+// ahead of it (the k heavier candidates' first pairs and (k, 1 .. d-1)), so
+// only pairs with d <= R - k can be picked and only those are ranked.  All
+// pairs of all nodes are ranked in parallel; the picks need no serial chain.
+__device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
+                                const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
+                                int32_t *rrank) {
+  const int R = s.ppn - s.lpn, nc = num_cand(s);
+  const int grid = nc * R;
+  for (int t = threadIdx.x; t < s.N * grid; t += nthr()) {
+    const int n = t / grid;
+    const int p = t - n * grid;
+    const int k = p / R;
+    const int d = p - k * R + 1;
+    if (d > R - k) continue;
+    const int64_t w = cand_w[n * nc + k];
+    const int id = cand_i[n * nc + k];
+    int rank = 0;
+    for (int k2 = 0; k2 < nc; ++k2) {
+      const int64_t w2 = cand_w[n * nc + k2];
+      const int id2 = cand_i[n * nc + k2];
+      const bool lower = id2 < id, same = id2 == id;
+      for (int d2 = 1; d2 <= R - k2; ++d2) {
+        const int64_t lhs = w2 * d, rhs = w * d2;
+        rank += (lhs > rhs || (lhs == rhs && (lower || (same && d2 < d)))) ? 1 : 0;
+      }
+    }
+    if (rank < R) {
+      p2m[n * s.ppn + s.lpn + rank] = id;
+      rrank[n * s.ppn + s.lpn + rank] = d;
+      atomicAdd(&cand_c[n * nc + k], 1);
+    }
+  }
+}
+
+// Greedy over nc <= 32 candidates, one per lane of a warp.
+__device__ void replicate_warp(const RebalanceShape &s, int n, const int64_t *cand_w,
+                               const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
+                               int32_t *rrank) {
+  const int lane = threadIdx.x & 31;
+  const int nc = num_cand(s);
+  const int bp = n * s.ppn;
+  const bool valid = lane < nc;
+  const int64_t w = valid ? cand_w[n * nc + lane] : 0;
+  const int id = valid ? cand_i[n * nc + lane] : 0x7fffffff;
+  int c = 1;
+  int rounds = 0;
+  while ((1 << rounds) < min(nc, 32)) ++rounds;
+  for (int r = 0; r < s.ppn - s.lpn; ++r) {
+    int64_t bw = w;
+    int bc = c, bi = id, bl = lane;
+    for (int k = rounds - 1; k >= 0; --k) {
+      const int64_t ow = static_cast<int64_t>(shfl_xor(static_cast<uint64_t>(bw), 1 << k));
+      const int oc = __shfl_xor_sync(0xffffffffu, bc, 1 << k);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, 1 << k);
+      const int ol = __shfl_xor_sync(0xffffffffu, bl, 1 << k);
+      if (rep_better(ow, oc, oi, bw, bc, bi)) {
+        bw = ow;
+        bc = oc;
+        bi = oi;
+        bl = ol;
+      }
+    }
+    if (valid && lane == bl) {
+      p2m[bp + s.lpn + r] = id;
+      rrank[bp + s.lpn + r] = c;
+      ++c;
+    }
+  }
+  if (valid) cand_c[n * nc + lane] = c;
+  __syncwarp();
+}
+
+// Any number of candidates (all experts of the node), counts in shared memory.
+__device__ void replicate_smem(const RebalanceShape &s, int n, const int64_t *wm, int32_t *cnt,
+                               int32_t *p2m, int32_t *rrank) {
+  const int lane = threadIdx.x & 31;
+  const int bm = n * s.lpn, bp = n * s.ppn;
+  auto local_best = [&](int64_t &bw, int &bc, int &bi) {
+    bw = 0;
+    bc = 1;
+    bi = 0x7fffffff;
+    for (int i = lane; i < s.lpn; i += 32)
+      if (rep_better(wm[bm + i], cnt[bm + i], i, bw, bc, bi)) {
+        bw = wm[bm + i];
+        bc = cnt[bm + i];
+        bi = i;
+      }
+  };
+  int64_t bw;
+  int bc, bi;
+  local_best(bw, bc, bi);
+  for (int r = 0; r < s.ppn - s.lpn; ++r) {
+    int64_t mw = bw;
+    int mc = bc, mi = bi;
+    for (int k = 16; k >= 1; k >>= 1) {
+      const int64_t ow = static_cast<int64_t>(shfl_xor(static_cast<uint64_t>(mw), k));
+      const int oc = __shfl_xor_sync(0xffffffffu, mc, k);
+      const int oi = __shfl_xor_sync(0xffffffffu, mi, k);
+      if (rep_better(ow, oc, oi, mw, mc, mi)) {
+        mw = ow;
+        mc = oc;
+        mi = oi;
+      }
+    }
+    if (lane == (mi & 31)) {
+      cnt[bm + mi] = mc + 1;
+      p2m[bp + s.lpn + r] = mi;
+      rrank[bp + s.lpn + r] = mc;
+      local_best(bw, bc, bi);
+    }
+    __syncwarp();
+  }
 }
 
 __device__ void write_error_row(const RbArgs &a, int64_t row) {
   const RebalanceShape &s = a.s;
-  for (int t = threadIdx.x; t < s.P; t += kThreads) {
+  for (int t = threadIdx.x; t < s.P; t += nthr()) {
     a.phy2log[row * s.P + t] = -1;
     a.phyrank[row * s.P + t] = -1;
   }
-  for (int e = threadIdx.x; e < s.E; e += kThreads) a.logcnt[row * s.E + e] = 0;
+  for (int e = threadIdx.x; e < s.E; e += nthr()) a.logcnt[row * s.E + e] = 0;
   int32_t *gl = a.log2phy + row * static_cast<int64_t>(s.E) * s.X;
-  for (int i = threadIdx.x; i < s.E * s.X; i += kThreads) gl[i] = -1;
+  for (int i = threadIdx.x; i < s.E * s.X; i += nthr()) gl[i] = -1;
 }
 
 template <typename K>
-__device__ void step3_pack(const RbArgs &a, unsigned char *smem, const Layout &lay) {
+__device__ void step3(const RbArgs &a, unsigned char *smem, const Layout &lay) {
   const RebalanceShape &s = a.s;
   K *keys = reinterpret_cast<K *>(smem + lay.keys);
-  K *pw = reinterpret_cast<K *>(smem + lay.pw);
+  K *sorted = reinterpret_cast<K *>(smem + lay.sorted);
   const int64_t *wm = reinterpret_cast<const int64_t *>(smem + lay.wm);
   const uint64_t *lam = reinterpret_cast<const uint64_t *>(smem + lay.lam);
   const int32_t *cnt = reinterpret_cast<const int32_t *>(smem + lay.cnt);
   const int32_t *p2m = reinterpret_cast<const int32_t *>(smem + lay.p2m);
-  int32_t *pc = reinterpret_cast<int32_t *>(smem + lay.pc);
-  int32_t *ipack = reinterpret_cast<int32_t *>(smem + lay.ipack);
-  int32_t *irank = reinterpret_cast<int32_t *>(smem + lay.irank);
-  const K imask = (K(1) << s.ibits) - 1;
-  for (int t = threadIdx.x; t < s.N * s.npad; t += kThreads) {
-    const int n = t / s.npad;
-    const int j = t - n * s.npad;
+  const K imask = K(kIdxMask);
+  const bool ranked = s.npad <= kRankSortMax;
+  const int per = ranked ? s.ppn : s.npad;
+  for (int t = threadIdx.x; t < s.N * per; t += nthr()) {
+    const int n = t / per;
+    const int j = t - n * per;
     K key = 0;
     if (j < s.ppn) {
       const int m = n * s.lpn + p2m[n * s.ppn + j];
-      const K load = K(static_cast<uint64_t>(wm[m])) * K(lam[n] / static_cast<uint64_t>(cnt[m]));
-      key = (load << s.ibits) | (imask - K(j));
+      const uint32_t c = static_cast<uint32_t>(cnt[m]);
+      const uint64_t scale = c == 1 ? lam[n] : lam[n] / c;
+      key = ((K(static_cast<uint64_t>(wm[m])) * K(scale)) << kIdxBits) | (imask - K(j));
     }
-    keys[t] = key;
+    keys[n * s.npad + j] = key;
   }
   __syncthreads();
-  bitonic_desc<K>(keys, s.npad, s.N);
-  const int warp = threadIdx.x >> 5;
-  for (int n = warp; n < s.N; n += kWarps)
-    warp_pack<K>(keys + n * s.npad, s.ppn, s.mpn, s.ppg, s.ibits, s.qbits, pw + n * s.mpn,
-                 pc + n * s.mpn, ipack + n * s.ppn, irank + n * s.ppn);
+  const K *skeys = keys;
+  if (ranked) {
+    rank_segments<K>(keys, s.npad, s.N, s.ppn,
+                     [&](int g, int, int r, K k) { sorted[g * s.npad + r] = k; });
+    skeys = sorted;
+    __syncthreads();
+  } else {
+    bitonic_desc<K>(keys, s.npad, s.N);
+  }
+  pack_segments<K>(skeys, s.npad, s.N, s.ppn, s.mpn, s.ppg, reinterpret_cast<K *>(smem + lay.pw), reinterpret_cast<int32_t *>(smem + lay.pc),
+                   reinterpret_cast<int32_t *>(smem + lay.ipack),
+                   reinterpret_cast<int32_t *>(smem + lay.irank), s.ppn);
 }
 
-__global__ void __launch_bounds__(kThreads) rebalance_kernel(RbArgs a) {
+__global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  __shared__ int flags[2];  // [0] 128-bit keys needed, [1] exact ratio too wide
+  __shared__ int flags[2];  // [0] 128-bit keys needed, [1] exact ratio not representable
   const RebalanceShape &s = a.s;
   const Layout lay(s);
   int64_t *w = reinterpret_cast<int64_t *>(smem + lay.w);
   int64_t *wm = reinterpret_cast<int64_t *>(smem + lay.wm);
   uint64_t *gkey = reinterpret_cast<uint64_t *>(smem + lay.gkey);
-  uint64_t *npw = reinterpret_cast<uint64_t *>(smem + lay.npw);
+  uint64_t *gsorted = reinterpret_cast<uint64_t *>(smem + lay.gsorted);
   uint64_t *lam = reinterpret_cast<uint64_t *>(smem + lay.lam);
+  int64_t *cand_w = reinterpret_cast<int64_t *>(smem + lay.cand_w);
   int32_t *mlog2log = reinterpret_cast<int32_t *>(smem + lay.mlog2log);
   int32_t *cnt = reinterpret_cast<int32_t *>(smem + lay.cnt);
   int32_t *lc = reinterpret_cast<int32_t *>(smem + lay.lc);
@@ -261,11 +529,10 @@ __global__ void __launch_bounds__(kThreads) rebalance_kernel(RbArgs a) {
   int32_t *outr = reinterpret_cast<int32_t *>(smem + lay.outr);
   int32_t *gpack = reinterpret_cast<int32_t *>(smem + lay.gpack);
   int32_t *grank = reinterpret_cast<int32_t *>(smem + lay.grank);
-  int32_t *npc = reinterpret_cast<int32_t *>(smem + lay.npc);
+  int32_t *cand_i = reinterpret_cast<int32_t *>(smem + lay.cand_i);
+  int32_t *cand_c = reinterpret_cast<int32_t *>(smem + lay.cand_c);
 
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
   const int64_t row = blockIdx.x;
   if (tid == 0) {
     flags[0] = 0;
@@ -274,7 +541,7 @@ __global__ void __launch_bounds__(kThreads) rebalance_kernel(RbArgs a) {
 
   // ---- load the row; loads must lie in [0, 2^40) -------------------------
   bool bad = false;
-  for (int e = tid; e < s.E; e += kThreads) {
+  for (int e = tid; e < s.E; e += nthr()) {
     const int64_t x = __ldg(a.loads + row * s.E + e);
     w[e] = x;
     bad |= (x < 0) | (x >= kLoadLimit);
@@ -287,110 +554,127 @@ __global__ void __launch_bounds__(kThreads) rebalance_kernel(RbArgs a) {
 
   // ---- step 1: groups -> nodes ---------------------------------------------
   if (s.gpn == 1) {  // one group per node: the pages' identity short-cut
-    for (int g = tid; g < s.G; g += kThreads) {
+    for (int g = tid; g < s.G; g += nthr()) {
       gpack[g] = g;
       grank[g] = 0;
     }
   } else {
-    const uint64_t gmask = (uint64_t(1) << s.gibits) - 1;
-    for (int g = tid; g < s.gpad; g += kThreads) {
-      uint64_t key = 0;
-      if (g < s.G) {
-        uint64_t sum = 0;
-        for (int i = 0; i < s.gs; ++i) sum += static_cast<uint64_t>(w[g * s.gs + i]);
-        key = (sum << s.gibits) | (gmask - g);
-      }
-      gkey[g] = key;
+    for (int g = tid; g < s.G; g += nthr()) {
+      uint64_t sum = 0;
+#pragma unroll 8
+      for (int i = 0; i < s.gs; ++i) sum += static_cast<uint64_t>(w[g * s.gs + i]);
+      gkey[g] = (sum << kIdxBits) | (kIdxMask - g);
     }
     __syncthreads();
-    bitonic_desc<uint64_t>(gkey, s.gpad, 1);
-    if (warp == 0)
-      warp_pack<uint64_t>(gkey, s.G, s.N, s.gpn, s.gibits, s.nqbits, npw, npc, gpack, grank);
+    const uint64_t *gs_keys = gsorted;
+    if (s.gpad <= kRankSortMax) {
+      rank_segments<uint64_t>(gkey, s.gpad, 1, s.G,
+                              [&](int, int, int r, uint64_t k) { gsorted[r] = k; });
+    } else {
+      for (int g = s.G + tid; g < s.gpad; g += nthr()) gkey[g] = 0;
+      __syncthreads();
+      bitonic_desc<uint64_t>(gkey, s.gpad, 1);
+      gs_keys = gkey;
+    }
+    __syncthreads();
+    pack_segments<uint64_t>(gs_keys, s.gpad, 1, s.G, s.N, s.gpn,
+                            reinterpret_cast<uint64_t *>(smem + lay.npw),
+                            reinterpret_cast<int32_t *>(smem + lay.npc), gpack, grank, s.G);
   }
   __syncthreads();
-  // mlog = logical order after the node permutation
-  for (int e = tid; e < s.E; e += kThreads) {
+  // mlog = logical order after the node permutation; replicate's initial state
+  for (int e = tid; e < s.E; e += nthr()) {
     const int g = e / s.gs;
     const int m = (gpack[g] * s.gpn + grank[g]) * s.gs + (e - g * s.gs);
     mlog2log[m] = e;
     wm[m] = w[e];
+    cnt[m] = 1;
+    const int n = m / s.lpn;
+    const int i = m - n * s.lpn;
+    p2m[n * s.ppn + i] = i;
+    rrank[n * s.ppn + i] = 0;
   }
   __syncthreads();
 
-  // ---- step 2: replicate_experts inside every node (warp n % 4) ----------
-  const int kb = max(s.ibits, s.qbits);
-  for (int n = warp; n < s.N; n += kWarps) {
-    const int bm = n * s.lpn, bp = n * s.ppn;
-    int64_t bw = 0;
-    uint32_t bci = kNone;
-    for (int i = lane; i < s.lpn; i += 32) {
-      cnt[bm + i] = 1;
-      p2m[bp + i] = i;
-      rrank[bp + i] = 0;
-      const uint32_t ci = (1u << 16) | static_cast<uint32_t>(i);
-      if (rep_better(wm[bm + i], ci, bw, bci)) {
-        bw = wm[bm + i];
-        bci = ci;
-      }
+  // ---- step 2: replicate_experts inside every node -------------------------
+  const int nc = num_cand(s);
+  if (nc > 0 && nc <= 32) {
+    // candidates: the nc heaviest experts of each node (ties by index)
+    uint64_t *ckey = reinterpret_cast<uint64_t *>(smem + lay.keys);
+    for (int m = tid; m < s.E; m += nthr()) {
+      const int n = m / s.lpn;
+      ckey[m] = (static_cast<uint64_t>(wm[m]) << kIdxBits) | (kIdxMask - (m - n * s.lpn));
     }
-    __syncwarp();
-    int rounds = 0;
-    while ((1 << rounds) < min(s.lpn, 32)) ++rounds;
-    const int extra = s.ppn - s.lpn;
-    for (int r = 0; r < extra; ++r) {
-      int64_t mw = bw;
-      uint32_t mci = bci;
-      for (int k = rounds - 1; k >= 0; --k) {
-        const int64_t ow = static_cast<int64_t>(shfl_xor(static_cast<uint64_t>(mw), 1 << k));
-        const uint32_t oci = __shfl_xor_sync(0xffffffffu, mci, 1 << k);
-        if (rep_better(ow, oci, mw, mci)) {
-          mw = ow;
-          mci = oci;
-        }
+    __syncthreads();
+    rank_segments<uint64_t>(ckey, s.lpn, s.N, s.lpn, [&](int g, int j, int r, uint64_t) {
+      if (r < nc) {
+        cand_w[g * nc + r] = wm[g * s.lpn + j];
+        cand_i[g * nc + r] = j;
       }
-      const int b = static_cast<int>(mci & 0xffffu);
-      if (mci != kNone && lane == (b & 31)) {
-        const int old = cnt[bm + b];
-        cnt[bm + b] = old + 1;
-        p2m[bp + s.lpn + r] = b;
-        rrank[bp + s.lpn + r] = old;
-        bw = 0;
-        bci = kNone;
-        for (int i = lane; i < s.lpn; i += 32) {
-          const uint32_t ci = (static_cast<uint32_t>(cnt[bm + i]) << 16) | static_cast<uint32_t>(i);
-          if (rep_better(wm[bm + i], ci, bw, bci)) {
-            bw = wm[bm + i];
-            bci = ci;
-          }
-        }
-      }
-      __syncwarp();
+    });
+    __syncthreads();
+    if (nc * (s.ppn - s.lpn) <= 256) {
+      for (int t = tid; t < s.N * nc; t += nthr()) cand_c[t] = 1;
+      __syncthreads();
+      replicate_pairs(s, cand_w, cand_i, cand_c, p2m, rrank);
+    } else {
+      for (int n = tid >> 5; n < s.N; n += nwarps())
+        replicate_warp(s, n, cand_w, cand_i, cand_c, p2m, rrank);
     }
-    // Lambda = lcm of this node's replica counts; choose the key width
-    if (s.ppg > 1) {
-      bool ovf = false;
-      uint64_t lm = 1;
-      int64_t wmax = 0;
-      for (int i = lane; i < s.lpn; i += 32) {
-        lm = lcm_u64(lm, static_cast<uint64_t>(cnt[bm + i]), ovf);
-        wmax = max(wmax, wm[bm + i]);
-      }
-      for (int k = 16; k > 0; k >>= 1) {
-        lm = lcm_u64(lm, shfl_xor(lm, k), ovf);
-        wmax = max(wmax, static_cast<int64_t>(shfl_xor(static_cast<uint64_t>(wmax), k)));
-      }
-      ovf = __any_sync(0xffffffffu, ovf);
-      if (lane == 0) {
-        lam[n] = lm;
-        const u128 maxsum = static_cast<u128>(static_cast<uint64_t>(wmax)) * lm * s.ppg;
-        if (ovf || (maxsum >> (128 - kb - 1)) != 0)
-          atomicOr(&flags[1], 1);
-        else if ((maxsum >> (64 - kb - 1)) != 0)
-          atomicOr(&flags[0], 1);
-      }
+    __syncthreads();
+    for (int t = tid; t < s.N * nc; t += nthr()) {
+      const int n = t / nc;
+      cnt[n * s.lpn + cand_i[t]] = cand_c[t];
     }
+  } else if (nc > 32) {
+    for (int n = tid >> 5; n < s.N; n += nwarps()) replicate_smem(s, n, wm, cnt, p2m, rrank);
   }
   __syncthreads();
+
+  // ---- Lambda and key width per node (one thread per node) ----------------
+  if (s.ppg > 1) {
+    for (int n = tid; n < s.N; n += nthr()) {
+      int64_t wmax = 0;
+      if (nc > 0 && nc <= 32) {
+        wmax = cand_w[n * nc];
+      } else {
+        for (int i = 0; i < s.lpn; ++i) wmax = max(wmax, wm[n * s.lpn + i]);
+      }
+      auto width = [&](uint64_t l) -> int {
+        const u128 maxsum = static_cast<u128>(static_cast<uint64_t>(wmax)) * l * s.ppg;
+        if ((maxsum >> (63 - kIdxBits)) == 0) return 0;
+        if ((maxsum >> (127 - kIdxBits)) == 0) return 1;
+        return 2;
+      };
+      uint64_t l = s.lam_fixed;
+      int wd = 2;
+      if (l != 0) wd = width(l);
+      if (wd != 0) {
+        // lcm of the counts present in the node
+        l = 1;
+        bool ok = true;
+        if (nc > 0 && nc <= 32 && s.cmax < 64) {
+          uint64_t present = 0;  // bit c: some candidate has c replicas
+          for (int k = 0; k < nc; ++k) present |= uint64_t(1) << cand_c[n * nc + k];
+          present &= ~uint64_t(3);
+          while (present && ok) {
+            const int c = __ffsll(static_cast<long long>(present)) - 1;
+            present &= present - 1;
+            ok = lcm_into(l, static_cast<uint32_t>(c));
+          }
+        } else if (nc > 0 && nc <= 32) {
+          for (int k = 0; k < nc && ok; ++k) ok = lcm_into(l, static_cast<uint32_t>(cand_c[n * nc + k]));
+        } else {
+          for (int i = 0; i < s.lpn && ok; ++i) ok = lcm_into(l, static_cast<uint32_t>(cnt[n * s.lpn + i]));
+        }
+        wd = ok ? width(l) : 2;
+      }
+      lam[n] = l;
+      if (wd == 2) atomicOr(&flags[1], 1);
+      if (wd == 1) atomicOr(&flags[0], 1);
+    }
+    __syncthreads();
+  }
   if (flags[1]) {
     write_error_row(a, row);
     if (tid == 0) report(a.status, EPLB_ERR_RANGE);
@@ -399,45 +683,67 @@ __global__ void __launch_bounds__(kThreads) rebalance_kernel(RbArgs a) {
 
   // ---- step 3: replicas -> GPUs of each node ------------------------------
   if (s.ppg == 1) {  // one replica per GPU: identity short-cut
-    for (int t = tid; t < s.P; t += kThreads) {
+    for (int t = tid; t < s.P; t += nthr()) {
       const int n = t / s.ppn;
       ipack[t] = t - n * s.ppn;
       irank[t] = 0;
     }
   } else if (flags[0] == 0) {
-    step3_pack<uint64_t>(a, smem, lay);
+    step3<uint64_t>(a, smem, lay);
   } else {
-    step3_pack<u128>(a, smem, lay);
+    step3<u128>(a, smem, lay);
   }
   __syncthreads();
 
   // ---- assembly: pphy = node*ppn + gpu*ppg + rank -------------------------
-  for (int t = tid; t < s.P; t += kThreads) {
+  for (int t = tid; t < s.P; t += nthr()) {
     const int n = t / s.ppn;
     const int pphy = n * s.ppn + ipack[t] * s.ppg + irank[t];
     outp[pphy] = mlog2log[n * s.lpn + p2m[t]];
     outr[pphy] = rrank[t];
   }
-  for (int m = tid; m < s.E; m += kThreads) lc[mlog2log[m]] = cnt[m];
+  for (int m = tid; m < s.E; m += nthr()) lc[mlog2log[m]] = cnt[m];
   __syncthreads();
-  for (int t = tid; t < s.P; t += kThreads) {
+  for (int t = tid; t < s.P; t += nthr()) {
     a.phy2log[row * s.P + t] = outp[t];
     a.phyrank[row * s.P + t] = outr[t];
   }
-  for (int e = tid; e < s.E; e += kThreads) a.logcnt[row * s.E + e] = lc[e];
-  int32_t *gl = a.log2phy + row * static_cast<int64_t>(s.E) * s.X;
+  for (int e = tid; e < s.E; e += nthr()) a.logcnt[row * s.E + e] = lc[e];
+  const int EX = s.E * s.X;
+  int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
   bool slots = false;
-  for (int t = tid; t < s.P; t += kThreads) {
-    const int k = outr[t];
-    if (k < s.X)
-      gl[outp[t] * s.X + k] = t;
-    else
-      slots = true;
-  }
-  const uint32_t X = static_cast<uint32_t>(s.X);
-  for (int i = tid; i < s.E * s.X; i += kThreads) {
-    const uint32_t e = div_magic(static_cast<uint32_t>(i), X, a.x_magic);
-    if (static_cast<int>(i - e * X) >= lc[e]) gl[i] = -1;
+  if (table_in_smem(s)) {
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
+    for (int i = tid; i < EX; i += nthr()) tbl[i] = -1;
+    __syncthreads();
+    for (int t = tid; t < s.P; t += nthr()) {
+      const int k = outr[t];
+      if (k < s.X)
+        tbl[outp[t] * s.X + k] = t;
+      else
+        slots = true;
+    }
+    __syncthreads();
+    if (a.table_vec4) {
+      const int4 *src = reinterpret_cast<const int4 *>(tbl);
+      int4 *dst = reinterpret_cast<int4 *>(gl);
+      for (int i = tid; i < (EX >> 2); i += nthr()) dst[i] = src[i];
+    } else {
+      for (int i = tid; i < EX; i += nthr()) gl[i] = tbl[i];
+    }
+  } else {
+    for (int t = tid; t < s.P; t += nthr()) {
+      const int k = outr[t];
+      if (k < s.X)
+        gl[outp[t] * s.X + k] = t;
+      else
+        slots = true;
+    }
+    const uint32_t X = static_cast<uint32_t>(s.X);
+    for (int i = tid; i < EX; i += nthr()) {
+      const uint32_t e = div_magic(static_cast<uint32_t>(i), X, a.x_magic);
+      if (static_cast<int>(i - e * X) >= lc[e]) gl[i] = -1;
+    }
   }
   if (slots) report(a.status, EPLB_ERR_SLOTS);
 }
@@ -464,7 +770,10 @@ eplb_status launch_rebalance(const int64_t *loads, int64_t R, const RebalanceSha
   a.status = status;
   a.s = sh;
   a.x_magic = 0xffffffffu / static_cast<uint32_t>(sh.X);
-  rebalance_kernel<<<static_cast<unsigned>(R), kThreads, lay.total, stream>>>(a);
+  a.table_vec4 = ((static_cast<int64_t>(sh.E) * sh.X) % 4 == 0) &&
+                 (reinterpret_cast<uintptr_t>(log2phy) % 16 == 0);
+  const int threads = R <= 2 * static_cast<int64_t>(di.sms) ? kFewRowThreads : kManyRowThreads;
+  rebalance_kernel<<<static_cast<unsigned>(R), threads, lay.total, stream>>>(a);
   err = cudaGetLastError();
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }

@@ -5,29 +5,34 @@
 // (global token t0 + t) uses replica (t0 + t) mod logcnt[l, e] for all K
 // slots:  out[l, t, k] = log2phy[l, e, (t0 + t) mod logcnt[l, e]].
 //
-// HBM-bound gather, designed like the count kernel: a persistent grid
-// streams 16 KB chunks of the index array through a 4-stage bulk-copy ring;
-// the layer's tables (log2phy [E, X] and {logcnt, magic} [E]) sit in shared
-// memory, reloaded only when a CTA crosses a layer boundary; results leave
-// as 16-byte streaming stores.  Both divisions (position / K for the token,
-// token mod logcnt for the slot) are multiply-high with per-divisor magic
-// numbers.
+// HBM-bound gather, streamed like the count kernel: each CTA owns a
+// contiguous 16-byte aligned run of the flattened index array and walks it
+// layer segment by layer segment; the segment's tables (log2phy [E, X] and
+// {logcnt, magic} [E]) are loaded into shared memory once per segment;
+// every thread keeps U = 4 independent 16-byte streaming loads in flight and
+// writes 16-byte streaming stores.  Both divisions (position / K for the
+// token, token mod logcnt for the slot) are multiply-high with per-divisor
+// magic numbers; with K % 4 == 0 the four indices of a vector share a token.
+//
+// The same walker with kCount also builds the load histogram of S1 (the
+// count kernel's lane-banked shared histogram, flushed per layer segment),
+// so counting and redirecting one batch read its indices from HBM once:
+// 8 bytes per index instead of 4 + 8.
 #include "common.cuh"
 #include "internal.h"
 
 namespace eplb {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kChunk = 4096;  // int32 elements per stage (16 KB)
-constexpr int kStages = 4;
+constexpr int kThreads = 512;
+constexpr int kU = 4;
 
 struct RedirectArgs {
   const int32_t *idx;
+  int64_t *counts;  // kCount only
   int32_t *out;
   int64_t per_layer;  // T * K  (< 2^31)
-  int64_t cpl;
-  int64_t nchunks;
+  int64_t total;
   uint32_t K, k_magic;
   uint32_t t0;
   int32_t E, X;
@@ -37,54 +42,49 @@ struct RedirectArgs {
   int32_t *status;
 };
 
-struct Chunk {
-  int64_t layer, g0, g1, b0, b1;
-};
-
-__device__ __forceinline__ Chunk chunk_geometry(const RedirectArgs &a, int64_t c) {
-  Chunk k;
-  k.layer = c / a.cpl;
-  const int64_t within = c - k.layer * a.cpl;
-  k.g0 = k.layer * a.per_layer + within * kChunk;
-  k.g1 = min(k.g0 + (int64_t)kChunk, (k.layer + 1) * a.per_layer);
-  k.b0 = min((k.g0 + 3) & ~(int64_t)3, k.g1);
-  k.b1 = max(k.g1 & ~(int64_t)3, k.b0);
-  return k;
-}
-
+template <bool kVecToken, bool kCount>
 __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  int32_t *stage = reinterpret_cast<int32_t *>(smem);
-  uint2 *cm = reinterpret_cast<uint2 *>(smem + kStages * kChunk * sizeof(int32_t));
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t *hist = reinterpret_cast<uint32_t *>(smem);  // [E][32], kCount only
+  uint2 *cm = reinterpret_cast<uint2 *>(smem + (kCount ? a.E * 32 * sizeof(uint32_t) : 0));
   int32_t *l2p = reinterpret_cast<int32_t *>(cm + a.E);
-  __shared__ __align__(8) uint64_t full[kStages];
-
   const int tid = threadIdx.x;
-  const int64_t c_begin = a.nchunks * blockIdx.x / gridDim.x;
-  const int64_t c_end = a.nchunks * (blockIdx.x + 1) / gridDim.x;
-  const int64_t n = c_end - c_begin;
+  const int lane = tid & 31;
+  if (kCount) {
+    for (int i = tid; i < a.E * 32; i += kThreads) hist[i] = 0;
+  }
   const uint32_t E = static_cast<uint32_t>(a.E);
   const int EX = a.E * a.X;
 
-  uint64_t policy = 0;
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
-    fence_mbar_init();
-    policy = l2_policy_evict_first();
-  }
-  __syncthreads();
-
-  auto issue = [&](int64_t i) {
-    const Chunk k = chunk_geometry(a, c_begin + i);
-    const int s = static_cast<int>(i % kStages);
-    const uint32_t bytes = static_cast<uint32_t>((k.b1 - k.b0) * sizeof(int32_t));
-    mbar_arrive_expect_tx(&full[s], bytes);
-    if (bytes) bulk_g2s_stream(stage + s * kChunk, a.idx + k.b0, bytes, &full[s], policy);
+  const int64_t r0 = (a.total * blockIdx.x / gridDim.x) & ~int64_t(3);
+  const int64_t r1 = blockIdx.x + 1 == gridDim.x
+                         ? a.total
+                         : (a.total * (blockIdx.x + 1) / gridDim.x) & ~int64_t(3);
+  uint32_t nbad = 0;
+  bool range_err = false;
+  // physical index of element value e whose token is tok (global)
+  auto map = [&](int32_t e, uint32_t tok) -> int32_t {
+    if (static_cast<uint32_t>(e) >= E) {
+      ++nbad;
+      return -1;
+    }
+    if (kCount) atomicAdd(&hist[static_cast<uint32_t>(e) * 32u + lane], 1u);
+    const uint2 c = cm[e];
+    if (c.x == 0) {
+      range_err = true;
+      return -1;
+    }
+    return l2p[e * a.X + static_cast<int>(mod_magic(tok, c.x, c.y))];
   };
-  if (tid == 0)
-    for (int64_t i = 0; i < n && i < kStages; ++i) issue(i);
+  const int4 *vin = reinterpret_cast<const int4 *>(a.idx);
+  int4 *vout = reinterpret_cast<int4 *>(a.out);
 
-  auto load_tables = [&](int64_t layer) {  // all threads; callers synchronise
+  int64_t g = r0;
+  while (g < r1) {
+    const int64_t layer = g / a.per_layer;
+    const int64_t lbase = layer * a.per_layer;
+    const int64_t g1 = min(r1, lbase + a.per_layer);
+    __syncthreads();  // previous segment's table reads are done
     const int32_t *cnt = a.logcnt + layer * a.E;
     for (int e = tid; e < a.E; e += kThreads) {
       const int32_t c = __ldg(cnt + e);
@@ -94,74 +94,64 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
     }
     const int32_t *src = a.log2phy + layer * EX;
     for (int i = tid; i < EX; i += kThreads) l2p[i] = __ldg(src + i);
-  };
+    __syncthreads();
 
-  uint32_t nbad = 0;
-  bool range_err = false;
-  // Physical index of the element at within-layer position pos with value e.
-  auto map = [&](uint32_t pos, int32_t e) -> int32_t {
-    if (static_cast<uint32_t>(e) >= E) {
-      ++nbad;
-      return -1;
+    const int64_t b0 = min((g + 3) & ~int64_t(3), g1);
+    const int64_t b1 = max(g1 & ~int64_t(3), b0);
+    if (tid < b0 - g) {
+      const int64_t p = g + tid;
+      a.out[p] = map(__ldg(a.idx + p),
+                     a.t0 + div_magic(static_cast<uint32_t>(p - lbase), a.K, a.k_magic));
     }
-    const uint2 c = cm[e];
-    if (c.x == 0) {
-      range_err = true;
-      return -1;
+    if (tid >= 32 && tid - 32 < g1 - b1) {
+      const int64_t p = b1 + (tid - 32);
+      a.out[p] = map(__ldg(a.idx + p),
+                     a.t0 + div_magic(static_cast<uint32_t>(p - lbase), a.K, a.k_magic));
     }
-    const uint32_t tok = a.t0 + div_magic(pos, a.K, a.k_magic);
-    return l2p[e * a.X + static_cast<int>(mod_magic(tok, c.x, c.y))];
-  };
-
-  int64_t cur_layer = chunk_geometry(a, c_begin).layer;
-  load_tables(cur_layer);
-  __syncthreads();
-  for (int64_t i = 0; i < n; ++i) {
-    const Chunk k = chunk_geometry(a, c_begin + i);
-    if (k.layer != cur_layer) {
-      cur_layer = k.layer;
-      load_tables(cur_layer);
+    const int64_t v1 = b1 >> 2;
+    for (int64_t v = (b0 >> 2) + tid; v < v1; v += kThreads * kU) {
+      int4 x[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        x[u] = v + u * kThreads < v1 ? __ldcs(vin + v + u * kThreads) : make_int4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t vv = v + u * kThreads;
+        if (vv < v1) {
+          const uint32_t pos = static_cast<uint32_t>(vv * 4 - lbase);
+          int4 y;
+          if (kVecToken) {
+            const uint32_t tok = a.t0 + div_magic(pos, a.K, a.k_magic);
+            y.x = map(x[u].x, tok);
+            y.y = map(x[u].y, tok);
+            y.z = map(x[u].z, tok);
+            y.w = map(x[u].w, tok);
+          } else {
+            y.x = map(x[u].x, a.t0 + div_magic(pos, a.K, a.k_magic));
+            y.y = map(x[u].y, a.t0 + div_magic(pos + 1, a.K, a.k_magic));
+            y.z = map(x[u].z, a.t0 + div_magic(pos + 2, a.K, a.k_magic));
+            y.w = map(x[u].w, a.t0 + div_magic(pos + 3, a.K, a.k_magic));
+          }
+          __stcs(vout + vv, y);
+        }
+      }
+    }
+    if (kCount) {
       __syncthreads();
-    }
-    const int s = static_cast<int>(i % kStages);
-    const bool ok = mbar_wait_bounded(&full[s], static_cast<uint32_t>((i / kStages) & 1));
-    if (ok) {
-      const int64_t layer_base = k.layer * a.per_layer;
-      const int4 *v = reinterpret_cast<const int4 *>(stage + s * kChunk);
-      int4 *o = reinterpret_cast<int4 *>(a.out + k.b0);
-      const uint32_t pos0 = static_cast<uint32_t>(k.b0 - layer_base);
-      const int nv = static_cast<int>((k.b1 - k.b0) >> 2);
-#pragma unroll 4
-      for (int j = tid; j < nv; j += kThreads) {
-        const int4 x = v[j];
-        const uint32_t p = pos0 + 4u * static_cast<uint32_t>(j);
-        int4 y;
-        y.x = map(p, x.x);
-        y.y = map(p + 1, x.y);
-        y.z = map(p + 2, x.z);
-        y.w = map(p + 3, x.w);
-        __stcs(o + j, y);
-      }
-      const int head = static_cast<int>(k.b0 - k.g0);
-      const int tail = static_cast<int>(k.g1 - k.b1);
-      if (tid < head) {
-        const int64_t g = k.g0 + tid;
-        a.out[g] = map(static_cast<uint32_t>(g - layer_base), __ldg(a.idx + g));
-      }
-      if (tid >= 32 && tid - 32 < tail) {
-        const int64_t g = k.b1 + (tid - 32);
-        a.out[g] = map(static_cast<uint32_t>(g - layer_base), __ldg(a.idx + g));
+      for (int b = tid; b < a.E; b += kThreads) {
+        uint32_t sum = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+          const int w = b * 32 + ((j + b) & 31);
+          sum += hist[w];
+          hist[w] = 0;
+        }
+        if (sum)
+          atomicAdd(reinterpret_cast<unsigned long long *>(a.counts + layer * a.E + b),
+                    static_cast<unsigned long long>(sum));
       }
     }
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) {
-        for (int64_t j = i; j < n && j < i + kStages; ++j)
-          mbar_wait_bounded(&full[j % kStages], static_cast<uint32_t>((j / kStages) & 1));
-        report(a.status, EPLB_ERR_TIMEOUT);
-      }
-      return;
-    }
-    if (tid == 0 && i + kStages < n) issue(i + kStages);
+    g = g1;
   }
 
   if (range_err) report(a.status, EPLB_ERR_RANGE);
@@ -169,35 +159,24 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
   if ((tid & 31) == 0 && nbad && a.bad) atomicAdd(a.bad, static_cast<unsigned long long>(nbad));
 }
 
-size_t redirect_smem_bytes(int E, int X) {
-  return static_cast<size_t>(kStages) * kChunk * sizeof(int32_t) + static_cast<size_t>(E) * 8 +
-         static_cast<size_t>(E) * X * sizeof(int32_t);
-}
-
 }  // namespace
 
 eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
                             const int32_t *log2phy, int32_t X, const int32_t *logcnt, int64_t t0,
-                            int32_t *out, unsigned long long *bad, int32_t *status,
-                            cudaStream_t stream) {
+                            int32_t *out, int64_t *counts, unsigned long long *bad,
+                            int32_t *status, cudaStream_t stream) {
   DeviceInfo di;
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
-  const size_t smem = redirect_smem_bytes(E, X);
+  const bool count = counts != nullptr;
+  const size_t smem = (count ? static_cast<size_t>(E) * 32 * sizeof(uint32_t) : 0) +
+                      static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * X * sizeof(int32_t);
   if (smem > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
-  cudaError_t err = cudaFuncSetAttribute(redirect_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return cuda_fail(err);
-  int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, redirect_kernel, kThreads, smem);
-  if (err != cudaSuccess) return cuda_fail(err);
-  if (per_sm < 1) per_sm = 1;
   RedirectArgs a;
   a.idx = idx;
+  a.counts = counts;
   a.out = out;
   a.per_layer = T * K;
-  a.cpl = (a.per_layer + kChunk - 1) / kChunk;
-  a.nchunks = a.cpl * L;
+  a.total = a.per_layer * L;
   a.K = static_cast<uint32_t>(K);
   a.k_magic = 0xffffffffu / static_cast<uint32_t>(K);
   a.t0 = static_cast<uint32_t>(t0);
@@ -207,9 +186,25 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
   a.logcnt = logcnt;
   a.bad = bad;
   a.status = status;
-  const int64_t grid = std::min<int64_t>(a.nchunks, static_cast<int64_t>(di.sms) * per_sm);
-  redirect_kernel<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(a);
-  err = cudaGetLastError();
+  const bool vec_token = (K % 4) == 0;
+  const void *fn;
+  if (count)
+    fn = vec_token ? reinterpret_cast<const void *>(redirect_kernel<true, true>)
+                   : reinterpret_cast<const void *>(redirect_kernel<false, true>);
+  else
+    fn = vec_token ? reinterpret_cast<const void *>(redirect_kernel<true, false>)
+                   : reinterpret_cast<const void *>(redirect_kernel<false, false>);
+  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return cuda_fail(err);
+  int per_sm = 0;
+  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
+  if (err != cudaSuccess) return cuda_fail(err);
+  per_sm = std::max(1, std::min(per_sm, 2));
+  const int64_t grid = std::max<int64_t>(
+      1, std::min<int64_t>(static_cast<int64_t>(di.sms) * per_sm, (a.total + 4095) / 4096));
+  void *args[] = {&a};
+  err = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), args, smem, stream);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

@@ -72,12 +72,16 @@ eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W,
                           int64_t *snaps, cudaStream_t stream) {
   DeviceInfo di;
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
-  // Pick the strip width: fill the SMs evenly (strips per SM rounded up
-  // costs the tail), with enough threads per SM to keep loads in flight.
+  // Pick the strip width cw and row groups rg: rg never exceeds the row
+  // blocks there are (short rings), the strip count fills the SMs evenly
+  // (strips per SM rounded up cost the tail), and enough threads per SM keep
+  // loads in flight.
+  const int64_t max_rg = std::max<int64_t>(1, (S + kU - 1) / kU);
   int best_cw = 32;
   double best_score = -1.0;
-  for (int cw = 8; cw <= 128; ++cw) {
-    const int rg = std::max(1, 256 / cw);
+  for (int cw = 8; cw <= 256; ++cw) {
+    const int rg = static_cast<int>(std::min<int64_t>(std::max(1, 256 / cw), max_rg));
+    if (cw * rg > 1024) continue;
     const int64_t strips = (C + cw - 1) / cw;
     const int64_t waves = (strips + di.sms - 1) / di.sms;
     const double balance = static_cast<double>(strips) / static_cast<double>(waves * di.sms);
@@ -91,7 +95,7 @@ eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W,
     }
   }
   const int cw = static_cast<int>(std::min<int64_t>(best_cw, C));
-  const int rg = std::max(1, 256 / cw);
+  const int rg = static_cast<int>(std::min<int64_t>(std::max(1, 256 / cw), max_rg));
   const int64_t strips = (C + cw - 1) / cw;
   const size_t smem = static_cast<size_t>(rg) * cw * sizeof(int64_t);
   window_kernel<<<static_cast<unsigned>(strips), cw * rg, smem, stream>>>(steps, S, C, W, s_first,

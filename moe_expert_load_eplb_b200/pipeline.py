@@ -1,13 +1,17 @@
-"""One serving step of the EPLB hot path on one GPU, with preallocated buffers.
+"""One step of the EPLB hot path on one GPU, with preallocated buffers.
 
-Per step (all stream-ordered, no host round-trip):
-  1. count_loads: this step's routed indices -> its row of the load window
-     ring (int64 [W, L, E], row step % W);
-  2. window_accumulate over the ring (s_first = W - 1): the window sum, which
-     is the moving-average load estimate times W (page "DualPipe и EPLB",
-     Part 2, section "Алгоритм");
-  3. rebalance: the replica/placement plan of every layer;
-  4. redirect: this step's indices to physical replicas.
+Two orders of the same four stages, both stream-ordered with no host
+round-trip:
+
+serving (default): the plan in force (built from earlier steps' loads, the
+  moving-average estimate of page "DualPipe и EPLB", Part 2, section
+  "Алгоритм") redirects this step's indices in the same pass that counts
+  them, so the indices cross HBM once:
+    1. count_redirect: indices -> ring row (step % W) and physical indices;
+    2. window_accumulate over the ring (s_first = W - 1): the window sum;
+    3. rebalance: the next plan of every layer.
+fresh: the plan is rebuilt from this step's counts before redirecting:
+    count_loads -> window_accumulate -> rebalance -> redirect.
 
 With ``group`` set (torch.distributed, NCCL), every rank counts its own
 token shard and the ring row is summed over ranks with one all-reduce before
@@ -17,17 +21,27 @@ tokens with its global token offset.
 """
 from __future__ import annotations
 
-from typing import Optional
+from typing import Optional, Sequence
 
 import torch
 
-from . import Plan, count_loads, default_slots, rebalance, redirect, window_accumulate
+from . import (Plan, count_loads, count_redirect, default_slots, rebalance, redirect,
+               window_accumulate)
+
+
+def _plan(L, E, P, X, dev) -> Plan:
+    return Plan(torch.empty((L, P), dtype=torch.int32, device=dev),
+                torch.empty((L, P), dtype=torch.int32, device=dev),
+                torch.empty((L, E), dtype=torch.int32, device=dev),
+                torch.empty((L, E, X), dtype=torch.int32, device=dev))
 
 
 class EplbStep:
+    STAGES = ("count", "allreduce", "window", "rebalance", "redirect")
+
     def __init__(self, L: int, T: int, K: int, E: int, P: int, G: int, N: int, gpus: int,
                  window: int = 1, device="cuda", slots: Optional[int] = None,
-                 token_offset: int = 0, group=None):
+                 token_offset: int = 0, group=None, fused: bool = True):
         self.L, self.T, self.K, self.E = L, T, K, E
         self.P, self.G, self.N, self.gpus = P, G, N, gpus
         self.W = window
@@ -35,35 +49,77 @@ class EplbStep:
         self.X = default_slots(E, P, G, N) if slots is None else slots
         self.token_offset = token_offset
         self.group = group
+        self.fused = fused
         dev = self.device
         self.ring = torch.zeros((window, L, E), dtype=torch.int64, device=dev)
         self.loads = torch.zeros((1, L, E), dtype=torch.int64, device=dev)
-        self.plan = Plan(torch.empty((L, P), dtype=torch.int32, device=dev),
-                         torch.empty((L, P), dtype=torch.int32, device=dev),
-                         torch.empty((L, E), dtype=torch.int32, device=dev),
-                         torch.empty((L, E, self.X), dtype=torch.int32, device=dev))
+        self.plans = [_plan(L, E, P, self.X, dev), _plan(L, E, P, self.X, dev)]
+        self.cur = 0  # index of the plan in force
         self.out = torch.empty((L, T, K), dtype=torch.int32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.bad = torch.zeros(1, dtype=torch.int64, device=dev)
         self.steps_done = 0
+        self.primed = False
 
-    def fill_history(self, history: torch.Tensor):
-        """Set the ring to earlier per-step counts (int64 [W, L, E])."""
-        self.ring.copy_(history)
+    @property
+    def launches_per_step(self) -> int:
+        """Kernels of this library launched per step."""
+        return 3 if self.fused else 4
 
-    def __call__(self, idx: torch.Tensor):
-        """Run one step on idx (int32 [L, T, K]); returns (plan, redirected indices)."""
-        slot = self.steps_done % self.W
-        row = self.ring[slot]
-        count_loads(idx, self.E, counts=row, bad=self.bad, status=self.status)
+    @property
+    def plan(self) -> Plan:
+        """The plan in force (the newest one built)."""
+        return self.plans[self.cur]
+
+    def fill_history(self, history: torch.Tensor, steps_done: Optional[int] = None):
+        """Load earlier per-step counts into the ring and build the plan in force."""
+        n = history.shape[0]
+        self.ring[:n].copy_(history)
+        self.steps_done = n if steps_done is None else steps_done
+        self._plan_from_ring(self.plans[self.cur])
+        self.primed = True
+
+    def _plan_from_ring(self, plan: Plan):
+        window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads, status=self.status)
+        rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=plan,
+                  status=self.status)
+
+    def __call__(self, idx: torch.Tensor, marks: Optional[Sequence] = None):
+        """Run one step on idx (int32 [L, T, K]).
+
+        Returns (plan used for this step's redirect, redirected indices); the
+        serving order's new plan is ``self.plan`` afterwards.  ``marks``: six
+        CUDA events recorded on the current stream around the stages
+        count | allreduce | window | rebalance | redirect (the serving order
+        records its fused pass under count and an empty redirect stage).
+        """
+        if self.fused and not self.primed:
+            raise RuntimeError("serving order needs a plan in force: call fill_history() first")
+        rec = (lambda k: marks[k].record()) if marks else (lambda k: None)
+        row = self.ring[self.steps_done % self.W]
+        used = self.plans[self.cur]
+        rec(0)
+        if self.fused:
+            count_redirect(idx, self.E, used.log2phy, used.logcnt, self.token_offset, counts=row,
+                           out=self.out, bad=self.bad, status=self.status)
+        else:
+            count_loads(idx, self.E, counts=row, bad=self.bad, status=self.status)
+        rec(1)
         if self.group is not None:
             torch.distributed.all_reduce(row, group=self.group)
+        rec(2)
         window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads, status=self.status)
-        rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=self.plan,
+        rec(3)
+        nxt = self.plans[1 - self.cur] if self.fused else used
+        rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=nxt,
                   status=self.status)
-        redirect(idx, self.plan.log2phy, self.plan.logcnt, self.token_offset, out=self.out,
-                 bad=self.bad, status=self.status)
+        rec(4)
+        if not self.fused:
+            redirect(idx, nxt.log2phy, nxt.logcnt, self.token_offset, out=self.out, bad=self.bad,
+                     status=self.status)
+        rec(5)
         self.steps_done += 1
-        return self.plan, self.out
-
-    launches_per_step = 4  # count, window, rebalance, redirect kernels
+        if self.fused:
+            self.cur = 1 - self.cur
+            return used, self.out
+        return nxt, self.out

@@ -365,22 +365,97 @@ def test_redirect_sharded_equals_whole(c2_idx):
     assert torch.equal(torch.cat([a, b], dim=1), whole)
 
 
+# ---------------------------------------------------- fused count + redirect --
+
+def _plan_in_force(c, seed):
+    loads = W.histogram_steps(1, c.L, c.E, max(c.T, 1) * max(c.K, 1), seed, device=DEV)[0]
+    return eplb.rebalance(loads, c.P, c.G, c.N, c.gpus)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 5])
+def test_count_redirect_configs(cfg, request):
+    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
+    c = W.CONFIGS[cfg]
+    plan = _plan_in_force(c, 100 + cfg)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    st = _status()
+    counts, out = eplb.count_redirect(idx, c.E, plan.log2phy, plan.logcnt, bad=bad, status=st)
+    idx_h = _np(idx)
+    ref_c, nb = oracle.count_loads(idx_h, c.E)
+    ref_o, nb2 = oracle.redirect(idx_h, _np(plan.log2phy), _np(plan.logcnt))
+    assert np.array_equal(_np(counts), ref_c)
+    assert np.array_equal(_np(out), ref_o)
+    assert int(bad.item()) == nb == nb2 == 0 and int(st.item()) == 0
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1), (3, 1001, 3), (2, 4097, 8), (5, 3, 7), (2, 70001, 5),
+                                   (4, 2048, 6), (7, 12345, 2)])
+@pytest.mark.parametrize("t0", [0, 19, (1 << 31) - 80000])
+def test_count_redirect_ragged(shape, t0):
+    L, T, K = shape
+    E, P, G, N, gpus = 24, 40, 6, 2, 4
+    rng = np.random.default_rng(L * 7 + T + K)
+    ref_plan = oracle.rebalance(rng.integers(0, 1000, (L, E)), P, G, N, gpus)
+    l2p = torch.from_numpy(ref_plan[3]).to(DEV)
+    cnt = torch.from_numpy(ref_plan[2]).to(DEV)
+    g = torch.Generator(device=DEV).manual_seed(T + 1)
+    idx = torch.randint(-2, E + 2, (L, T, K), generator=g, device=DEV, dtype=torch.int32)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    counts, out = eplb.count_redirect(idx, E, l2p, cnt, token_offset=t0, bad=bad)
+    idx_h = _np(idx)
+    ref_c, nb = oracle.count_loads(idx_h, E)
+    ref_o, _ = oracle.redirect(idx_h, ref_plan[3], ref_plan[2], t0)
+    assert np.array_equal(_np(counts), ref_c)
+    assert np.array_equal(_np(out), ref_o)
+    assert int(bad.item()) == nb
+    counts2, _ = eplb.count_redirect(idx, E, l2p, cnt, token_offset=t0, counts=counts, accumulate=True)
+    assert np.array_equal(_np(counts2), 2 * ref_c)
+
+
 # --------------------------------------------------------------- pipeline --
 
-def test_pipeline_step_c2(c2_idx):
+def _oracle_plan_from_ring(ring, c, X):
+    loads = oracle.window(ring, ring.shape[0], ring.shape[0] - 1)[0]
+    return oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=X)
+
+
+def test_pipeline_fresh_order_c2(c2_idx):
     from moe_expert_load_eplb_b200.pipeline import EplbStep
     c = W.CONFIGS[2]
     hist = W.histogram_steps(15, c.L, c.E, c.T * c.K, 2, device=DEV)
-    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=16, device=DEV)
-    step.ring[:15].copy_(hist)
-    step.steps_done = 15
+    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=16, device=DEV, fused=False)
+    step.fill_history(hist)
     plan, out = step(c2_idx)
     torch.cuda.synchronize()
     assert int(step.status.item()) == 0
     counts, _ = oracle.count_loads(_np(c2_idx), c.E)
-    ring = np.concatenate([_np(hist), counts[None]], axis=0)
-    loads = oracle.window(ring, 16, 15)[0]
-    ref = oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=step.X)
+    ref = _oracle_plan_from_ring(np.concatenate([_np(hist), counts[None]], axis=0), c, step.X)
     _assert_plan_equal(plan, ref)
     red, _ = oracle.redirect(_np(c2_idx), ref[3], ref[2])
     assert np.array_equal(_np(out), red)
+
+
+def test_pipeline_serving_order_c2(c2_idx):
+    """Three serving steps: each redirects with the plan in force, then rebuilds it."""
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+    c = W.CONFIGS[2]
+    W_ = 4
+    hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, 2, device=DEV)
+    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV, fused=True,
+                    token_offset=1000)
+    step.fill_history(hist)
+    ring = np.concatenate([_np(hist), np.zeros((1, c.L, c.E), np.int64)], axis=0)
+    plan_ref = _oracle_plan_from_ring(ring, c, step.X)
+    _assert_plan_equal(step.plan, plan_ref)
+    batches = [c2_idx, W.routed_indices(2, device=DEV, shard=1), c2_idx.flip(1).contiguous()]
+    for s_i, idx in enumerate(batches):
+        used, out = step(idx)
+        torch.cuda.synchronize()
+        assert int(step.status.item()) == 0
+        idx_h = _np(idx)
+        red, _ = oracle.redirect(idx_h, plan_ref[3], plan_ref[2], 1000)
+        assert np.array_equal(_np(out), red), f"step {s_i}: redirect"
+        counts, _ = oracle.count_loads(idx_h, c.E)
+        ring[(W_ - 1 + s_i) % W_] = counts
+        plan_ref = _oracle_plan_from_ring(ring, c, step.X)
+        _assert_plan_equal(step.plan, plan_ref)
