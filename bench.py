@@ -51,6 +51,10 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e measurement")
+    ap.add_argument("--no-fresh", action="store_true", help="skip the fresh-plan-order comparison")
+    ap.add_argument("--fresh-only", action="store_true",
+                    help="time only the fresh-plan order (for profiling its kernels)")
     return ap.parse_args()
 
 
@@ -240,6 +244,17 @@ def run_ours(args, rank: int, world: int, group):
         if code != 0:
             raise RuntimeError(f"device status {eplb.STATUS.get(code)} in {where}")
 
+    if args.fresh_only:
+        fresh = make(False)
+        for i in range(args.warmup):
+            flush.fill_(i & 0xff)
+            fresh(idx)
+        check(fresh, "fresh-order warm-up")
+        f_total, f_stage, clocks = _timed_steps(fresh, idx, flush, args.steps, group, dev)
+        check(fresh, "fresh-order steps")
+        return {"fresh_only": True, "steps": args.steps, "ms_per_step": round(f_total / args.steps, 5),
+                "stages": _stage_report(f_stage, False, fresh.X, world, hbm_peak), "clocks": clocks}
+
     # ---- the timed step: serving order (count+redirect fused, then plan) ----
     step = make(True)
     for i in range(args.warmup):
@@ -279,6 +294,8 @@ def run_ours(args, rank: int, world: int, group):
            "stages": stages, "roofline": roof, "clocks": clocks}
 
     # ---- the same four stages in the fresh-plan order, for comparison -----
+    if args.no_fresh:
+        return _finish(out, args, step, idx, hist, flush, group, dev, rank, world)
     fresh = make(False)
     for i in range(max(3, args.warmup // 4)):
         flush.fill_(i & 0xff)
@@ -293,36 +310,49 @@ def run_ours(args, rank: int, world: int, group):
     out["load_count_gbs"] = fstages["count"]["gbs"]
     out["load_count_frac_hbm"] = fstages["count"]["frac_hbm"]
     del fresh
+    return _finish(out, args, step, idx, hist, flush, group, dev, rank, world)
+
+
+def _finish(out, args, step, idx, hist, flush, group, dev, rank, world):
+    c = CFG
+    K = args.steps
+
+    def check(st, where):
+        torch.cuda.synchronize()
+        code = int(st.status.item())
+        if code != 0:
+            raise RuntimeError(f"device status {code} in {where}")
 
     # ---- e2e: the serving step through the public API with host buffers --
-    Ke = max(5, min(K, 50))
-    idx_host = idx.cpu().pin_memory()
-    out_host = torch.empty(step.out.shape, dtype=torch.int32).pin_memory()
-    plan_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.plan]
-    idx_dev = torch.empty_like(idx)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(Ke)]
-    if group is not None:
-        torch.distributed.barrier(group=group)
-    torch.cuda.synchronize()
-    for i in range(Ke):
-        flush.fill_(i & 0xff)
-        ev[i][0].record()
-        idx_dev.copy_(idx_host, non_blocking=True)
-        step(idx_dev)
-        out_host.copy_(step.out, non_blocking=True)
-        for h, d in zip(plan_host, step.plan):
-            h.copy_(d, non_blocking=True)
-        ev[i][1].record()
-    check(step, "e2e steps")
-    e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
-    if group is not None:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX, group=group)
-    e2e_ms = float(e2e_ms.item())
-    out["e2e"] = {"value": round(c.L * Ke / (e2e_ms / 1e3), 1), "unit": UNIT,
-                  "h2d_bytes_per_step": idx.numel() * 4,
-                  "d2h_bytes_per_step": out_host.numel() * 4 + sum(t.numel() * 4 for t in plan_host),
-                  "steps": Ke, "ms_per_step": round(e2e_ms / Ke, 4)}
+    if not args.no_e2e:
+        Ke = max(5, min(K, 50))
+        idx_host = idx.cpu().pin_memory()
+        out_host = torch.empty(step.out.shape, dtype=torch.int32).pin_memory()
+        plan_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.plan]
+        idx_dev = torch.empty_like(idx)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(Ke)]
+        if group is not None:
+            torch.distributed.barrier(group=group)
+        torch.cuda.synchronize()
+        for i in range(Ke):
+            flush.fill_(i & 0xff)
+            ev[i][0].record()
+            idx_dev.copy_(idx_host, non_blocking=True)
+            step(idx_dev)
+            out_host.copy_(step.out, non_blocking=True)
+            for h, d in zip(plan_host, step.plan):
+                h.copy_(d, non_blocking=True)
+            ev[i][1].record()
+        check(step, "e2e steps")
+        e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
+        if group is not None:
+            torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX, group=group)
+        e2e_ms = float(e2e_ms.item())
+        out["e2e"] = {"value": round(c.L * Ke / (e2e_ms / 1e3), 1), "unit": UNIT,
+                      "h2d_bytes_per_step": idx.numel() * 4,
+                      "d2h_bytes_per_step": out_host.numel() * 4 + sum(t.numel() * 4 for t in plan_host),
+                      "steps": Ke, "ms_per_step": round(e2e_ms / Ke, 4)}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(idx.cpu().numpy(), hist.cpu().numpy(), args.cpu_seconds)
@@ -409,13 +439,9 @@ def main():
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
+    from moe_expert_load_eplb_b200.distributed import init_from_env
+    rank, world, local, group = init_from_env("nccl" if world > 1 else None)
     torch.cuda.set_device(local)
-    group = None
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-        group = torch.distributed.group.WORLD
     try:
         res = run_ours(args, rank, world, group)
         if rank == 0:

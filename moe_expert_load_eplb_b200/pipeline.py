@@ -27,6 +27,7 @@ import torch
 
 from . import (Plan, count_loads, count_redirect, default_slots, rebalance, redirect,
                window_accumulate)
+from .distributed import allreduce_loads
 
 
 def _plan(L, E, P, X, dev) -> Plan:
@@ -106,7 +107,7 @@ class EplbStep:
             count_loads(idx, self.E, counts=row, bad=self.bad, status=self.status)
         rec(1)
         if self.group is not None:
-            torch.distributed.all_reduce(row, group=self.group)
+            allreduce_loads(row, self.group)
         rec(2)
         window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads, status=self.status)
         rec(3)
