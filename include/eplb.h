@@ -170,6 +170,59 @@ eplb_status eplb_count_redirect(const int32_t *idx, int64_t L, int64_t T, int32_
                                 int32_t X, const int32_t *logcnt, int64_t t0, int32_t *out,
                                 unsigned long long *bad, int32_t *status, cudaStream_t stream);
 
+/*
+ * Plan quality ([EPLB] box "От переводчика: что на рисунке": per-GPU load of
+ * the worked example, 86.5 .. 156, mean 129; exercise 2 of "что сделать
+ * руками": compare max / mean between policies).  Per row r:
+ *   gpu_load[r, g] = sum over GPU g's slots p (p / (P/gpus) == g, in slot
+ *                    order) of loads[r, phy2log[r,p]] / logcnt[r, phy2log[r,p]]
+ *   stats[r] = { min_g, max_g, mean_g (summed in GPU order), mean / max }
+ *              (balancedness 1 when max is 0).
+ * fp64 with round-to-nearest adds and divides in exactly that order.
+ * loads int64 [R, E]; phy2log int32 [R, P]; logcnt int32 [R, E]; gpu_load
+ * double [R, gpus] and stats double [R, 4], either may be NULL (not both).
+ * A slot naming no expert in [0, E) or an expert with logcnt < 1 is skipped
+ * and *status = EPLB_ERR_RANGE.  Limits: gpus | P, gpus <= 16384.
+ */
+eplb_status eplb_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,
+                            int64_t R, int32_t E, int32_t P, int32_t gpus, double *gpu_load,
+                            double *stats, int32_t *status, cudaStream_t stream);
+
+/*
+ * Fold loads recorded per physical expert into loads per logical expert:
+ *   logical[r, e] = sum of phys[r, p] over slots p with phy2log[r, p] == e.
+ * A serving engine counts routed tokens after redirection (physical space,
+ * e.g. eplb_count_loads with E = P on redirected indices) and folds them
+ * before the next rebalance.  phys int64 [R, P]; phy2log int32 [R, P];
+ * logical int64 [R, E] (overwritten).  Slots naming no expert in [0, E) are
+ * skipped and *status = EPLB_ERR_RANGE.  Limits: E <= 4096.
+ */
+eplb_status eplb_fold_loads(const int64_t *phys, const int32_t *phy2log, int64_t R, int32_t E,
+                            int32_t P, int64_t *logical, int32_t *status, cudaStream_t stream);
+
+/*
+ * The plan before any load is known: routed experts first, then the
+ * redundant slots cycle through the experts from 0:
+ *   phy2log[r, p] = p mod E,  phyrank[r, p] = p div E  (phyrank nullable).
+ */
+eplb_status eplb_initial_map(int64_t R, int32_t E, int32_t P, int32_t *phy2log, int32_t *phyrank,
+                             cudaStream_t stream);
+
+/*
+ * Plan diff: which slots of a new plan must fetch their expert's weights.
+ * GPU g (slots g*P/gpus ..) keeps min(old_g(e), new_g(e)) replicas of each
+ * expert e in place; going through g's new slots in order, slot p keeps its
+ * expert when fewer earlier new slots of g hold it than old slots of g did:
+ *   src[r, p] = -1 (kept) or the lowest old slot holding phy2log_new[r, p]
+ *               (-2 if no old slot holds it);
+ *   moves[r]  = number of slots with src != -1 (nullable).
+ * old / new phy2log int32 [R, P]; src int32 [R, P].  Entries outside [0, E)
+ * give src = -2 and *status = EPLB_ERR_RANGE.  Limits: gpus | P, E <= 8192.
+ */
+eplb_status eplb_plan_diff(const int32_t *old_phy2log, const int32_t *new_phy2log, int64_t R,
+                           int32_t E, int32_t P, int32_t gpus, int32_t *src, int32_t *moves,
+                           int32_t *status, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,6 +25,7 @@ import torch
 
 __all__ = [
     "EplbError", "Plan", "count_loads", "window_accumulate", "rebalance", "redirect", "count_redirect",
+    "plan_stats", "fold_loads", "initial_map", "plan_diff",
     "default_slots", "lib_path", "load_library", "STATUS",
 ]
 
@@ -80,6 +81,10 @@ def load_library():
         "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p], i32),
         "eplb_redirect": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, p], i32),
         "eplb_count_redirect": ([p, i64, i64, i32, i32, p, i32, p, i32, p, i64, p, p, p, p], i32),
+        "eplb_plan_stats": ([p, p, p, i64, i32, i32, i32, p, p, p, p], i32),
+        "eplb_fold_loads": ([p, p, i64, i32, i32, p, p, p], i32),
+        "eplb_initial_map": ([i64, i32, i32, p, p, p], i32),
+        "eplb_plan_diff": ([p, p, i64, i32, i32, i32, p, p, p, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -248,3 +253,64 @@ def count_redirect(idx: torch.Tensor, num_experts: int, log2phy: torch.Tensor, l
             _ptr(logcnt), int(token_offset), _ptr(out), _ptr(bad), _ptr(status),
             _stream(idx.device)), "eplb_count_redirect")
     return counts, out
+
+
+def plan_stats(loads: torch.Tensor, phy2log: torch.Tensor, logcnt: torch.Tensor, num_gpus: int,
+               status: Optional[torch.Tensor] = None):
+    """Per-GPU load (fp64, sum of w/logcnt over the GPU's slots in order) and
+    per-row stats {min, max, mean, mean/max}.  Returns (gpu_load [R, gpus], stats [R, 4])."""
+    _cuda(loads, torch.int64, "loads")
+    _cuda(phy2log, torch.int32, "phy2log")
+    _cuda(logcnt, torch.int32, "logcnt")
+    R, E = loads.shape
+    P = phy2log.shape[1]
+    gl = torch.empty((R, num_gpus), dtype=torch.float64, device=loads.device)
+    st = torch.empty((R, 4), dtype=torch.float64, device=loads.device)
+    with torch.cuda.device(loads.device):
+        _check(load_library().eplb_plan_stats(
+            _ptr(loads), _ptr(phy2log), _ptr(logcnt), R, E, P, num_gpus, _ptr(gl), _ptr(st),
+            _ptr(status), _stream(loads.device)), "eplb_plan_stats")
+    return gl, st
+
+
+def fold_loads(phys: torch.Tensor, phy2log: torch.Tensor, num_logical: int,
+               status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """logical[r, e] = sum of phys[r, p] over slots with phy2log[r, p] == e."""
+    _cuda(phys, torch.int64, "phys")
+    _cuda(phy2log, torch.int32, "phy2log")
+    R, P = phys.shape
+    out = torch.empty((R, num_logical), dtype=torch.int64, device=phys.device)
+    with torch.cuda.device(phys.device):
+        _check(load_library().eplb_fold_loads(
+            _ptr(phys), _ptr(phy2log), R, num_logical, P, _ptr(out), _ptr(status),
+            _stream(phys.device)), "eplb_fold_loads")
+    return out
+
+
+def initial_map(rows: int, num_logical: int, num_replicas: int, device="cuda"):
+    """phy2log[r, p] = p mod E, phyrank[r, p] = p div E (routed first, then redundant)."""
+    p2l = torch.empty((rows, num_replicas), dtype=torch.int32, device=device)
+    prk = torch.empty((rows, num_replicas), dtype=torch.int32, device=device)
+    dev = p2l.device
+    with torch.cuda.device(dev):
+        _check(load_library().eplb_initial_map(rows, num_logical, num_replicas, _ptr(p2l), _ptr(prk),
+                                               _stream(dev)), "eplb_initial_map")
+    return p2l, prk
+
+
+def plan_diff(old_phy2log: torch.Tensor, new_phy2log: torch.Tensor, num_logical: int, num_gpus: int,
+              status: Optional[torch.Tensor] = None):
+    """src[r, p] = -1 where the new slot keeps its expert on its GPU, else the old slot
+    to copy from; moves[r] = number of copies.  Returns (src, moves)."""
+    _cuda(old_phy2log, torch.int32, "old_phy2log")
+    _cuda(new_phy2log, torch.int32, "new_phy2log")
+    if old_phy2log.shape != new_phy2log.shape:
+        raise ValueError("plans must have the same shape")
+    R, P = new_phy2log.shape
+    src = torch.empty((R, P), dtype=torch.int32, device=new_phy2log.device)
+    moves = torch.empty((R,), dtype=torch.int32, device=new_phy2log.device)
+    with torch.cuda.device(new_phy2log.device):
+        _check(load_library().eplb_plan_diff(
+            _ptr(old_phy2log), _ptr(new_phy2log), R, num_logical, P, num_gpus, _ptr(src),
+            _ptr(moves), _ptr(status), _stream(new_phy2log.device)), "eplb_plan_diff")
+    return src, moves

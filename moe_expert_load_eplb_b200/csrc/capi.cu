@@ -202,4 +202,43 @@ eplb_status eplb_count_redirect(const int32_t *idx, int64_t L, int64_t T, int32_
                          stream);
 }
 
+eplb_status eplb_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,
+                            int64_t R, int32_t E, int32_t P, int32_t gpus, double *gpu_load,
+                            double *stats, int32_t *status, cudaStream_t stream) {
+  if (R < 0 || E < 1 || P < 1 || gpus < 1) return EPLB_ERR_SHAPE;
+  if (P % gpus != 0) return EPLB_ERR_DIVISIBILITY;
+  if (gpus > 16384 || R > 0x7fffffffLL) return EPLB_ERR_LIMIT;
+  if (R == 0) return EPLB_OK;
+  if (!loads || !phy2log || !logcnt || (!gpu_load && !stats)) return EPLB_ERR_NULL;
+  return launch_plan_stats(loads, phy2log, logcnt, R, E, P, gpus, gpu_load, stats, status, stream);
+}
+
+eplb_status eplb_fold_loads(const int64_t *phys, const int32_t *phy2log, int64_t R, int32_t E,
+                            int32_t P, int64_t *logical, int32_t *status, cudaStream_t stream) {
+  if (R < 0 || E < 1 || P < 1) return EPLB_ERR_SHAPE;
+  if (E > 4096 || R > 0x7fffffffLL) return EPLB_ERR_LIMIT;
+  if (R == 0) return EPLB_OK;
+  if (!phys || !phy2log || !logical) return EPLB_ERR_NULL;
+  return launch_fold_loads(phys, phy2log, R, E, P, logical, status, stream);
+}
+
+eplb_status eplb_initial_map(int64_t R, int32_t E, int32_t P, int32_t *phy2log, int32_t *phyrank,
+                             cudaStream_t stream) {
+  if (R < 0 || E < 1 || P < E) return EPLB_ERR_SHAPE;
+  if (R == 0) return EPLB_OK;
+  if (!phy2log) return EPLB_ERR_NULL;
+  return launch_initial_map(R, E, P, phy2log, phyrank, stream);
+}
+
+eplb_status eplb_plan_diff(const int32_t *old_phy2log, const int32_t *new_phy2log, int64_t R,
+                           int32_t E, int32_t P, int32_t gpus, int32_t *src, int32_t *moves,
+                           int32_t *status, cudaStream_t stream) {
+  if (R < 0 || E < 1 || P < 1 || gpus < 1) return EPLB_ERR_SHAPE;
+  if (P % gpus != 0) return EPLB_ERR_DIVISIBILITY;
+  if (E > 8192 || R > 0x7fffffffLL) return EPLB_ERR_LIMIT;
+  if (R == 0) return EPLB_OK;
+  if (!old_phy2log || !new_phy2log || !src) return EPLB_ERR_NULL;
+  return launch_plan_diff(old_phy2log, new_phy2log, R, E, P, gpus, src, moves, status, stream);
+}
+
 }  // extern "C"

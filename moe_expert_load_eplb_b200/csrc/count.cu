@@ -15,7 +15,9 @@
 //     not);
 //   * increments go to a lane-banked shared histogram: bin e of lane j is
 //     word e*32 + j, so lane j always hits bank j and one warp-wide atomic
-//     is conflict-free whatever the skew of the routing distribution;
+//     is conflict-free whatever the skew of the routing distribution; an
+//     index outside [0, E) lands in a sentinel bin E, whose total is the
+//     bad-index count (no branch per index);
 //   * at each layer boundary and at the end the 32 lane copies of a bin are
 //     summed (rotated reads, conflict-free) and added to the int64 output
 //     with one global atomic per bin and CTA.
@@ -39,11 +41,12 @@ struct CountArgs {
 };
 
 __global__ void __launch_bounds__(kThreads, 1) count_loads_kernel(CountArgs a) {
-  extern __shared__ __align__(16) uint32_t hist[];  // [E][32]
+  extern __shared__ __align__(16) uint32_t hist[];  // [E+1][32]; bin E counts bad indices
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
+  const uint32_t lane = tid & 31;
   const uint32_t E = static_cast<uint32_t>(a.E);
-  for (int i = tid; i < a.E * 32; i += kThreads) hist[i] = 0;
+  const int E1 = a.E + 1;
+  for (int i = tid; i < E1 * 32; i += kThreads) hist[i] = 0;
   __syncthreads();
 
   // this CTA's elements [r0, r1): boundaries rounded down to 4 elements
@@ -53,10 +56,8 @@ __global__ void __launch_bounds__(kThreads, 1) count_loads_kernel(CountArgs a) {
                          : (a.total * (blockIdx.x + 1) / gridDim.x) & ~int64_t(3);
   uint32_t nbad = 0;
   auto add = [&](int32_t e) {
-    if (static_cast<uint32_t>(e) < E)
-      atomicAdd(&hist[static_cast<uint32_t>(e) * 32u + lane], 1u);
-    else
-      ++nbad;
+    const uint32_t ee = static_cast<uint32_t>(e) < E ? static_cast<uint32_t>(e) : E;
+    atomicAdd(&hist[ee * 32u + lane], 1u);
   };
   const int4 *vec = reinterpret_cast<const int4 *>(a.idx);
 
@@ -69,15 +70,16 @@ __global__ void __launch_bounds__(kThreads, 1) count_loads_kernel(CountArgs a) {
     const int64_t b1 = max(g1 & ~int64_t(3), b0);
     if (tid < b0 - g) add(__ldg(a.idx + g + tid));
     if (tid >= 32 && tid - 32 < g1 - b1) add(__ldg(a.idx + b1 + (tid - 32)));
-    const int64_t v1 = b1 >> 2;
-    for (int64_t v = (b0 >> 2) + tid; v < v1; v += kThreads * kU) {
+    const int4 *pin = vec + (b0 >> 2);
+    const int nvec = static_cast<int>((b1 - b0) >> 2);
+    for (int i = tid; i < nvec; i += kThreads * kU) {
       int4 x[kU];
 #pragma unroll
       for (int u = 0; u < kU; ++u)
-        x[u] = v + u * kThreads < v1 ? __ldcs(vec + v + u * kThreads) : make_int4(-1, -1, -1, -1);
+        x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        if (v + u * kThreads < v1) {
+        if (i + u * kThreads < nvec) {
           add(x[u].x);
           add(x[u].y);
           add(x[u].z);
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(kThreads, 1) count_loads_kernel(CountArgs a) {
       }
     }
     __syncthreads();
-    for (int b = tid; b < a.E; b += kThreads) {
+    for (int b = tid; b <= a.E; b += kThreads) {
       uint32_t sum = 0;
 #pragma unroll 8
       for (int j = 0; j < 32; ++j) {
@@ -94,9 +96,12 @@ __global__ void __launch_bounds__(kThreads, 1) count_loads_kernel(CountArgs a) {
         sum += hist[w];
         hist[w] = 0;
       }
-      if (sum)
+      if (sum == 0) continue;
+      if (b < a.E)
         atomicAdd(reinterpret_cast<unsigned long long *>(a.counts + layer * a.E + b),
                   static_cast<unsigned long long>(sum));
+      else
+        nbad += sum;
     }
     __syncthreads();
     g = g1;
@@ -114,7 +119,7 @@ eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer,
   (void)status;  // this kernel has no wait that could run out
   DeviceInfo di;
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
-  const size_t smem = static_cast<size_t>(E) * 32 * sizeof(uint32_t);
+  const size_t smem = static_cast<size_t>(E + 1) * 32 * sizeof(uint32_t);
   if (smem > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
   cudaError_t err = cudaFuncSetAttribute(count_loads_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,

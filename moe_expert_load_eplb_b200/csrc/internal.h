@@ -46,4 +46,15 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
                             int32_t *out, int64_t *counts, unsigned long long *bad,
                             int32_t *status, cudaStream_t stream);
 
+eplb_status launch_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,
+                              int64_t R, int32_t E, int32_t P, int32_t gpus, double *gpu_load,
+                              double *stats, int32_t *status, cudaStream_t stream);
+eplb_status launch_fold_loads(const int64_t *phys, const int32_t *phy2log, int64_t R, int32_t E,
+                              int32_t P, int64_t *logical, int32_t *status, cudaStream_t stream);
+eplb_status launch_initial_map(int64_t R, int32_t E, int32_t P, int32_t *phy2log,
+                               int32_t *phyrank, cudaStream_t stream);
+eplb_status launch_plan_diff(const int32_t *old_p2l, const int32_t *new_p2l, int64_t R, int32_t E,
+                             int32_t P, int32_t gpus, int32_t *src, int32_t *moves,
+                             int32_t *status, cudaStream_t stream);
+
 }  // namespace eplb

@@ -27,11 +27,12 @@
 //     so it never gets an extra replica; the R candidates are selected by
 //     rank and the greedy runs on them alone -- in one lane's registers for
 //     R <= 8, one candidate per lane with an xor-butterfly argmax for R <= 32;
-//   * balanced_packing keeps a node's packs (<= 16) sorted by composite key
-//     (weight << 12 | pack) in one lane's registers: each item takes the
-//     first (lightest, lowest index) pack and re-inserts it with one parallel
-//     compare and two selects, with no shuffle, barrier or memory access on
-//     the chain; wider nodes use one warp per node and a butterfly argmin;
+//   * balanced_packing keeps a node's packs sorted by composite key
+//     (weight << 12 | pack) across the lanes of a segment (one position per
+//     lane up to 32 packs, several per lane up to 256): each item takes the
+//     first (lightest, lowest index) pack, and one ballot + popc gives the
+//     position where the updated pack re-enters; wider nodes use one warp per
+//     node and a butterfly argmin;
 //   * Lambda is lcm(1..cmax) from the host when 64-bit keys can hold it, else
 //     the lcm of the counts present in the node; keys are 64-bit when the
 //     row's magnitudes allow and 128-bit otherwise.  All paths are exact, so
@@ -129,6 +130,22 @@ __device__ __forceinline__ u128 shfl_xor(u128 v, int off) {
   const uint64_t hi = shfl_xor(static_cast<uint64_t>(v >> 64), off);
   return (static_cast<u128>(hi) << 64) | lo;
 }
+__device__ __forceinline__ uint64_t shfl_idx(uint64_t v, int src, int width) {
+  return __shfl_sync(0xffffffffu, static_cast<unsigned long long>(v), src, width);
+}
+__device__ __forceinline__ u128 shfl_idx(u128 v, int src, int width) {
+  const uint64_t lo = shfl_idx(static_cast<uint64_t>(v), src, width);
+  const uint64_t hi = shfl_idx(static_cast<uint64_t>(v >> 64), src, width);
+  return (static_cast<u128>(hi) << 64) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_down_k(uint64_t v, int d, int width) {
+  return __shfl_down_sync(0xffffffffu, static_cast<unsigned long long>(v), d, width);
+}
+__device__ __forceinline__ u128 shfl_down_k(u128 v, int d, int width) {
+  const uint64_t lo = shfl_down_k(static_cast<uint64_t>(v), d, width);
+  const uint64_t hi = shfl_down_k(static_cast<uint64_t>(v >> 64), d, width);
+  return (static_cast<u128>(hi) << 64) | lo;
+}
 template <typename K>
 __device__ __forceinline__ K kmin(K a, K b) {
   return b < a ? b : a;
@@ -166,12 +183,11 @@ __device__ __forceinline__ bool lcm_into(uint64_t &lam, uint32_t c) {
 // ---------------------------------------------------------------------------
 // Descending ranks of n distinct keys in each of nseg segments (segment g at
 // key + g * stride).  Threads are grouped by segment (nthr() / nseg per
-// segment); each ranks up to 4 keys per pass against every key it loads.
-// emit(g, j, rank, key) receives every key.
-template <typename K, typename Emit>
-__device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit emit) {
-  constexpr int Q = 4;
-  const int tps = nseg >= nthr() ? 1 : nthr() / nseg;
+// segment); each ranks Q keys per pass (Q = 1, 2 or 4, the fewest that cover
+// the segment) against every key it loads.  emit(g, j, rank, key) receives
+// every key.
+template <int Q, typename K, typename Emit>
+__device__ void rank_pass(const K *key, int stride, int nseg, int n, int tps, Emit &emit) {
   const int segs_per_pass = nthr() / tps;
   const int sub = threadIdx.x % tps;
   for (int g0 = 0; g0 < nseg; g0 += segs_per_pass) {
@@ -202,6 +218,17 @@ __device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit em
   }
 }
 
+template <typename K, typename Emit>
+__device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit emit) {
+  const int tps = nseg >= nthr() ? 1 : nthr() / nseg;
+  if (n <= tps)
+    rank_pass<1, K>(key, stride, nseg, n, tps, emit);
+  else if (n <= 2 * tps)
+    rank_pass<2, K>(key, stride, nseg, n, tps, emit);
+  else
+    rank_pass<4, K>(key, stride, nseg, n, tps, emit);
+}
+
 // CTA-wide bitonic sort, descending, of nseg segments of npad (power of two)
 // keys each, in place; padding keys must be 0.
 template <typename K>
@@ -226,48 +253,73 @@ __device__ void bitonic_desc(K *key, int npad, int nseg) {
 
 // ---------------------------------------------------------------------------
 // balanced_packing's greedy over items sorted as composite keys
-// (load << 12 | (4095 - item)), descending.  One lane runs one segment.
-// Its m <= MAXM packs are kept sorted ascending by ck = weight << 12 | pack
-// (all ones once full), with each pack's item count alongside; the lightest
-// non-full pack (lowest index on ties) is ck[0], and adding an item's load is
-// one 64- or 128-bit add of (key & ~4095).  After an item is added the pack
-// is re-inserted: lt[k] = ck[k] < new is a prefix, and slot i takes ck[i+1]
-// where lt[i+1], the new key where the prefix ends, else ck[i].
-template <typename K, int MAXM>
-__device__ void pack_lane(const K *skey, int n, int m, int cap, int32_t *ipack, int32_t *irank) {
-  if (n <= 0) return;
+// (load << 12 | (4095 - item)), descending; the pack keys are
+// weight << 12 | pack, so adding an item's load is one add of (key & ~4095).
+//
+// Same greedy with a node's packs spread over the lanes of a segment, in
+// sorted order: for m <= 32 a segment is the next power of two >= m lanes
+// with one position each; for larger m a segment is a whole warp and lane l
+// holds positions l*PL .. l*PL+PL-1.  Per item: position 0 (the lightest,
+// lowest index on ties) is broadcast, every lane compares its keys with the
+// pack's new key, one ballot + popc gives the insertion point p among the
+// remaining positions, and position i takes the key of position i+1 (i < p),
+// the new key (i == p) or keeps its own (i > p).  Counts move with keys.
+template <typename K, int PL>
+__device__ void pack_seg(const K *skey_base, int stride, int nseg, int n, int m, int cap,
+                         int32_t *ipack, int32_t *irank, int out_stride) {
   const K imask = K(kIdxMask);
   const K kmax = ~K(0);
-  K ck[MAXM];
-  int pc[MAXM];
+  int ms = 2;  // lanes per segment
+  while (ms < m && ms < 32) ms <<= 1;
+  if (PL > 1) ms = 32;
+  const int lane = threadIdx.x & 31;
+  const int li = lane & (ms - 1);            // lane within the segment
+  const unsigned segmask = ms == 32 ? 0xffffffffu : ((1u << ms) - 1u) << (lane & ~(ms - 1));
+  const int slot = static_cast<int>(threadIdx.x) / ms;
+  const int slots = nthr() / ms;
+  const int warp_first_slot = (static_cast<int>(threadIdx.x) & ~31) / ms;
+  for (int g0 = 0; g0 < nseg; g0 += slots) {
+    if (g0 + warp_first_slot >= nseg) continue;  // no segment of this warp is live: skip the chain
+    const int g = g0 + slot;
+    const bool active = g < nseg;
+    const K *skey = skey_base + (active ? g : 0) * stride;
+    K key[PL];
+    int cnt[PL];
 #pragma unroll
-  for (int k = 0; k < MAXM; ++k) {
-    ck[k] = k < m ? K(k) : kmax;
-    pc[k] = 0;
-  }
-  K nxt = skey[0];
-  for (int j = 0; j < n; ++j) {
-    const K c = nxt;
-    if (j + 1 < n) nxt = skey[j + 1];
-    const K best = ck[0];
-    const int r = pc[0];
-    const K nk = r + 1 < cap ? best + (c & ~imask) : kmax;
-    bool lt[MAXM + 1];
-    lt[0] = true;
-    lt[MAXM] = false;
-#pragma unroll
-    for (int k = 1; k < MAXM; ++k) lt[k] = ck[k] < nk;
-#pragma unroll
-    for (int i = 0; i < MAXM; ++i) {
-      const bool here = lt[i] && !lt[i + 1];
-      const K up = i + 1 < MAXM ? ck[i + 1] : kmax;
-      const int upc = i + 1 < MAXM ? pc[i + 1] : 0;
-      ck[i] = lt[i + 1] ? up : (here ? nk : ck[i]);
-      pc[i] = lt[i + 1] ? upc : (here ? r + 1 : pc[i]);
+    for (int r = 0; r < PL; ++r) {
+      const int pos = li * PL + r;
+      key[r] = pos < m ? K(pos) : kmax;  // pack pos, weight 0
+      cnt[r] = 0;
     }
-    const int item = static_cast<int>(imask - (c & imask));
-    ipack[item] = static_cast<int>(best & imask);
-    irank[item] = r;
+    K nxt = skey[0];
+    for (int j = 0; j < n; ++j) {
+      const K c = nxt;
+      if (j + 1 < n) nxt = skey[j + 1];
+      const K best = shfl_idx(key[0], 0, ms);
+      const int bc = __shfl_sync(0xffffffffu, cnt[0], 0, ms);
+      const K up = shfl_down_k(key[0], 1, ms);  // position (li+1)*PL of the next lane
+      const int upc = __shfl_down_sync(0xffffffffu, cnt[0], 1, ms);
+      const K nk = bc + 1 < cap ? best + (c & ~imask) : kmax;
+      int p = 0;
+#pragma unroll
+      for (int r = 0; r < PL; ++r) {
+        const bool lt = (li * PL + r) >= 1 && key[r] < nk;
+        p += __popc(__ballot_sync(0xffffffffu, lt) & segmask);
+      }
+#pragma unroll
+      for (int r = 0; r < PL; ++r) {
+        const int pos = li * PL + r;
+        const K right = r + 1 < PL ? key[r + 1 < PL ? r + 1 : r] : up;
+        const int rightc = r + 1 < PL ? cnt[r + 1 < PL ? r + 1 : r] : upc;
+        key[r] = pos < p ? right : (pos == p ? nk : key[r]);
+        cnt[r] = pos < p ? rightc : (pos == p ? bc + 1 : cnt[r]);
+      }
+      if (li == 0 && active) {
+        const int item = static_cast<int>(imask - (c & imask));
+        ipack[g * out_stride + item] = static_cast<int>(best & imask);
+        irank[g * out_stride + item] = bc;
+      }
+    }
   }
 }
 
@@ -311,19 +363,20 @@ __device__ void pack_warp(const K *skey, int n, int m, int cap, K *pw, int32_t *
 }
 
 // Packs nseg segments (segment g: n sorted keys at skey + g * stride, results
-// at ipack/irank + g * out_stride) into m packs of cap items each.
+// at ipack/irank + g * out_stride) into m packs of cap items each.  Called by
+// every thread of the CTA (the lane-parallel variant needs whole warps).
 template <typename K>
 __device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
                               int32_t *pc, int32_t *ipack, int32_t *irank, int out_stride) {
-  // 128-bit keys keep the register variant to 8 packs (register pressure)
-  if (m <= 8 || (m <= 16 && sizeof(K) == 8)) {
-    for (int g = threadIdx.x; g < nseg; g += nthr()) {
-      if (m <= 8)
-        pack_lane<K, 8>(skey + g * stride, n, m, cap, ipack + g * out_stride, irank + g * out_stride);
-      else
-        pack_lane<K, (sizeof(K) == 8 ? 16 : 8)>(skey + g * stride, n, m, cap, ipack + g * out_stride,
-                                                irank + g * out_stride);
-    }
+  if (n <= 0) return;
+  if (m <= 32) {
+    pack_seg<K, 1>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
+  } else if (m <= 64) {
+    pack_seg<K, 2>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
+  } else if (m <= 128) {
+    pack_seg<K, 4>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
+  } else if (m <= 256 && sizeof(K) == 8) {
+    pack_seg<K, 8>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
   } else {
     for (int g = threadIdx.x >> 5; g < nseg; g += nwarps())
       pack_warp<K>(skey + g * stride, n, m, cap, pw + g * m, pc + g * m, ipack + g * out_stride,

@@ -44,16 +44,22 @@ struct RedirectArgs {
 
 template <bool kVecToken, bool kCount>
 __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
+  // Tables carry a sentinel row E: an index outside [0, E) maps to it, so the
+  // per-index path has no branch -- its log2phy entry is -1 and its histogram
+  // bin (kCount) counts the bad indices.  An expert whose logcnt is outside
+  // [1, X] gets logcnt 1 and a -1 entry in the shared copy (reported once).
   extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t *hist = reinterpret_cast<uint32_t *>(smem);  // [E][32], kCount only
-  uint2 *cm = reinterpret_cast<uint2 *>(smem + (kCount ? a.E * 32 * sizeof(uint32_t) : 0));
-  int32_t *l2p = reinterpret_cast<int32_t *>(cm + a.E);
+  const int E1 = a.E + 1;
+  uint32_t *hist = reinterpret_cast<uint32_t *>(smem);  // [E+1][32], kCount only
+  uint2 *cm = reinterpret_cast<uint2 *>(smem + (kCount ? E1 * 32 * sizeof(uint32_t) : 0));
+  int32_t *l2p = reinterpret_cast<int32_t *>(cm + E1);  // [E+1][X]
   const int tid = threadIdx.x;
-  const int lane = tid & 31;
+  const uint32_t lane = tid & 31;
   if (kCount) {
-    for (int i = tid; i < a.E * 32; i += kThreads) hist[i] = 0;
+    for (int i = tid; i < E1 * 32; i += kThreads) hist[i] = 0;
   }
   const uint32_t E = static_cast<uint32_t>(a.E);
+  const uint32_t X = static_cast<uint32_t>(a.X);
   const int EX = a.E * a.X;
 
   const int64_t r0 = (a.total * blockIdx.x / gridDim.x) & ~int64_t(3);
@@ -64,20 +70,15 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
   bool range_err = false;
   // physical index of element value e whose token is tok (global)
   auto map = [&](int32_t e, uint32_t tok) -> int32_t {
-    if (static_cast<uint32_t>(e) >= E) {
-      ++nbad;
-      return -1;
-    }
-    if (kCount) atomicAdd(&hist[static_cast<uint32_t>(e) * 32u + lane], 1u);
-    const uint2 c = cm[e];
-    if (c.x == 0) {
-      range_err = true;
-      return -1;
-    }
-    return l2p[e * a.X + static_cast<int>(mod_magic(tok, c.x, c.y))];
+    const bool ok = static_cast<uint32_t>(e) < E;
+    const uint32_t ee = ok ? static_cast<uint32_t>(e) : E;
+    if (kCount)
+      atomicAdd(&hist[ee * 32u + lane], 1u);
+    else
+      nbad += ok ? 0u : 1u;
+    const uint2 c = cm[ee];
+    return l2p[ee * X + mod_magic(tok, c.x, c.y)];
   };
-  const int4 *vin = reinterpret_cast<const int4 *>(a.idx);
-  int4 *vout = reinterpret_cast<int4 *>(a.out);
 
   int64_t g = r0;
   while (g < r1) {
@@ -85,15 +86,20 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
     const int64_t lbase = layer * a.per_layer;
     const int64_t g1 = min(r1, lbase + a.per_layer);
     __syncthreads();  // previous segment's table reads are done
-    const int32_t *cnt = a.logcnt + layer * a.E;
-    for (int e = tid; e < a.E; e += kThreads) {
-      const int32_t c = __ldg(cnt + e);
-      const bool valid = c >= 1 && c <= a.X;
-      cm[e] = make_uint2(valid ? static_cast<uint32_t>(c) : 0u,
-                         valid ? 0xffffffffu / static_cast<uint32_t>(c) : 0u);
-    }
     const int32_t *src = a.log2phy + layer * EX;
     for (int i = tid; i < EX; i += kThreads) l2p[i] = __ldg(src + i);
+    if (tid < a.X) l2p[EX + tid] = -1;
+    __syncthreads();
+    const int32_t *cnt = a.logcnt + layer * a.E;
+    for (int e = tid; e <= a.E; e += kThreads) {
+      int32_t c = e < a.E ? __ldg(cnt + e) : 1;
+      if (c < 1 || c > a.X) {
+        range_err = true;
+        c = 1;
+        l2p[e * a.X] = -1;
+      }
+      cm[e] = make_uint2(static_cast<uint32_t>(c), 0xffffffffu / static_cast<uint32_t>(c));
+    }
     __syncthreads();
 
     const int64_t b0 = min((g + 3) & ~int64_t(3), g1);
@@ -108,17 +114,21 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
       a.out[p] = map(__ldg(a.idx + p),
                      a.t0 + div_magic(static_cast<uint32_t>(p - lbase), a.K, a.k_magic));
     }
-    const int64_t v1 = b1 >> 2;
-    for (int64_t v = (b0 >> 2) + tid; v < v1; v += kThreads * kU) {
+    // 16-byte vectors of this segment, indexed from its first one (32-bit)
+    const int4 *pin = reinterpret_cast<const int4 *>(a.idx + b0);
+    int4 *pout = reinterpret_cast<int4 *>(a.out + b0);
+    const int nvec = static_cast<int>((b1 - b0) >> 2);
+    const uint32_t pos0 = static_cast<uint32_t>(b0 - lbase);
+    for (int i = tid; i < nvec; i += kThreads * kU) {
       int4 x[kU];
 #pragma unroll
       for (int u = 0; u < kU; ++u)
-        x[u] = v + u * kThreads < v1 ? __ldcs(vin + v + u * kThreads) : make_int4(0, 0, 0, 0);
+        x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        const int64_t vv = v + u * kThreads;
-        if (vv < v1) {
-          const uint32_t pos = static_cast<uint32_t>(vv * 4 - lbase);
+        const int v = i + u * kThreads;
+        if (v < nvec) {
+          const uint32_t pos = pos0 + 4u * static_cast<uint32_t>(v);
           int4 y;
           if (kVecToken) {
             const uint32_t tok = a.t0 + div_magic(pos, a.K, a.k_magic);
@@ -132,13 +142,13 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
             y.z = map(x[u].z, a.t0 + div_magic(pos + 2, a.K, a.k_magic));
             y.w = map(x[u].w, a.t0 + div_magic(pos + 3, a.K, a.k_magic));
           }
-          __stcs(vout + vv, y);
+          __stcs(pout + v, y);
         }
       }
     }
     if (kCount) {
       __syncthreads();
-      for (int b = tid; b < a.E; b += kThreads) {
+      for (int b = tid; b <= a.E; b += kThreads) {
         uint32_t sum = 0;
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) {
@@ -146,9 +156,12 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
           sum += hist[w];
           hist[w] = 0;
         }
-        if (sum)
+        if (sum == 0) continue;
+        if (b < a.E)
           atomicAdd(reinterpret_cast<unsigned long long *>(a.counts + layer * a.E + b),
                     static_cast<unsigned long long>(sum));
+        else
+          nbad += sum;
       }
     }
     g = g1;
@@ -156,7 +169,7 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
 
   if (range_err) report(a.status, EPLB_ERR_RANGE);
   for (int off = 16; off > 0; off >>= 1) nbad += __shfl_xor_sync(0xffffffffu, nbad, off);
-  if ((tid & 31) == 0 && nbad && a.bad) atomicAdd(a.bad, static_cast<unsigned long long>(nbad));
+  if (lane == 0 && nbad && a.bad) atomicAdd(a.bad, static_cast<unsigned long long>(nbad));
 }
 
 }  // namespace
@@ -168,8 +181,8 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
   DeviceInfo di;
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
   const bool count = counts != nullptr;
-  const size_t smem = (count ? static_cast<size_t>(E) * 32 * sizeof(uint32_t) : 0) +
-                      static_cast<size_t>(E) * 8 + static_cast<size_t>(E) * X * sizeof(int32_t);
+  const size_t smem = (count ? static_cast<size_t>(E + 1) * 32 * sizeof(uint32_t) : 0) +
+                      static_cast<size_t>(E + 1) * 8 + static_cast<size_t>(E + 1) * X * sizeof(int32_t);
   if (smem > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
   RedirectArgs a;
   a.idx = idx;

@@ -59,6 +59,14 @@ def _load():
         lib.oracle_balanced_packing_frac.restype = ctypes.c_int
         lib.oracle_replicate_experts.argtypes = [p, i32, i32, p, p, p]
         lib.oracle_replicate_experts.restype = None
+        lib.oracle_plan_stats.argtypes = [p, p, p, i64, i32, i32, i32, p, p]
+        lib.oracle_plan_stats.restype = None
+        lib.oracle_fold_loads.argtypes = [p, p, i64, i32, i32, p]
+        lib.oracle_fold_loads.restype = None
+        lib.oracle_initial_map.argtypes = [i64, i32, i32, p, p]
+        lib.oracle_initial_map.restype = None
+        lib.oracle_plan_diff.argtypes = [p, p, i64, i32, i32, i32, p, p]
+        lib.oracle_plan_diff.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -177,3 +185,51 @@ def replicate_experts(weight, num_phy: int):
     c = np.empty(n, dtype=np.int32)
     _load().oracle_replicate_experts(_ptr(w), n, num_phy, _ptr(p), _ptr(r), _ptr(c))
     return p, r, c
+
+
+def plan_stats(loads, phy2log, logcnt, num_gpus: int):
+    """Per-GPU load (sum of w/logcnt over the GPU's replicas, fp64, slot order)
+    and per-row {min, max, mean, mean/max}."""
+    loads = _c(loads, np.int64)
+    phy2log = _c(phy2log, np.int32)
+    logcnt = _c(logcnt, np.int32)
+    R, E = loads.shape
+    P = phy2log.shape[1]
+    gl = np.empty((R, num_gpus), dtype=np.float64)
+    st = np.empty((R, 4), dtype=np.float64)
+    _load().oracle_plan_stats(_ptr(loads), _ptr(phy2log), _ptr(logcnt), R, E, P, num_gpus,
+                              _ptr(gl), _ptr(st))
+    return gl, st
+
+
+def fold_loads(phys, phy2log, num_logical: int):
+    """logical[r, e] = sum of phys[r, p] over slots p with phy2log[r, p] == e."""
+    phys = _c(phys, np.int64)
+    phy2log = _c(phy2log, np.int32)
+    R, P = phys.shape
+    out = np.empty((R, num_logical), dtype=np.int64)
+    _load().oracle_fold_loads(_ptr(phys), _ptr(phy2log), R, num_logical, P, _ptr(out))
+    return out
+
+
+def initial_map(R: int, num_logical: int, num_replicas: int):
+    """phy2log[p] = p mod E (routed experts first, then redundant), phyrank = p div E."""
+    p2l = np.empty((R, num_replicas), dtype=np.int32)
+    prk = np.empty((R, num_replicas), dtype=np.int32)
+    _load().oracle_initial_map(R, num_logical, num_replicas, _ptr(p2l), _ptr(prk))
+    return p2l, prk
+
+
+def plan_diff(old_phy2log, new_phy2log, num_logical: int, num_gpus: int):
+    """src[r, p]: -1 if new slot p's expert stays on its GPU, else the old slot to copy
+    from; moves[r]: number of copies."""
+    old = _c(old_phy2log, np.int32)
+    new = _c(new_phy2log, np.int32)
+    R, P = new.shape
+    src = np.empty((R, P), dtype=np.int32)
+    moves = np.empty(R, dtype=np.int32)
+    rc = _load().oracle_plan_diff(_ptr(old), _ptr(new), R, num_logical, P, num_gpus, _ptr(src),
+                                  _ptr(moves))
+    if rc != OK:
+        raise OracleError(rc)
+    return src, moves

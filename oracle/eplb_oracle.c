@@ -413,3 +413,97 @@ void oracle_replicate_experts(const int64_t *weight, int32_t num_log,
   for (int i = 0; i < num_log; ++i) logcnt[i] = c[i];
   free(p); free(r); free(c);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Plan quality ([EPLB] box "От переводчика: что сделать руками", exercise  */
+/* 2, and the per-GPU load range of "От переводчика: что на рисунке"): the   */
+/* load of GPU g is the sum of w[e] / logcnt[e] over its replicas.  fp64,    */
+/* summed in slot order p = g*ppg, g*ppg + 1, ...; stats[r] = {min, max,     */
+/* mean, mean / max} over the GPUs (balancedness 1 when max is 0).           */
+/* ------------------------------------------------------------------------ */
+void oracle_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,
+                       int64_t R, int32_t E, int32_t P, int32_t gpus, double *gpu_load,
+                       double *stats) {
+  const int ppg = P / gpus;
+  for (int64_t r = 0; r < R; ++r) {
+    double mn = 0, mx = 0, sum = 0;
+    for (int g = 0; g < gpus; ++g) {
+      double acc = 0.0;
+      for (int k = 0; k < ppg; ++k) {
+        int e = phy2log[r * P + g * ppg + k];
+        acc += (double)loads[r * E + e] / (double)logcnt[r * E + e];
+      }
+      gpu_load[r * gpus + g] = acc;
+      if (g == 0 || acc < mn) mn = acc;
+      if (g == 0 || acc > mx) mx = acc;
+      sum += acc;
+    }
+    double mean = sum / gpus;
+    stats[r * 4 + 0] = mn;
+    stats[r * 4 + 1] = mx;
+    stats[r * 4 + 2] = mean;
+    stats[r * 4 + 3] = mx > 0 ? mean / mx : 1.0;
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Physical -> logical load fold: logical[r, e] = sum of phys[r, p] over the */
+/* physical slots p with phy2log[r, p] == e (the serving engine records      */
+/* load per physical expert and folds it before rebalancing).                */
+/* ------------------------------------------------------------------------ */
+void oracle_fold_loads(const int64_t *phys, const int32_t *phy2log, int64_t R, int32_t E,
+                       int32_t P, int64_t *logical) {
+  memset(logical, 0, sizeof(int64_t) * (size_t)(R * E));
+  for (int64_t r = 0; r < R; ++r)
+    for (int p = 0; p < P; ++p) logical[r * E + phy2log[r * P + p]] += phys[r * P + p];
+}
+
+/* Initial map: routed experts first, then the redundant slots cycle through */
+/* the experts from 0 (phy2log[p] = p mod E, phyrank[p] = p div E).          */
+void oracle_initial_map(int64_t R, int32_t E, int32_t P, int32_t *phy2log, int32_t *phyrank) {
+  for (int64_t r = 0; r < R; ++r)
+    for (int p = 0; p < P; ++p) {
+      phy2log[r * P + p] = p % E;
+      phyrank[r * P + p] = p / E;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Plan diff: which new physical slots need their expert's weights copied.   */
+/* GPU g keeps min(old_g(e), new_g(e)) replicas of expert e in place; going  */
+/* through g's new slots in order, a slot whose expert still has a kept      */
+/* replica to spare is kept (src = -1), every other slot copies from the     */
+/* lowest old physical slot that held its expert.  moves[r] = slots copied.  */
+/* ------------------------------------------------------------------------ */
+int oracle_plan_diff(const int32_t *old_p2l, const int32_t *new_p2l, int64_t R, int32_t E,
+                     int32_t P, int32_t gpus, int32_t *src, int32_t *moves) {
+  if (gpus <= 0 || P % gpus != 0) return ORACLE_ERR_DIVISIBILITY;
+  const int ppg = P / gpus;
+  int *first_old = (int *)malloc(sizeof(int) * (size_t)E);
+  int *old_cnt = (int *)malloc(sizeof(int) * (size_t)E);
+  if (!first_old || !old_cnt) { free(first_old); free(old_cnt); return ORACLE_ERR_ALLOC; }
+  for (int64_t r = 0; r < R; ++r) {
+    const int32_t *o = old_p2l + r * P, *n = new_p2l + r * P;
+    for (int e = 0; e < E; ++e) first_old[e] = -1;
+    for (int p = P - 1; p >= 0; --p) first_old[o[p]] = p;
+    int m = 0;
+    for (int g = 0; g < gpus; ++g) {
+      for (int e = 0; e < E; ++e) old_cnt[e] = 0;
+      for (int k = 0; k < ppg; ++k) old_cnt[o[g * ppg + k]] += 1;
+      for (int k = 0; k < ppg; ++k) {
+        int p = g * ppg + k, e = n[p];
+        if (old_cnt[e] > 0) {
+          old_cnt[e] -= 1;
+          src[r * P + p] = -1;
+        } else {
+          src[r * P + p] = first_old[e];
+          ++m;
+        }
+      }
+    }
+    moves[r] = m;
+  }
+  free(first_old);
+  free(old_cnt);
+  return ORACLE_OK;
+}

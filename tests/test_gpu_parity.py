@@ -459,3 +459,90 @@ def test_pipeline_serving_order_c2(c2_idx):
         ring[(W_ - 1 + s_i) % W_] = counts
         plan_ref = _oracle_plan_from_ring(ring, c, step.X)
         _assert_plan_equal(step.plan, plan_ref)
+
+
+# ------------------------------------------- plan stats, fold, initial map, diff --
+
+def _plans_for(c, loads_np):
+    return oracle.rebalance(loads_np, c.P, c.G, c.N, c.gpus)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_plan_stats_matches_oracle(cfg, request):
+    c = W.CONFIGS[cfg]
+    if cfg == 3:
+        loads_np = W.c3_loads()
+    else:
+        idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx"}[cfg])
+        loads_np, _ = oracle.count_loads(_np(idx), c.E)
+    p2l, _, cnt, _ = _plans_for(c, loads_np)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    st_word = _status()
+    gl, st = eplb.plan_stats(dev(loads_np), dev(p2l), dev(cnt), c.gpus, status=st_word)
+    ref_gl, ref_st = oracle.plan_stats(loads_np, p2l, cnt, c.gpus)
+    # fp64, same operations in the same order: identical bits
+    assert np.array_equal(_np(gl), ref_gl) and np.array_equal(_np(st), ref_st)
+    assert int(st_word.item()) == 0
+
+
+def test_plan_stats_worked_example_gpu():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "eplb_readme_example.json")) as f:
+        ex = json.load(f)
+    w = np.array(ex["weight"], dtype=np.int64)
+    plan = eplb.rebalance(torch.from_numpy(w).to(DEV), 16, 4, 2, 8)
+    _, st = eplb.plan_stats(torch.from_numpy(w).to(DEV), plan.phy2log, plan.logcnt, 8)
+    h = ex["layer0_gpu_load_hierarchical"]
+    assert _np(st)[0, 0] == h["min"] and _np(st)[0, 1] == h["max"]
+
+
+@pytest.mark.parametrize("shape", [(58, 256, 288), (3, 12, 16), (1000, 64, 96), (2, 1, 1)])
+def test_fold_loads_matches_oracle(shape):
+    R, E, P = shape
+    rng = np.random.default_rng(R + E + P)
+    p2l = rng.integers(0, E, (R, P)).astype(np.int32)
+    phys = rng.integers(0, 1 << 40, (R, P))
+    got = eplb.fold_loads(torch.from_numpy(phys).to(DEV), torch.from_numpy(p2l).to(DEV), E)
+    assert np.array_equal(_np(got), oracle.fold_loads(phys, p2l, E))
+
+
+def test_fold_of_physical_counts_after_redirect(c2_idx):
+    c = W.CONFIGS[2]
+    counts = eplb.count_loads(c2_idx, c.E)
+    plan = eplb.rebalance(counts, c.P, c.G, c.N, c.gpus)
+    out = eplb.redirect(c2_idx, plan.log2phy, plan.logcnt)
+    phys = eplb.count_loads(out, c.P)
+    assert torch.equal(eplb.fold_loads(phys, plan.phy2log, c.E), counts)
+
+
+def test_initial_map_matches_oracle():
+    p2l, prk = eplb.initial_map(58, 256, 288, device=DEV)
+    ref_p, ref_r = oracle.initial_map(58, 256, 288)
+    assert np.array_equal(_np(p2l), ref_p) and np.array_equal(_np(prk), ref_r)
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_plan_diff_matches_oracle(cfg, c4_steps):
+    c = W.CONFIGS[cfg]
+    if cfg == 3:
+        old_l = W.c3_loads()
+        new_l = np.roll(old_l, 1, axis=1)
+    else:
+        snaps = _np(c4_steps)
+        old_l, new_l = snaps[10], snaps[900]
+    old = _plans_for(c, old_l)[0]
+    new = _plans_for(c, new_l)[0]
+    src, moves = eplb.plan_diff(torch.from_numpy(old).to(DEV), torch.from_numpy(new).to(DEV),
+                                c.E, c.gpus)
+    ref_src, ref_moves = oracle.plan_diff(old, new, c.E, c.gpus)
+    assert np.array_equal(_np(src), ref_src) and np.array_equal(_np(moves), ref_moves)
+
+
+def test_plan_diff_initial_to_first_plan(c2_idx):
+    c = W.CONFIGS[2]
+    init, _ = eplb.initial_map(c.L, c.E, c.P, device=DEV)
+    plan = eplb.rebalance(eplb.count_loads(c2_idx, c.E), c.P, c.G, c.N, c.gpus)
+    src, moves = eplb.plan_diff(init, plan.phy2log, c.E, c.gpus)
+    ref_src, ref_moves = oracle.plan_diff(_np(init), _np(plan.phy2log), c.E, c.gpus)
+    assert np.array_equal(_np(src), ref_src) and np.array_equal(_np(moves), ref_moves)

@@ -392,3 +392,100 @@ def test_redirect_shards_concatenate():
     a, _ = oracle.redirect(idx[:, :37], l2p, cnt, 0)
     b, _ = oracle.redirect(idx[:, 37:], l2p, cnt, 37)
     assert (np.concatenate([a, b], axis=1) == whole).all()
+
+
+# --------------------------------------------------------------------------
+# Plan quality, physical-load fold, initial map, plan diff
+# --------------------------------------------------------------------------
+
+def test_plan_stats_worked_example(ex):
+    # the per-GPU loads the page prints for layer 0, both policies
+    w = np.array(ex["weight"], dtype=np.int64)
+    for G, key in ((4, "layer0_gpu_load_hierarchical"), (3, "layer0_gpu_load_global_groups3")):
+        p2l, _, cnt, _ = oracle.rebalance(w, 16, G, 2, 8)
+        gl, st = oracle.plan_stats(w, p2l, cnt, 8)
+        exact = gpu_loads(w[0], p2l[0], cnt[0], 8)
+        assert [float(x) for x in exact] == gl[0].tolist()
+        assert st[0, 0] == ex[key]["min"] and st[0, 1] == ex[key]["max"]
+        assert st[0, 2] == float(sum(exact) / 8) and st[0, 3] == st[0, 2] / st[0, 1]
+        assert round(st[0, 2]) == ex["layer0_gpu_load_hierarchical"]["mean_rounded"]
+
+
+def test_plan_stats_zero_loads_are_balanced():
+    w = np.zeros((2, 12), dtype=np.int64)
+    p2l, _, cnt, _ = oracle.rebalance(w, 16, 4, 2, 8)
+    gl, st = oracle.plan_stats(w, p2l, cnt, 8)
+    assert (gl == 0).all() and (st[:, 3] == 1.0).all()
+
+
+def test_fold_is_weighted_bincount():
+    rng = np.random.default_rng(5)
+    R, E, P = 4, 12, 20
+    p2l = rng.integers(0, E, (R, P)).astype(np.int32)
+    phys = rng.integers(0, 1 << 40, (R, P))
+    got = oracle.fold_loads(phys, p2l, E)
+    for r in range(R):
+        want = np.zeros(E, dtype=np.int64)
+        np.add.at(want, p2l[r], phys[r])
+        assert (got[r] == want).all()
+
+
+def test_fold_of_redirected_counts_is_the_logical_count():
+    # counting redirected (physical) indices and folding gives the logical counts
+    rng = np.random.default_rng(6)
+    L, T, K, E, P = 2, 300, 4, 12, 16
+    p2l, prk, cnt, l2p = oracle.rebalance(rng.integers(0, 99, (L, E)), P, 4, 2, 8)
+    idx = rng.integers(0, E, (L, T, K)).astype(np.int32)
+    out, _ = oracle.redirect(idx, l2p, cnt)
+    phys, _ = oracle.count_loads(out, P)
+    logical, _ = oracle.count_loads(idx, E)
+    assert (oracle.fold_loads(phys, p2l, E) == logical).all()
+
+
+def test_initial_map_closed_form():
+    p2l, prk = oracle.initial_map(3, 256, 288)
+    assert (p2l == np.arange(288) % 256).all() and (prk == np.arange(288) // 256).all()
+
+
+def test_plan_diff_identity_and_swap():
+    rng = np.random.default_rng(9)
+    w = rng.integers(0, 500, (3, 24))
+    p2l, _, _, _ = oracle.rebalance(w, 32, 6, 2, 8)
+    src, moves = oracle.plan_diff(p2l, p2l, 24, 8)
+    assert (src == -1).all() and (moves == 0).all()
+    # swapping the contents of GPUs 0 and 1 (4 slots each) moves every slot of
+    # both GPUs whose expert the other GPU did not hold
+    swapped = p2l.copy()
+    swapped[:, 0:4], swapped[:, 4:8] = p2l[:, 4:8], p2l[:, 0:4]
+    src, moves = oracle.plan_diff(p2l, swapped, 24, 8)
+    assert (src[:, 8:] == -1).all()
+    for r in range(3):
+        for g, other in ((0, 1), (1, 0)):
+            for k in range(4):
+                p = g * 4 + k
+                e = swapped[r, p]
+                if e in p2l[r, g * 4:(g + 1) * 4]:
+                    continue
+                assert src[r, p] == int(np.flatnonzero(p2l[r] == e)[0])
+
+
+@pytest.mark.parametrize("seed", range(20))
+def test_plan_diff_invariants(seed):
+    rng = np.random.default_rng(400 + seed)
+    E, P, gpus = 16, 32, 8
+    a, _, _, _ = oracle.rebalance(rng.integers(0, 300, (2, E)), P, 4, 2, gpus)
+    b, _, _, _ = oracle.rebalance(rng.integers(0, 300, (2, E)), P, 4, 2, gpus)
+    src, moves = oracle.plan_diff(a, b, E, gpus)
+    ppg = P // gpus
+    for r in range(2):
+        assert moves[r] == int((src[r] != -1).sum())
+        for g in range(gpus):
+            old = list(a[r, g * ppg:(g + 1) * ppg])
+            new = list(b[r, g * ppg:(g + 1) * ppg])
+            kept = [int(b[r, g * ppg + k]) for k in range(ppg) if src[r, g * ppg + k] == -1]
+            for e in set(new):
+                assert kept.count(e) == min(old.count(e), new.count(e))
+            for k in range(ppg):
+                s = src[r, g * ppg + k]
+                if s != -1:
+                    assert a[r, s] == b[r, g * ppg + k]   # the copy source holds the expert
