@@ -134,6 +134,25 @@ eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P
                            int32_t *log2phy, int32_t *status, cudaStream_t stream);
 
 /*
+ * S2 + S3/S4 for a serving ring -- rebalance from the window sum of a ring
+ * of per-step counts, in one launch:
+ *   loads[r, e] = sum_{w < W} ring[w, r, e]     (the window of the last W
+ *                 steps, row order irrelevant: eplb_window_accumulate with
+ *                 S = W, s_first = W - 1)
+ * then exactly eplb_rebalance on those loads (same outputs, limits, errors).
+ * ring       device int64 [W, R, E]; each window sum must lie in [0, 2^40).
+ * zero_slot  -1, or the ring row to clear after it has been read (the slot
+ *            the next step's counts go to, e.g. with eplb_count_redirect and
+ *            accumulate = 1); the rest of the ring is only read.
+ * loads_out  device int64 [R, E], nullable: receives the window sums.
+ */
+eplb_status eplb_rebalance_window(int64_t *ring, int64_t W, int64_t zero_slot, int64_t R,
+                                  int32_t E, int32_t P, int32_t G, int32_t N, int32_t gpus,
+                                  int32_t X, int64_t *loads_out, int32_t *phy2log,
+                                  int32_t *phyrank, int32_t *logcnt, int32_t *log2phy,
+                                  int32_t *status, cudaStream_t stream);
+
+/*
  * S5 -- redirect logical expert indices to physical replicas ([LPLB] usage
  * example: logical indices in, physical indices out).  Replica rule (this
  * library's fixed choice; the pages leave it open): token t of the call is

@@ -25,7 +25,7 @@ import torch
 
 __all__ = [
     "EplbError", "Plan", "count_loads", "window_accumulate", "rebalance", "redirect", "count_redirect",
-    "plan_stats", "fold_loads", "initial_map", "plan_diff",
+    "plan_stats", "fold_loads", "initial_map", "plan_diff", "rebalance_window",
     "default_slots", "lib_path", "load_library", "STATUS",
 ]
 
@@ -82,6 +82,8 @@ def load_library():
         "eplb_redirect": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, p], i32),
         "eplb_count_redirect": ([p, i64, i64, i32, i32, p, i32, p, i32, p, i64, p, p, p, p], i32),
         "eplb_plan_stats": ([p, p, p, i64, i32, i32, i32, p, p, p, p], i32),
+        "eplb_rebalance_window": ([p, i64, i64, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p, p],
+                                  i32),
         "eplb_fold_loads": ([p, p, i64, i32, i32, p, p, p], i32),
         "eplb_initial_map": ([i64, i32, i32, p, p, p], i32),
         "eplb_plan_diff": ([p, p, i64, i32, i32, i32, p, p, p, p], i32),
@@ -192,6 +194,42 @@ def rebalance(loads: torch.Tensor, num_replicas: int, num_groups: int, num_nodes
             _ptr(loads), R, E, P, num_groups, num_nodes, num_gpus, X,
             _ptr(out.phy2log), _ptr(out.phyrank), _ptr(out.logcnt), _ptr(out.log2phy),
             _ptr(status), _stream(dev)), "eplb_rebalance")
+    return out
+
+
+def rebalance_window(ring: torch.Tensor, num_replicas: int, num_groups: int, num_nodes: int,
+                     num_gpus: int, zero_slot: int = -1, slots: Optional[int] = None,
+                     out: Optional[Plan] = None, loads_out: Optional[torch.Tensor] = None,
+                     status: Optional[torch.Tensor] = None) -> Plan:
+    """S2 + S3/S4 in one launch: rebalance_experts on the window sum of a ring of
+    per-step counts (int64 [W, R, E]); zero_slot >= 0 clears that ring row after
+    reading it (the next step's counting slot)."""
+    _cuda(ring, torch.int64, "ring")
+    if ring.dim() != 3:
+        raise ValueError("ring must be [W, R, E]")
+    Wr, R, E = ring.shape
+    P = num_replicas
+    X = default_slots(E, P, num_groups, num_nodes) if slots is None else slots
+    dev = ring.device
+    if out is None:
+        out = Plan(torch.empty((R, P), dtype=torch.int32, device=dev),
+                   torch.empty((R, P), dtype=torch.int32, device=dev),
+                   torch.empty((R, E), dtype=torch.int32, device=dev),
+                   torch.empty((R, E, X), dtype=torch.int32, device=dev))
+    for name, t, shape in (("phy2log", out.phy2log, (R, P)), ("phyrank", out.phyrank, (R, P)),
+                           ("logcnt", out.logcnt, (R, E)), ("log2phy", out.log2phy, (R, E, X))):
+        _cuda(t, torch.int32, name)
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be {shape}")
+    if loads_out is not None:
+        _cuda(loads_out, torch.int64, "loads_out")
+        if tuple(loads_out.shape) not in ((R, E), (1, R, E)):
+            raise ValueError("loads_out must be [R, E]")
+    with torch.cuda.device(dev):
+        _check(load_library().eplb_rebalance_window(
+            _ptr(ring), Wr, zero_slot, R, E, P, num_groups, num_nodes, num_gpus, X, _ptr(loads_out),
+            _ptr(out.phy2log), _ptr(out.phyrank), _ptr(out.logcnt), _ptr(out.log2phy),
+            _ptr(status), _stream(dev)), "eplb_rebalance_window")
     return out
 
 

@@ -113,10 +113,8 @@ eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, i
   return launch_window(steps, S, C, W, s_first, snaps, stream);
 }
 
-eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P, int32_t G,
-                           int32_t N, int32_t gpus, int32_t X, int32_t *phy2log,
-                           int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
-                           cudaStream_t stream) {
+static eplb_status rebalance_shape(int64_t R, int32_t E, int32_t P, int32_t G, int32_t N,
+                                   int32_t gpus, int32_t X, RebalanceShape *out) {
   if (R < 0 || E < 1 || P < 1 || G < 1 || N < 1 || gpus < 1 || X < 1) return EPLB_ERR_SHAPE;
   if (P < E) return EPLB_ERR_SHAPE;
   if (E > 1024 || P > 2048 || R > 0x7fffffffLL) return EPLB_ERR_LIMIT;
@@ -162,9 +160,35 @@ eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P
     }
     sh.lam_fixed = static_cast<uint64_t>(lam);
   }
-  if (R == 0) return EPLB_OK;
+  *out = sh;
+  return EPLB_OK;
+}
+
+eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P, int32_t G,
+                           int32_t N, int32_t gpus, int32_t X, int32_t *phy2log,
+                           int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
+                           cudaStream_t stream) {
+  RebalanceShape sh;
+  const eplb_status st = rebalance_shape(R, E, P, G, N, gpus, X, &sh);
+  if (st != EPLB_OK || R == 0) return st;
   if (!loads || !phy2log || !phyrank || !logcnt || !log2phy) return EPLB_ERR_NULL;
-  return launch_rebalance(loads, R, sh, phy2log, phyrank, logcnt, log2phy, status, stream);
+  // the kernel only reads the load array when no ring slot is cleared
+  return launch_rebalance(const_cast<int64_t *>(loads), 1, -1, nullptr, R, sh, phy2log, phyrank,
+                          logcnt, log2phy, status, stream);
+}
+
+eplb_status eplb_rebalance_window(int64_t *ring, int64_t W, int64_t zero_slot, int64_t R,
+                                  int32_t E, int32_t P, int32_t G, int32_t N, int32_t gpus,
+                                  int32_t X, int64_t *loads_out, int32_t *phy2log,
+                                  int32_t *phyrank, int32_t *logcnt, int32_t *log2phy,
+                                  int32_t *status, cudaStream_t stream) {
+  if (W < 1 || zero_slot < -1 || zero_slot >= W) return EPLB_ERR_SHAPE;
+  RebalanceShape sh;
+  const eplb_status st = rebalance_shape(R, E, P, G, N, gpus, X, &sh);
+  if (st != EPLB_OK || R == 0) return st;
+  if (!ring || !phy2log || !phyrank || !logcnt || !log2phy) return EPLB_ERR_NULL;
+  return launch_rebalance(ring, W, zero_slot, loads_out, R, sh, phy2log, phyrank, logcnt, log2phy,
+                          status, stream);
 }
 
 eplb_status eplb_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,

@@ -36,9 +36,12 @@ struct RebalanceShape {
   uint64_t lam_fixed;            // lcm(1..cmax) when <= 2^62, else 0
 };
 
-eplb_status launch_rebalance(const int64_t *loads, int64_t R, const RebalanceShape &sh,
-                             int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
-                             int32_t *log2phy, int32_t *status, cudaStream_t stream);
+// Rows' loads are sums of ring_w ring rows of [R, E] (ring_w = 1: a plain
+// load array); zero_slot >= 0 clears that ring row after reading it.
+eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, int64_t *loads_out,
+                             int64_t R, const RebalanceShape &sh, int32_t *phy2log,
+                             int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
+                             cudaStream_t stream);
 
 // Redirect; with counts != nullptr the same pass also adds the load histogram.
 eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,

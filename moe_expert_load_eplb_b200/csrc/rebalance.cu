@@ -64,7 +64,12 @@ constexpr uint64_t kIdxMask = (uint64_t(1) << kIdxBits) - 1;
 typedef unsigned __int128 u128;
 
 struct RbArgs {
-  const int64_t *loads;
+  // A row's loads are the sum of W ring rows: loads[r, e] = sum_w ring[w, r, e]
+  // (W = 1 for a plain load array).  zero_slot >= 0 clears that ring row's
+  // part of each row after it was read; loads_out (nullable) gets the sums.
+  int64_t *ring;
+  int64_t ring_w, ring_stride, zero_slot;
+  int64_t *loads_out;
   int32_t *phy2log, *phyrank, *logcnt, *log2phy, *status;
   RebalanceShape s;
   uint32_t x_magic;
@@ -260,10 +265,11 @@ __device__ void bitonic_desc(K *key, int npad, int nseg) {
 // sorted order: for m <= 32 a segment is the next power of two >= m lanes
 // with one position each; for larger m a segment is a whole warp and lane l
 // holds positions l*PL .. l*PL+PL-1.  Per item: position 0 (the lightest,
-// lowest index on ties) is broadcast, every lane compares its keys with the
-// pack's new key, one ballot + popc gives the insertion point p among the
-// remaining positions, and position i takes the key of position i+1 (i < p),
-// the new key (i == p) or keeps its own (i > p).  Counts move with keys.
+// lowest index on ties) is broadcast, every position compares its key and
+// its right neighbour's with the pack's new key, and takes the neighbour's
+// key, the new key or its own -- one shuffle pair and a few selects per item
+// (a ballot + popc for the insertion point measured 45 cycles on the chain).
+// Counts move with keys.
 template <typename K, int PL>
 __device__ void pack_seg(const K *skey_base, int stride, int nseg, int n, int m, int cap,
                          int32_t *ipack, int32_t *irank, int out_stride) {
@@ -300,19 +306,22 @@ __device__ void pack_seg(const K *skey_base, int stride, int nseg, int n, int m,
       const K up = shfl_down_k(key[0], 1, ms);  // position (li+1)*PL of the next lane
       const int upc = __shfl_down_sync(0xffffffffu, cnt[0], 1, ms);
       const K nk = bc + 1 < cap ? best + (c & ~imask) : kmax;
-      int p = 0;
+      // lt(q) = position q >= 1 holds a key below the new one; the lt
+      // positions are a prefix 1..p.  Position q takes position q+1's key
+      // when lt(q+1), the new key when lt(q) or q == 0 (and not lt(q+1)),
+      // else keeps its own: no ballot needed, each lane sees q and q+1.
+      bool ltk[PL];
+#pragma unroll
+      for (int r = 0; r < PL; ++r) ltk[r] = (li * PL + r) >= 1 && key[r] < nk;
+      const bool lt_up = li + 1 < ms && up < nk;
 #pragma unroll
       for (int r = 0; r < PL; ++r) {
-        const bool lt = (li * PL + r) >= 1 && key[r] < nk;
-        p += __popc(__ballot_sync(0xffffffffu, lt) & segmask);
-      }
-#pragma unroll
-      for (int r = 0; r < PL; ++r) {
-        const int pos = li * PL + r;
+        const bool next_lt = r + 1 < PL ? ltk[r + 1 < PL ? r + 1 : r] : lt_up;
         const K right = r + 1 < PL ? key[r + 1 < PL ? r + 1 : r] : up;
         const int rightc = r + 1 < PL ? cnt[r + 1 < PL ? r + 1 : r] : upc;
-        key[r] = pos < p ? right : (pos == p ? nk : key[r]);
-        cnt[r] = pos < p ? rightc : (pos == p ? bc + 1 : cnt[r]);
+        const bool here = ltk[r] || (li * PL + r) == 0;
+        key[r] = next_lt ? right : (here ? nk : key[r]);
+        cnt[r] = next_lt ? rightc : (here ? bc + 1 : cnt[r]);
       }
       if (li == 0 && active) {
         const int item = static_cast<int>(imask - (c & imask));
@@ -592,11 +601,16 @@ __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
     flags[1] = 0;
   }
 
-  // ---- load the row; loads must lie in [0, 2^40) -------------------------
+  // ---- load the row (the window sum over the ring); loads in [0, 2^40) --
   bool bad = false;
   for (int e = tid; e < s.E; e += nthr()) {
-    const int64_t x = __ldg(a.loads + row * s.E + e);
+    const int64_t at = row * s.E + e;
+    int64_t x = 0;
+#pragma unroll 4
+    for (int64_t k = 0; k < a.ring_w; ++k) x += a.ring[k * a.ring_stride + at];
     w[e] = x;
+    if (a.loads_out) a.loads_out[at] = x;
+    if (a.zero_slot >= 0) a.ring[a.zero_slot * a.ring_stride + at] = 0;
     bad |= (x < 0) | (x >= kLoadLimit);
   }
   if (__syncthreads_or(bad)) {
@@ -803,9 +817,10 @@ __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
 
 }  // namespace
 
-eplb_status launch_rebalance(const int64_t *loads, int64_t R, const RebalanceShape &sh,
-                             int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
-                             int32_t *log2phy, int32_t *status, cudaStream_t stream) {
+eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, int64_t *loads_out,
+                             int64_t R, const RebalanceShape &sh, int32_t *phy2log,
+                             int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
+                             cudaStream_t stream) {
   DeviceInfo di;
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
   const Layout lay(sh);
@@ -815,7 +830,11 @@ eplb_status launch_rebalance(const int64_t *loads, int64_t R, const RebalanceSha
                                          static_cast<int>(lay.total));
   if (err != cudaSuccess) return cuda_fail(err);
   RbArgs a;
-  a.loads = loads;
+  a.ring = ring;
+  a.ring_w = ring_w;
+  a.ring_stride = R * sh.E;
+  a.zero_slot = zero_slot;
+  a.loads_out = loads_out;
   a.phy2log = phy2log;
   a.phyrank = phyrank;
   a.logcnt = logcnt;

@@ -6,10 +6,11 @@ round-trip:
 serving (default): the plan in force (built from earlier steps' loads, the
   moving-average estimate of page "DualPipe и EPLB", Part 2, section
   "Алгоритм") redirects this step's indices in the same pass that counts
-  them, so the indices cross HBM once:
-    1. count_redirect: indices -> ring row (step % W) and physical indices;
-    2. window_accumulate over the ring (s_first = W - 1): the window sum;
-    3. rebalance: the next plan of every layer.
+  them, so the indices cross HBM once; two launches per step:
+    1. count_redirect: indices -> ring row (step % W, cleared beforehand) and
+       physical indices;
+    2. rebalance_window: the window sum over the ring and the next plan of
+       every layer, clearing the ring row the next step counts into.
 fresh: the plan is rebuilt from this step's counts before redirecting:
     count_loads -> window_accumulate -> rebalance -> redirect.
 
@@ -25,8 +26,8 @@ from typing import Optional, Sequence
 
 import torch
 
-from . import (Plan, count_loads, count_redirect, default_slots, rebalance, redirect,
-               window_accumulate)
+from . import (Plan, count_loads, count_redirect, default_slots, rebalance, rebalance_window,
+               redirect, window_accumulate)
 from .distributed import allreduce_loads
 
 
@@ -65,7 +66,7 @@ class EplbStep:
     @property
     def launches_per_step(self) -> int:
         """Kernels of this library launched per step."""
-        return 3 if self.fused else 4
+        return 2 if self.fused else 4
 
     @property
     def plan(self) -> Plan:
@@ -73,10 +74,14 @@ class EplbStep:
         return self.plans[self.cur]
 
     def fill_history(self, history: torch.Tensor, steps_done: Optional[int] = None):
-        """Load earlier per-step counts into the ring and build the plan in force."""
-        n = history.shape[0]
-        self.ring[:n].copy_(history)
+        """Load earlier per-step counts (at most W - 1 rows kept) into the ring,
+        clear the slot the next step counts into, and build the plan in force."""
+        n = min(history.shape[0], self.W - 1)
+        self.ring.zero_()
+        if n:
+            self.ring[:n].copy_(history[history.shape[0] - n:])
         self.steps_done = n if steps_done is None else steps_done
+        self.ring[self.steps_done % self.W].zero_()
         self._plan_from_ring(self.plans[self.cur])
         self.primed = True
 
@@ -92,7 +97,8 @@ class EplbStep:
         serving order's new plan is ``self.plan`` afterwards.  ``marks``: six
         CUDA events recorded on the current stream around the stages
         count | allreduce | window | rebalance | redirect (the serving order
-        records its fused pass under count and an empty redirect stage).
+        records its fused count+redirect under count, its fused
+        window+rebalance under rebalance, and empty window / redirect stages).
         """
         if self.fused and not self.primed:
             raise RuntimeError("serving order needs a plan in force: call fill_history() first")
@@ -101,19 +107,28 @@ class EplbStep:
         used = self.plans[self.cur]
         rec(0)
         if self.fused:
+            # the ring row was cleared by the previous step's rebalance_window
             count_redirect(idx, self.E, used.log2phy, used.logcnt, self.token_offset, counts=row,
-                           out=self.out, bad=self.bad, status=self.status)
+                           accumulate=True, out=self.out, bad=self.bad, status=self.status)
         else:
             count_loads(idx, self.E, counts=row, bad=self.bad, status=self.status)
         rec(1)
         if self.group is not None:
             allreduce_loads(row, self.group)
         rec(2)
-        window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads, status=self.status)
-        rec(3)
-        nxt = self.plans[1 - self.cur] if self.fused else used
-        rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=nxt,
-                  status=self.status)
+        if self.fused:
+            rec(3)
+            nxt = self.plans[1 - self.cur]
+            rebalance_window(self.ring, self.P, self.G, self.N, self.gpus,
+                             zero_slot=(self.steps_done + 1) % self.W, slots=self.X, out=nxt,
+                             loads_out=self.loads, status=self.status)
+        else:
+            window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads,
+                              status=self.status)
+            rec(3)
+            nxt = used
+            rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=nxt,
+                      status=self.status)
         rec(4)
         if not self.fused:
             redirect(idx, nxt.log2phy, nxt.logcnt, self.token_offset, out=self.out, bad=self.bad,

@@ -546,3 +546,41 @@ def test_plan_diff_initial_to_first_plan(c2_idx):
     src, moves = eplb.plan_diff(init, plan.phy2log, c.E, c.gpus)
     ref_src, ref_moves = oracle.plan_diff(_np(init), _np(plan.phy2log), c.E, c.gpus)
     assert np.array_equal(_np(src), ref_src) and np.array_equal(_np(moves), ref_moves)
+
+
+# ------------------------------------------------------- rebalance_window --
+
+@pytest.mark.parametrize("W_,zero", [(16, 3), (1, -1), (4, 0), (7, -1)])
+def test_rebalance_window_matches_window_then_rebalance(W_, zero):
+    c = W.CONFIGS[2]
+    ring = W.histogram_steps(W_, c.L, c.E, c.T * c.K, 7, device=DEV).contiguous()
+    ring_h = _np(ring).copy()
+    loads_out = torch.empty((c.L, c.E), dtype=torch.int64, device=DEV)
+    st = _status()
+    plan = eplb.rebalance_window(ring, c.P, c.G, c.N, c.gpus, zero_slot=zero, loads_out=loads_out,
+                                 status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    sums = oracle.window(ring_h, W_, W_ - 1)[0]
+    assert np.array_equal(_np(loads_out), sums)
+    ref = oracle.rebalance(sums, c.P, c.G, c.N, c.gpus, slots=plan.log2phy.shape[2])
+    _assert_plan_equal(plan, ref)
+    after = _np(ring)
+    for k in range(W_):
+        if k == zero:
+            assert (after[k] == 0).all()
+        else:
+            assert np.array_equal(after[k], ring_h[k])
+
+
+def test_rebalance_window_range_error():
+    ring = torch.full((2, 3, 12), 1 << 39, dtype=torch.int64, device=DEV)  # sums reach 2^40
+    ring[:, 1] = 5
+    st = _status()
+    plan = eplb.rebalance_window(ring, 16, 4, 2, 8, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+    assert (_np(plan.phy2log[0]) == -1).all() and (_np(plan.phy2log[2]) == -1).all()
+    ref = oracle.rebalance(np.full((1, 12), 10, np.int64), 16, 4, 2, 8, slots=plan.log2phy.shape[2])
+    for got, want in zip(plan, ref):
+        assert np.array_equal(_np(got)[1:2], want)
