@@ -354,6 +354,35 @@ def test_redirect_invalid_logcnt_reports_range():
     assert int(st.item()) == 4 and (_np(out) == -1).all()
 
 
+@pytest.mark.parametrize("E,X,K", [(1, 1, 4), (7, 40, 4), (7, 40, 3), (1024, 32, 4), (300, 9, 8),
+                                   (16, 2048, 5), (33, 6, 4)])
+@pytest.mark.parametrize("fused", [False, True])
+def test_redirect_arbitrary_tables(E, X, K, fused):
+    """Any int32 log2phy entries and any logcnt in [1, X]: replicas held in the
+    per-expert descriptor (<= 5, index < 2048) and the rest must all agree."""
+    L, T = 3, 3001
+    rng = np.random.default_rng(E * 31 + X * 7 + K + fused)
+    l2p = rng.integers(-2 ** 31, 2 ** 31, (L, E, X)).astype(np.int32)
+    l2p[:, ::2] = rng.integers(0, 2048, (L, (E + 1) // 2, X))
+    l2p[:, 1::4] = rng.integers(2040, 2056, (L, len(range(1, E, 4)), X))
+    cnt = rng.integers(1, X + 1, (L, E)).astype(np.int32)
+    cnt[:, ::3] = rng.integers(1, min(5, X) + 1, (L, (E + 2) // 3))
+    idx = rng.integers(-3, E + 3, (L, T, K)).astype(np.int32)
+    t0 = 123457
+    l2p_d, cnt_d = torch.from_numpy(l2p).to(DEV), torch.from_numpy(cnt).to(DEV)
+    idx_d = torch.from_numpy(idx).to(DEV)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    st = _status()
+    if fused:
+        counts, out = eplb.count_redirect(idx_d, E, l2p_d, cnt_d, token_offset=t0, bad=bad, status=st)
+        assert np.array_equal(_np(counts), oracle.count_loads(idx, E)[0])
+    else:
+        out = eplb.redirect(idx_d, l2p_d, cnt_d, token_offset=t0, bad=bad, status=st)
+    ref, nbad = oracle.redirect(idx, l2p, cnt, t0)
+    assert np.array_equal(_np(out), ref)
+    assert int(bad.item()) == nbad and int(st.item()) == 0
+
+
 def test_redirect_sharded_equals_whole(c2_idx):
     c = W.CONFIGS[2]
     counts = eplb.count_loads(c2_idx, c.E)
