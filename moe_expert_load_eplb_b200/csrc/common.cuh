@@ -101,6 +101,18 @@ __device__ __forceinline__ void report(int32_t *status, int32_t code) {
 // x*(2^32/d - m)/2^32 < 2x/2^32 < 1), so one conditional subtraction fixes
 // the remainder.  Multiply-high division after Granlund & Montgomery,
 // "Division by invariant integers using multiplication", PLDI 1994.
+// Programmatic dependent launch.  Every kernel of the library is launched
+// with programmatic stream serialisation: at its start it lets the next
+// kernel of the stream be scheduled (pdl_trigger) and then waits until the
+// previous grid of the stream has finished and its memory is visible
+// (pdl_wait) before it touches global memory, so launch latency overlaps
+// the previous kernel's tail while stream order still holds for every read
+// and write.  Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t mod_magic(uint32_t x, uint32_t d, uint32_t m) {
   uint32_t q = __umulhi(x, m);
   uint32_t r = x - q * d;

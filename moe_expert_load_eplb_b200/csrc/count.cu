@@ -43,6 +43,8 @@ struct CountArgs {
 
 __global__ void __launch_bounds__(kThreads) count_loads_kernel(CountArgs a) {
   extern __shared__ __align__(16) uint32_t hist[];  // [E+1][32]; bin E counts bad indices
+  pdl_trigger();
+  pdl_wait();
   const int tid = threadIdx.x;
   const uint32_t lane = tid & 31;
   const uint32_t E = static_cast<uint32_t>(a.E);
@@ -149,8 +151,9 @@ eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer,
   const int64_t waves = std::min(std::max<int64_t>(total / (kChunk * slots), 1), kMaxWaves);
   a.chunks = std::max<int64_t>(1, std::min(waves * slots / L, (per_layer + 4095) / 4096));
   const int64_t grid = L * a.chunks;
-  count_loads_kernel<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(a);
-  err = cudaGetLastError();
+  void *args[] = {&a};
+  err = launch_pdl(reinterpret_cast<const void *>(count_loads_kernel), dim3(static_cast<unsigned>(grid)),
+                   dim3(kThreads), smem, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

@@ -9,6 +9,24 @@
 
 namespace eplb {
 
+// Launches fn with programmatic stream serialisation (see pdl_trigger /
+// pdl_wait in common.cuh); args as for cudaLaunchKernel.
+inline cudaError_t launch_pdl(const void *fn, dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, void **args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+
 struct DeviceInfo {
   int sms = 0;
   int max_smem_optin = 0;

@@ -280,7 +280,6 @@ __device__ void pack_seg(const K *skey_base, int stride, int nseg, int n, int m,
   if (PL > 1) ms = 32;
   const int lane = threadIdx.x & 31;
   const int li = lane & (ms - 1);            // lane within the segment
-  const unsigned segmask = ms == 32 ? 0xffffffffu : ((1u << ms) - 1u) << (lane & ~(ms - 1));
   const int slot = static_cast<int>(threadIdx.x) / ms;
   const int slots = nthr() / ms;
   const int warp_first_slot = (static_cast<int>(threadIdx.x) & ~31) / ms;
@@ -571,6 +570,8 @@ __device__ void step3(const RbArgs &a, unsigned char *smem, const Layout &lay) {
 
 __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
+  pdl_trigger();
+  pdl_wait();
   __shared__ int flags[2];  // [0] 128-bit keys needed, [1] exact ratio not representable
   const RebalanceShape &s = a.s;
   const Layout lay(s);
@@ -845,8 +846,9 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
   a.table_vec4 = ((static_cast<int64_t>(sh.E) * sh.X) % 4 == 0) &&
                  (reinterpret_cast<uintptr_t>(log2phy) % 16 == 0);
   const int threads = R <= 2 * static_cast<int64_t>(di.sms) ? kFewRowThreads : kManyRowThreads;
-  rebalance_kernel<<<static_cast<unsigned>(R), threads, lay.total, stream>>>(a);
-  err = cudaGetLastError();
+  void *args[] = {&a};
+  err = launch_pdl(reinterpret_cast<const void *>(rebalance_kernel), dim3(static_cast<unsigned>(R)),
+                   dim3(threads), lay.total, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

@@ -153,6 +153,8 @@ __device__ __forceinline__ uint32_t selector(uint32_t u) {
 template <bool kVecToken, bool kCount>
 __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
+  pdl_trigger();
+  pdl_wait();
   const int E1 = a.E + 1;
   uint32_t *hist = reinterpret_cast<uint32_t *>(smem);  // [E+1][32], kCount only
   unsigned char *region = smem + (kCount ? E1 * 32 * sizeof(uint32_t) : 0);
@@ -452,7 +454,7 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
   a.chunks = chunks;
   const int64_t grid = L * chunks;
   void *args[] = {&a};
-  err = cudaLaunchKernel(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), args, smem, stream);
+  err = launch_pdl(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

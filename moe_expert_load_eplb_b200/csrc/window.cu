@@ -25,6 +25,8 @@ constexpr int kU = 8;  // rows per thread per block
 __global__ void window_kernel(const int64_t *__restrict__ steps, int64_t S, int64_t C, int64_t W,
                               int64_t s_first, int64_t *__restrict__ snaps, int cw, int rg) {
   extern __shared__ int64_t part[];  // [rg][cw]
+  pdl_trigger();
+  pdl_wait();
   const int tid = threadIdx.x;
   const int col = tid % cw;
   const int g = tid / cw;
@@ -98,9 +100,10 @@ eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W,
   const int rg = static_cast<int>(std::min<int64_t>(std::max(1, 256 / cw), max_rg));
   const int64_t strips = (C + cw - 1) / cw;
   const size_t smem = static_cast<size_t>(rg) * cw * sizeof(int64_t);
-  window_kernel<<<static_cast<unsigned>(strips), cw * rg, smem, stream>>>(steps, S, C, W, s_first,
-                                                                          snaps, cw, rg);
-  const cudaError_t err = cudaGetLastError();
+  void *args[] = {&steps, &S, &C, &W, &s_first, &snaps, const_cast<int *>(&cw), const_cast<int *>(&rg)};
+  const cudaError_t err = launch_pdl(reinterpret_cast<const void *>(window_kernel),
+                                     dim3(static_cast<unsigned>(strips)), dim3(cw * rg), smem, stream,
+                                     args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 
