@@ -101,6 +101,17 @@ __device__ __forceinline__ void report(int32_t *status, int32_t code) {
 // x*(2^32/d - m)/2^32 < 2x/2^32 < 1), so one conditional subtraction fixes
 // the remainder.  Multiply-high division after Granlund & Montgomery,
 // "Division by invariant integers using multiplication", PLDI 1994.
+// Shared-memory access by 32-bit shared-window address: one multiply-add
+// per address, no generic-pointer arithmetic.
+__device__ __forceinline__ void red_shared_inc(uint32_t addr) {
+  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr));
+}
+__device__ __forceinline__ int32_t ld_shared_s16(uint32_t addr) {
+  int32_t v;
+  asm volatile("ld.shared.s16 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 // Programmatic dependent launch.  Every kernel of the library is launched
 // with programmatic stream serialisation: at its start it lets the next
 // kernel of the stream be scheduled (pdl_trigger) and then waits until the

@@ -277,9 +277,17 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
       nbad += ee == E ? 1u : 0u;
     return ee;
   };
-  // fast path: trow = tab + (token mod M)
-  auto map_fast = [&](int32_t e, const int16_t *trow) -> int32_t {
-    return trow[clamp_count(e) * M];
+  // fast path: ctx = shared address of tab[0][token mod M]
+  const uint32_t hist_addr = smem_u32(hist) + 4u * lane;
+  const uint32_t tab_addr = smem_u32(tab);
+  const uint32_t row_bytes = 2u * M;
+  auto map_fast = [&](int32_t e, uint32_t trow) -> int32_t {
+    const uint32_t ee = min(static_cast<uint32_t>(e), E);
+    if (kCount)
+      red_shared_inc(hist_addr + ee * 128u);
+    else
+      nbad += ee == E ? 1u : 0u;
+    return ld_shared_s16(trow + ee * row_bytes);
   };
   // descriptor path: ctx = {selector(token), token}
   auto map_desc = [&](int32_t e, uint2 ctx) -> int32_t {
@@ -295,7 +303,7 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
     const uint32_t r = mod_magic(ctx.y, c, static_cast<uint32_t>(d >> 5));
     return __ldg(l2p_layer + ee * static_cast<uint32_t>(a.X) + r);
   };
-  auto ctx_fast = [&](uint32_t tok) -> const int16_t * { return tab + mod_magic(tok, M, a.m_magic); };
+  auto ctx_fast = [&](uint32_t tok) -> uint32_t { return tab_addr + 2u * mod_magic(tok, M, a.m_magic); };
   auto ctx_desc = [&](uint32_t tok) -> uint2 { return make_uint2(selector(tok), tok); };
 
   auto stream = [&](auto ctx_of, auto map1) {
@@ -309,33 +317,35 @@ __global__ void __launch_bounds__(kThreads) redirect_kernel(RedirectArgs a) {
       const uint32_t tok = a.t0 + div_magic(static_cast<uint32_t>(p - lbase), a.K, a.k_magic);
       a.out[p] = map1(__ldg(a.idx + p), ctx_of(tok));
     }
-    while (i < nvec) {
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int v = i + u * kThreads;
-        if (v < nvec) {
-          const uint32_t pos = pos0 + 4u * static_cast<uint32_t>(v);
-          int4 y;
-          if (kVecToken) {
-            const auto ctx = ctx_of(a.t0 + div_magic(pos, a.K, a.k_magic));
-            y.x = map1(x[u].x, ctx);
-            y.y = map1(x[u].y, ctx);
-            y.z = map1(x[u].z, ctx);
-            y.w = map1(x[u].w, ctx);
-          } else {
-            y.x = map1(x[u].x, ctx_of(a.t0 + div_magic(pos, a.K, a.k_magic)));
-            y.y = map1(x[u].y, ctx_of(a.t0 + div_magic(pos + 1, a.K, a.k_magic)));
-            y.z = map1(x[u].z, ctx_of(a.t0 + div_magic(pos + 2, a.K, a.k_magic)));
-            y.w = map1(x[u].w, ctx_of(a.t0 + div_magic(pos + 3, a.K, a.k_magic)));
-          }
-          __stcs(pout + v, y);
-        }
+    auto vector = [&](int v, const int4 &xv) {
+      const uint32_t pos = pos0 + 4u * static_cast<uint32_t>(v);
+      int4 y;
+      if (kVecToken) {
+        const auto ctx = ctx_of(a.t0 + div_magic(pos, a.K, a.k_magic));
+        y.x = map1(xv.x, ctx);
+        y.y = map1(xv.y, ctx);
+        y.z = map1(xv.z, ctx);
+        y.w = map1(xv.w, ctx);
+      } else {
+        y.x = map1(xv.x, ctx_of(a.t0 + div_magic(pos, a.K, a.k_magic)));
+        y.y = map1(xv.y, ctx_of(a.t0 + div_magic(pos + 1, a.K, a.k_magic)));
+        y.z = map1(xv.z, ctx_of(a.t0 + div_magic(pos + 2, a.K, a.k_magic)));
+        y.w = map1(xv.w, ctx_of(a.t0 + div_magic(pos + 3, a.K, a.k_magic)));
       }
+      __stcs(pout + v, y);
+    };
+    // whole batches without per-vector range checks, then the guarded rest
+    while (i + (kU - 1) * kThreads < nvec) {
+#pragma unroll
+      for (int u = 0; u < kU; ++u) vector(i + u * kThreads, x[u]);
       i += kThreads * kU;
 #pragma unroll
       for (int u = 0; u < kU; ++u)
         x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
     }
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (i + u * kThreads < nvec) vector(i + u * kThreads, x[u]);
   };
   if (fast)
     stream(ctx_fast, map_fast);
