@@ -603,16 +603,31 @@ __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
   }
 
   // ---- load the row (the window sum over the ring); loads in [0, 2^40) --
+  // two threads per expert, each summing half of the ring rows with all its
+  // loads in flight
   bool bad = false;
-  for (int e = tid; e < s.E; e += nthr()) {
-    const int64_t at = row * s.E + e;
-    int64_t x = 0;
-#pragma unroll 4
-    for (int64_t k = 0; k < a.ring_w; ++k) x += a.ring[k * a.ring_stride + at];
-    w[e] = x;
-    if (a.loads_out) a.loads_out[at] = x;
-    if (a.zero_slot >= 0) a.ring[a.zero_slot * a.ring_stride + at] = 0;
-    bad |= (x < 0) | (x >= kLoadLimit);
+  {
+    const int lane = tid & 31;
+    const int64_t half = (a.ring_w + 1) >> 1;
+    for (int t = tid; t - lane < 2 * s.E; t += nthr()) {  // warp-uniform for the shuffle
+      const bool live = t < 2 * s.E;
+      const int e = t >> 1;
+      const int64_t at = row * s.E + e;
+      const int64_t k0 = (t & 1) * half;
+      const int64_t k1 = min(a.ring_w, k0 + half);
+      int64_t x = 0;
+      if (live) {
+#pragma unroll 8
+        for (int64_t k = k0; k < k1; ++k) x += a.ring[k * a.ring_stride + at];
+      }
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      if (live && !(t & 1)) {
+        w[e] = x;
+        if (a.loads_out) a.loads_out[at] = x;
+        if (a.zero_slot >= 0) a.ring[a.zero_slot * a.ring_stride + at] = 0;
+        bad |= (x < 0) | (x >= kLoadLimit);
+      }
+    }
   }
   if (__syncthreads_or(bad)) {
     write_error_row(a, row);
@@ -627,11 +642,13 @@ __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
       grank[g] = 0;
     }
   } else {
-    for (int g = tid; g < s.G; g += nthr()) {
+    for (int g = tid >> 5; g < s.G; g += nwarps()) {  // one warp per group
+      const int lane = tid & 31;
       uint64_t sum = 0;
-#pragma unroll 8
-      for (int i = 0; i < s.gs; ++i) sum += static_cast<uint64_t>(w[g * s.gs + i]);
-      gkey[g] = (sum << kIdxBits) | (kIdxMask - g);
+      for (int i = lane; i < s.gs; i += 32) sum += static_cast<uint64_t>(w[g * s.gs + i]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (lane == 0) gkey[g] = (sum << kIdxBits) | (kIdxMask - g);
     }
     __syncthreads();
     const uint64_t *gs_keys = gsorted;
