@@ -144,9 +144,17 @@ class ClockSampler:
 # --------------------------------------------------------------- profiles --
 
 def _kernel_sha(name: str) -> str:
-    path = os.path.join(ROOT, "moe_expert_load_eplb_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256 (first 16 hex digits) of a kernel's source; several files
+    separated by '+' are hashed in that order."""
+    h = hashlib.sha256()
+    for part in name.split("+"):
+        with open(os.path.join(ROOT, "moe_expert_load_eplb_b200", "csrc", part), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# the serving-step kernel's code: its file and the two headers it inlines
+SERVE_SOURCES = "serve.cu+redirect_chunk.cuh+rebalance_row.cuh"
 
 
 def _traffic(kernel_file: str, profile: str, scale: float):
@@ -246,9 +254,9 @@ def run_ours(args, rank: int, world: int, group):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     hbm_peak, peak_kind = _peaks()
 
-    def make(fused):
+    def make(fused, single=True):
         st = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=WINDOW, device=dev,
-                      token_offset=rank * c.T, group=group, fused=fused)
+                      token_offset=rank * c.T, group=group, fused=fused, single_launch=single)
         st.fill_history(hist)
         return st
 
@@ -270,7 +278,7 @@ def run_ours(args, rank: int, world: int, group):
         return {"fresh_only": True, "steps": args.steps, "ms_per_step": round(f_total / args.steps, 5),
                 "stages": _stage_report(f_stage, False, fresh.X, world, hbm_peak), "clocks": clocks}
 
-    # ---- the timed step: serving order (count+redirect fused, then plan) ----
+    # ---- the timed step: serving order (count+redirect, [all-reduce], plan) --
     step = make(True)
     for i in range(args.warmup):
         flush.fill_(i & 0xff)
@@ -279,38 +287,52 @@ def run_ours(args, rank: int, world: int, group):
     K = args.steps
     total_ms, _, clocks = _timed_steps(step, idx, flush, K, group, dev)
     check(step, "timed steps")
+    ms_per_step = total_ms / K
+    value = c.L * K / (total_ms / 1e3)
     # per-stage breakdown: a separate pass with events between the stages
     _, per_stage, _ = _timed_steps(step, idx, flush, max(3, min(K, 500)), group, dev, staged=True)
     check(step, "staged steps")
-    ms_per_step = total_ms / K
-    value = c.L * K / (total_ms / 1e3)
     stages = _stage_report(per_stage, True, step.X, world, hbm_peak)
-
-    dominant = max(("count", "rebalance"), key=lambda n: stages[n]["ms"])
-    if dominant == "count":
-        roof = {"kernel": "count_redirect", "bound": "hbm", "achieved": stages["count"]["gbs"],
-                "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                "frac": stages["count"]["frac_hbm"],
-                "traffic": _traffic("redirect.cu", "count_redirect_dsv3_prefill.md", 1.0)}
-    elif dominant == "window":
-        roof = {"kernel": "window", "bound": "hbm", "achieved": stages["window"]["gbs"],
-                "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-                "frac": stages["window"]["frac_hbm"],
-                "traffic": _traffic("window.cu", "window_dsv3_prefill.md", 1.0)}
-    else:
-        roof = {"kernel": "rebalance", "bound": "alu", "achieved": None, "peak": None,
-                "unit": None, "frac": None, "traffic": None}
+    stages["count"]["traffic"] = _traffic("redirect.cu+redirect_chunk.cuh",
+                                          "count_redirect_dsv3_prefill.md", 1.0)
+    roof = {"kernel": "count_redirect", "bound": "hbm", "achieved": stages["count"]["gbs"],
+            "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": stages["count"]["frac_hbm"], "traffic": stages["count"]["traffic"]}
+    order = ("serving: count+redirect with the plan in force (fused, one pass over the indices) "
+             + ("-> all-reduce of the counts " if world > 1 else "")
+             + "-> window sum + rebalance (fused) -> next plan")
 
     out = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
            "data": "synthetic (seeded group-limited routing, log-normal popularity)",
-           "config": dict(_config(world), step_order="serving: count+redirect with the plan in "
-                          "force (fused, one pass over the indices) -> window sum + rebalance "
-                          "(fused) -> next plan"),
+           "config": dict(_config(world), step_order=order),
            "gpu_launches": step.launches_per_step * K,
            "tokens_per_s": round(world * c.T * K / (total_ms / 1e3), 1),
            "stages": stages, "roofline": roof, "clocks": clocks}
+
+    # ---- the same step in one launch (serve_step), one GPU only -------------
+    if world == 1 and not args.no_fresh:
+        one = make(True, single=True)
+        for i in range(max(3, args.warmup // 4)):
+            flush.fill_(i & 0xff)
+            one(idx)
+        check(one, "one-launch warm-up")
+        Ko = max(3, min(K, 500))
+        o_total, _, _ = _timed_steps(one, idx, flush, Ko, group, dev)
+        check(one, "one-launch steps")
+        n_idx = c.L * c.T * c.K
+        # indices in and out, count atomics, ring rows summed, cleared slot,
+        # window sums and the next plan written
+        algo = (8.0 * n_idx + 8.0 * c.L * c.E + 8.0 * WINDOW * c.L * c.E + 16.0 * c.L * c.E
+                + 4.0 * c.L * (2 * c.P + c.E + c.E * one.X))
+        o_ms = o_total / Ko
+        out["one_launch_order"] = {
+            "steps": Ko, "ms_per_step": round(o_ms, 5), "value": round(c.L * Ko / (o_total / 1e3), 1),
+            "kernel": "serve_kernel (S1+S5 per chunk, then S2+S3/S4 per layer once counted)",
+            "algo_bytes": algo, "gbs": round(algo / (o_ms / 1e3) / 1e9, 1),
+            "traffic": _traffic(SERVE_SOURCES, "serve_step_dsv3_prefill.md", 1.0)}
+        del one
 
     # ---- the same four stages in the fresh-plan order, for comparison -----
     if args.no_fresh:

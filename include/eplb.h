@@ -190,6 +190,41 @@ eplb_status eplb_count_redirect(const int32_t *idx, int64_t L, int64_t T, int32_
                                 unsigned long long *bad, int32_t *status, cudaStream_t stream);
 
 /*
+ * The serving step in one launch (S1 + S5, then S2 + S3/S4 per layer).  The
+ * pages plan from a moving average of recent loads ([EPLB] "Алгоритм") and
+ * route with the plan in force ([LPLB] usage example); this call does both
+ * for one batch:
+ *   1. exactly eplb_count_redirect(idx, ..., counts = ring + slot * L * E,
+ *      accumulate = 1, log2phy, X, logcnt, t0, out, bad): the batch is
+ *      counted into ring slot `slot` and redirected with the plan in force;
+ *   2. then, for every layer l, exactly eplb_rebalance_window on row l of the
+ *      ring [W, L, E] (the window sum over all W slots, this batch included)
+ *      into next_phy2log / next_phyrank / next_logcnt / next_log2phy, writing
+ *      loads_out (nullable) and clearing ring row zero_slot (-1: none) after
+ *      the sum was read.
+ * A layer's plan is built by the CTA that finishes the layer's last chunk,
+ * while other layers are still being redirected.
+ * ring         device int64 [W, L, E]; ring[slot] must hold the counts that
+ *              should be added to (normally zero: cleared by the previous
+ *              step's zero_slot).
+ * next_*       the next plan, same shapes as eplb_rebalance's outputs with X
+ *              slots; must not be the plan in force (log2phy / logcnt).
+ * layer_done   device uint32 [L], caller-owned, all zero before the call; the
+ *              call leaves it all zero again.  One array per stream: two
+ *              calls in flight at once must not share it.
+ * Limits and errors: those of eplb_count_redirect and of eplb_rebalance with
+ *              R = L; 0 <= slot < W; -1 <= zero_slot < W.  T may be 0 (the
+ *              plan is then rebuilt from the ring alone).
+ */
+eplb_status eplb_serve_step(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                            const int32_t *log2phy, int32_t X, const int32_t *logcnt, int64_t t0,
+                            int32_t *out, unsigned long long *bad, int64_t *ring, int64_t W,
+                            int64_t slot, int64_t zero_slot, int32_t P, int32_t G, int32_t N,
+                            int32_t gpus, int64_t *loads_out, int32_t *next_phy2log,
+                            int32_t *next_phyrank, int32_t *next_logcnt, int32_t *next_log2phy,
+                            uint32_t *layer_done, int32_t *status, cudaStream_t stream);
+
+/*
  * Plan quality ([EPLB] box "От переводчика: что на рисунке": per-GPU load of
  * the worked example, 86.5 .. 156, mean 129; exercise 2 of "что сделать
  * руками": compare max / mean between policies).  Per row r:

@@ -25,7 +25,7 @@ import torch
 
 __all__ = [
     "EplbError", "Plan", "count_loads", "window_accumulate", "rebalance", "redirect", "count_redirect",
-    "plan_stats", "fold_loads", "initial_map", "plan_diff", "rebalance_window",
+    "plan_stats", "fold_loads", "initial_map", "plan_diff", "rebalance_window", "serve_step",
     "default_slots", "lib_path", "load_library", "STATUS",
 ]
 
@@ -87,6 +87,8 @@ def load_library():
         "eplb_fold_loads": ([p, p, i64, i32, i32, p, p, p], i32),
         "eplb_initial_map": ([i64, i32, i32, p, p, p], i32),
         "eplb_plan_diff": ([p, p, i64, i32, i32, i32, p, p, p, p], i32),
+        "eplb_serve_step": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, i64, i64, i64,
+                             i32, i32, i32, i32, p, p, p, p, p, p, p, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -291,6 +293,56 @@ def count_redirect(idx: torch.Tensor, num_experts: int, log2phy: torch.Tensor, l
             _ptr(logcnt), int(token_offset), _ptr(out), _ptr(bad), _ptr(status),
             _stream(idx.device)), "eplb_count_redirect")
     return counts, out
+
+
+def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, next_plan: Plan,
+               layer_done: torch.Tensor, num_groups: int, num_nodes: int, num_gpus: int,
+               zero_slot: int = -1, token_offset: int = 0, out: Optional[torch.Tensor] = None,
+               loads_out: Optional[torch.Tensor] = None, bad: Optional[torch.Tensor] = None,
+               status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The serving step in one launch: count idx into ring[slot] and redirect it
+    with ``plan`` (the plan in force), then rebuild every layer's plan from the
+    window sum over the ring into ``next_plan`` (clearing ring[zero_slot]).
+    ``layer_done``: uint32 [L] work array, zero before and after.  Returns out."""
+    _cuda(idx, torch.int32, "idx")
+    _cuda(ring, torch.int64, "ring")
+    if idx.dim() != 3 or ring.dim() != 3:
+        raise ValueError("idx [L, T, K] and ring [W, L, E] expected")
+    L, T, K = idx.shape
+    Wr, Lr, E = ring.shape
+    if Lr != L:
+        raise ValueError("ring and idx disagree on L")
+    for name, pl in (("plan", plan), ("next_plan", next_plan)):
+        _cuda(pl.log2phy, torch.int32, f"{name}.log2phy")
+        _cuda(pl.logcnt, torch.int32, f"{name}.logcnt")
+        _cuda(pl.phy2log, torch.int32, f"{name}.phy2log")
+        _cuda(pl.phyrank, torch.int32, f"{name}.phyrank")
+    P = next_plan.phy2log.shape[1]
+    X = plan.log2phy.shape[2]
+    if (tuple(plan.log2phy.shape) != (L, E, X) or tuple(next_plan.log2phy.shape) != (L, E, X)
+            or tuple(plan.logcnt.shape) != (L, E) or tuple(next_plan.logcnt.shape) != (L, E)
+            or tuple(next_plan.phy2log.shape) != (L, P) or tuple(next_plan.phyrank.shape) != (L, P)):
+        raise ValueError("plan shapes do not match idx / ring")
+    if not isinstance(layer_done, torch.Tensor) or not layer_done.is_cuda or \
+            layer_done.dtype not in (torch.int32, torch.uint32) or layer_done.numel() != L:
+        raise TypeError("layer_done must be a CUDA int32/uint32 tensor of L elements")
+    if out is None:
+        out = torch.empty_like(idx)
+    _cuda(out, torch.int32, "out")
+    if out.shape != idx.shape:
+        raise ValueError("out must match idx")
+    if loads_out is not None:
+        _cuda(loads_out, torch.int64, "loads_out")
+        if loads_out.numel() != L * E:
+            raise ValueError("loads_out must be [L, E]")
+    with torch.cuda.device(idx.device):
+        _check(load_library().eplb_serve_step(
+            _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
+            _ptr(out), _ptr(bad), _ptr(ring), Wr, slot, zero_slot, P, num_groups, num_nodes,
+            num_gpus, _ptr(loads_out), _ptr(next_plan.phy2log), _ptr(next_plan.phyrank),
+            _ptr(next_plan.logcnt), _ptr(next_plan.log2phy), _ptr(layer_done), _ptr(status),
+            _stream(idx.device)), "eplb_serve_step")
+    return out
 
 
 def plan_stats(loads: torch.Tensor, phy2log: torch.Tensor, logcnt: torch.Tensor, num_gpus: int,

@@ -80,7 +80,7 @@ const char *eplb_status_string(int32_t status) {
 
 const char *eplb_last_cuda_error(void) { return g_last_error; }
 
-int32_t eplb_abi_version(void) { return (1 << 16) | 0; }
+int32_t eplb_abi_version(void) { return (1 << 16) | 1; }
 
 eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
                              int64_t *counts, int32_t accumulate, unsigned long long *bad,
@@ -224,6 +224,32 @@ eplb_status eplb_count_redirect(const int32_t *idx, int64_t L, int64_t T, int32_
   if (T == 0) return EPLB_OK;
   return launch_redirect(idx, L, T, K, E, log2phy, X, logcnt, t0, out, counts, bad, status,
                          stream);
+}
+
+eplb_status eplb_serve_step(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                            const int32_t *log2phy, int32_t X, const int32_t *logcnt, int64_t t0,
+                            int32_t *out, unsigned long long *bad, int64_t *ring, int64_t W,
+                            int64_t slot, int64_t zero_slot, int32_t P, int32_t G, int32_t N,
+                            int32_t gpus, int64_t *loads_out, int32_t *next_phy2log,
+                            int32_t *next_phyrank, int32_t *next_logcnt, int32_t *next_log2phy,
+                            uint32_t *layer_done, int32_t *status, cudaStream_t stream) {
+  if (L < 0 || T < 0 || K < 1 || E < 1 || X < 1 || t0 < 0) return EPLB_ERR_SHAPE;
+  if (W < 1 || slot < 0 || slot >= W || zero_slot < -1 || zero_slot >= W) return EPLB_ERR_SHAPE;
+  if (E > 1024 || static_cast<int64_t>(E) * X > 32768) return EPLB_ERR_LIMIT;
+  if (T >= (int64_t(1) << 31) / K || t0 + T >= (int64_t(1) << 31)) return EPLB_ERR_LIMIT;
+  RebalanceShape sh;
+  const eplb_status st = rebalance_shape(L, E, P, G, N, gpus, X, &sh);
+  if (st != EPLB_OK || L == 0) return st;
+  if (!log2phy || !logcnt || !ring || !next_phy2log || !next_phyrank || !next_logcnt ||
+      !next_log2phy || !layer_done)
+    return EPLB_ERR_NULL;
+  if (T > 0 && (!idx || !out)) return EPLB_ERR_NULL;
+  if (T > 0 && (!aligned16(idx) || !aligned16(out))) return EPLB_ERR_ALIGN;
+  // the plan in force is read while the next one is written
+  if (next_log2phy == log2phy || next_logcnt == logcnt) return EPLB_ERR_SHAPE;
+  return launch_serve(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot, zero_slot,
+                      loads_out, sh, next_phy2log, next_phyrank, next_logcnt, next_log2phy,
+                      layer_done, status, stream);
 }
 
 eplb_status eplb_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,

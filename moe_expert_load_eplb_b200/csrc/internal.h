@@ -67,6 +67,17 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
                             int32_t *out, int64_t *counts, unsigned long long *bad,
                             int32_t *status, cudaStream_t stream);
 
+// The serving step in one launch: count + redirect with the plan in force
+// into ring[slot], then per layer, once its chunks are all counted, the window
+// sum and rebalance into the next plan (zeroing ring[zero_slot] if >= 0).
+eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
+                         const int32_t *log2phy, int32_t X, const int32_t *logcnt, int64_t t0,
+                         int32_t *out, unsigned long long *bad, int64_t *ring, int64_t W,
+                         int64_t slot, int64_t zero_slot, int64_t *loads_out,
+                         const RebalanceShape &sh, int32_t *next_phy2log, int32_t *next_phyrank,
+                         int32_t *next_logcnt, int32_t *next_log2phy, uint32_t *layer_done,
+                         int32_t *status, cudaStream_t stream);
+
 eplb_status launch_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,
                               int64_t R, int32_t E, int32_t P, int32_t gpus, double *gpu_load,
                               double *stats, int32_t *status, cudaStream_t stream);

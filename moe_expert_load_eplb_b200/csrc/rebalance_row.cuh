@@ -1,0 +1,841 @@
+// rebalance_row.cuh -- one row of S3/S4 (and the S2 ring sum) by one CTA:
+// the device code behind rebalance.cu's kernel and the serving-step kernel.
+//
+// Follows page "DualPipe и EPLB", Part 2: section "Алгоритм" (hierarchical
+// policy when num_groups % num_nodes == 0, else global = one group on one
+// node) and the appendix functions balanced_packing, replicate_experts and
+// rebalance_experts_hierarchical, with exact arithmetic:
+//   step 1  group loads -> balanced_packing over nodes (G/N groups each);
+//   step 2  replicate_experts per node: every extra replica goes to the
+//           largest load per replica w/c (cross-multiplied, lowest index on
+//           ties);
+//   step 3  replica loads w/c -> balanced_packing over the node's GPUs
+//           (P/gpus each); sums of w/c are held as integers w * (Lambda/c),
+//           Lambda a common multiple of the node's replica counts;
+//   then the index bookkeeping and log2phy.
+// balanced_packing visits items heaviest first with ties by ascending index
+// and puts each into the lightest non-full pack (lowest pack index on ties).
+//
+// Latency-bound design, measured phase by phase with clock64 probes:
+//   * the row lives in shared memory; every sort key is a composite integer
+//     (load << b | (mask - index)), so the stable (load desc, index asc)
+//     order is a plain descending order of distinct integers;
+//   * sorts count ranks CTA-wide (a key's rank is the number of larger keys
+//     in its segment); threads are grouped by segment and rank several keys
+//     against each loaded key; segments longer than 512 use a bitonic network;
+//   * replicate_experts: an expert outside the top R = P/N - E/N experts of
+//     its node (by load, ties by index) has at least R quotients ahead of it,
+//     so it never gets an extra replica; the R candidates are selected by
+//     rank and the greedy runs on them alone -- as a ranking of (candidate,
+//     divisor) pairs when there are few, else one candidate per lane with an
+//     xor-butterfly argmax;
+//   * balanced_packing keeps a node's packs sorted by composite key
+//     (weight << 12 | pack) across the lanes of a segment (one position per
+//     lane up to 32 packs, several per lane up to 256): each item takes the
+//     first (lightest, lowest index) pack, and every position compares its
+//     key and its right neighbour's with the updated pack's new key to shift
+//     or take it; wider nodes use one warp per node and a butterfly argmin;
+//   * Lambda is lcm(1..cmax) from the host when 64-bit keys can hold it, else
+//     the lcm of the counts present in the node; keys are 64-bit when the
+//     row's magnitudes allow and 128-bit otherwise.  All paths are exact, so
+//     none changes the result.
+#pragma once
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace eplb {
+namespace {
+
+
+// CTA size is chosen per launch: 512 threads when there are few rows (each
+// row's parallel phases then spread over 4 warps per scheduler), 128 when
+// many rows share every SM.
+constexpr int kMaxThreads = 512;
+constexpr int kFewRowThreads = 512;
+constexpr int kManyRowThreads = 128;
+__device__ __forceinline__ int nthr() { return static_cast<int>(blockDim.x); }
+__device__ __forceinline__ int nwarps() { return static_cast<int>(blockDim.x) >> 5; }
+constexpr int64_t kLoadLimit = int64_t(1) << 40;
+constexpr int kRankSortMax = 512;        // longer segments use the bitonic network
+constexpr int kTableMaxEntries = 16384;  // log2phy rows up to this size are built in smem
+// Every composite key keeps an index (item, pack, group or expert, all < 4096)
+// in its low kIdxBits bits, so keys are combined with constant shifts only.
+constexpr int kIdxBits = 12;
+constexpr uint64_t kIdxMask = (uint64_t(1) << kIdxBits) - 1;
+
+typedef unsigned __int128 u128;
+
+struct RbArgs {
+  // A row's loads are the sum of W ring rows: loads[r, e] = sum_w ring[w, r, e]
+  // (W = 1 for a plain load array).  zero_slot >= 0 clears that ring row's
+  // part of each row after it was read; loads_out (nullable) gets the sums.
+  int64_t *ring;
+  int64_t ring_w, ring_stride, zero_slot;
+  int64_t *loads_out;
+  int32_t *phy2log, *phyrank, *logcnt, *log2phy, *status;
+  RebalanceShape s;
+  uint32_t x_magic;
+  int table_vec4;  // log2phy rows may be written as 16-byte vectors
+};
+
+__host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
+__host__ __device__ inline int bitmap_words(const RebalanceShape &s) { return (s.cmax + 32) / 32; }
+__host__ __device__ inline bool table_in_smem(const RebalanceShape &s) {
+  return static_cast<int64_t>(s.E) * s.X <= kTableMaxEntries;
+}
+// experts per node that can receive extra replicas
+__host__ __device__ inline int num_cand(const RebalanceShape &s) {
+  return min(s.ppn - s.lpn, s.lpn);
+}
+
+// Shared-memory carve-up of one row (byte offsets), identical on host and device.
+struct Layout {
+  size_t keys, sorted, pw, w, wm, gkey, gsorted, npw, lam, cand_w, table, mlog2log, cnt, lc, p2m,
+      rrank, ipack, irank, outp, outr, gpack, grank, npc, pc, cand_i, cand_c, bitmap, total;
+  __host__ __device__ explicit Layout(const RebalanceShape &s) {
+    const int nc = num_cand(s);
+    size_t o = 0;
+    keys = o; o += size_t(s.N) * max(s.npad, s.lpn) * 16;  // u128/u64 keys, stride npad (or lpn)
+    sorted = o; o += size_t(s.N) * s.npad * 16;
+    pw = o; o += size_t(s.gpus) * 16;                       // pack weights of the warp fallback
+    o = align16(o);
+    w = o; o += size_t(s.E) * 8;
+    wm = o; o += size_t(s.E) * 8;
+    gkey = o; o += size_t(s.gpad) * 8;
+    gsorted = o; o += size_t(s.gpad) * 8;
+    npw = o; o += size_t(s.N) * 8;
+    lam = o; o += size_t(s.N) * 8;
+    cand_w = o; o += size_t(s.N) * nc * 8;
+    o = align16(o);
+    table = o; o += table_in_smem(s) ? size_t(s.E) * s.X * 4 : 0;
+    o = align16(o);
+    mlog2log = o; o += size_t(s.E) * 4;
+    cnt = o; o += size_t(s.E) * 4;
+    lc = o; o += size_t(s.E) * 4;
+    p2m = o; o += size_t(s.P) * 4;
+    rrank = o; o += size_t(s.P) * 4;
+    ipack = o; o += size_t(s.P) * 4;
+    irank = o; o += size_t(s.P) * 4;
+    outp = o; o += size_t(s.P) * 4;
+    outr = o; o += size_t(s.P) * 4;
+    gpack = o; o += size_t(s.G) * 4;
+    grank = o; o += size_t(s.G) * 4;
+    npc = o; o += size_t(s.N) * 4;
+    pc = o; o += size_t(s.gpus) * 4;
+    cand_i = o; o += size_t(s.N) * nc * 4;
+    cand_c = o; o += size_t(s.N) * nc * 4;
+    bitmap = o; o += size_t(s.N) * bitmap_words(s) * 4;
+    total = align16(o);
+  }
+};
+
+__device__ __forceinline__ uint64_t shfl_xor(uint64_t v, int off) {
+  return __shfl_xor_sync(0xffffffffu, static_cast<unsigned long long>(v), off);
+}
+__device__ __forceinline__ u128 shfl_xor(u128 v, int off) {
+  const uint64_t lo = shfl_xor(static_cast<uint64_t>(v), off);
+  const uint64_t hi = shfl_xor(static_cast<uint64_t>(v >> 64), off);
+  return (static_cast<u128>(hi) << 64) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_idx(uint64_t v, int src, int width) {
+  return __shfl_sync(0xffffffffu, static_cast<unsigned long long>(v), src, width);
+}
+__device__ __forceinline__ u128 shfl_idx(u128 v, int src, int width) {
+  const uint64_t lo = shfl_idx(static_cast<uint64_t>(v), src, width);
+  const uint64_t hi = shfl_idx(static_cast<uint64_t>(v >> 64), src, width);
+  return (static_cast<u128>(hi) << 64) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_down_k(uint64_t v, int d, int width) {
+  return __shfl_down_sync(0xffffffffu, static_cast<unsigned long long>(v), d, width);
+}
+__device__ __forceinline__ u128 shfl_down_k(u128 v, int d, int width) {
+  const uint64_t lo = shfl_down_k(static_cast<uint64_t>(v), d, width);
+  const uint64_t hi = shfl_down_k(static_cast<uint64_t>(v >> 64), d, width);
+  return (static_cast<u128>(hi) << 64) | lo;
+}
+template <typename K>
+__device__ __forceinline__ K kmin(K a, K b) {
+  return b < a ? b : a;
+}
+
+__device__ __forceinline__ uint32_t gcd_u32(uint32_t a, uint32_t b) {  // binary gcd
+  if (a == 0) return b;
+  if (b == 0) return a;
+  const int shift = __ffs(a | b) - 1;
+  a >>= __ffs(a) - 1;
+  do {
+    b >>= __ffs(b) - 1;
+    if (a > b) {
+      const uint32_t t = a;
+      a = b;
+      b = t;
+    }
+    b -= a;
+  } while (b != 0);
+  return a << shift;
+}
+
+// lcm(lam, c) with lam <= 2^62; false when the result would exceed 2^62.
+__device__ __forceinline__ bool lcm_into(uint64_t &lam, uint32_t c) {
+  if (c < 2) return true;
+  const uint32_t rem = lam >> 32 ? static_cast<uint32_t>(lam % c)
+                                 : static_cast<uint32_t>(lam) % c;
+  const uint32_t g = gcd_u32(rem, c);
+  const u128 next = static_cast<u128>(lam) * (c / g);
+  if (next > (static_cast<u128>(1) << 62)) return false;
+  lam = static_cast<uint64_t>(next);
+  return true;
+}
+
+// ---------------------------------------------------------------------------
+// Descending ranks of n distinct keys in each of nseg segments (segment g at
+// key + g * stride).  Threads are grouped by segment (nthr() / nseg per
+// segment); each ranks Q keys per pass (Q = 1, 2 or 4, the fewest that cover
+// the segment) against every key it loads.  emit(g, j, rank, key) receives
+// every key.
+template <int Q, typename K, typename Emit>
+__device__ void rank_pass(const K *key, int stride, int nseg, int n, int tps, Emit &emit) {
+  const int segs_per_pass = nthr() / tps;
+  const int sub = threadIdx.x % tps;
+  for (int g0 = 0; g0 < nseg; g0 += segs_per_pass) {
+    const int g = g0 + static_cast<int>(threadIdx.x) / tps;
+    if (static_cast<int>(threadIdx.x) / tps >= segs_per_pass || g >= nseg) continue;
+    const K *seg = key + g * stride;
+    for (int j0 = sub; j0 < n; j0 += tps * Q) {
+      K me[Q];
+      int r[Q];
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const int j = j0 + q * tps;
+        me[q] = j < n ? seg[j] : ~K(0);
+        r[q] = 0;
+      }
+#pragma unroll 4
+      for (int i = 0; i < n; ++i) {
+        const K kk = seg[i];
+#pragma unroll
+        for (int q = 0; q < Q; ++q) r[q] += kk > me[q] ? 1 : 0;
+      }
+#pragma unroll
+      for (int q = 0; q < Q; ++q) {
+        const int j = j0 + q * tps;
+        if (j < n) emit(g, j, r[q], me[q]);
+      }
+    }
+  }
+}
+
+template <typename K, typename Emit>
+__device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit emit) {
+  const int tps = nseg >= nthr() ? 1 : nthr() / nseg;
+  if (n <= tps)
+    rank_pass<1, K>(key, stride, nseg, n, tps, emit);
+  else if (n <= 2 * tps)
+    rank_pass<2, K>(key, stride, nseg, n, tps, emit);
+  else
+    rank_pass<4, K>(key, stride, nseg, n, tps, emit);
+}
+
+// CTA-wide bitonic sort, descending, of nseg segments of npad (power of two)
+// keys each, in place; padding keys must be 0.
+template <typename K>
+__device__ void bitonic_desc(K *key, int npad, int nseg) {
+  const int half = (npad * nseg) >> 1;
+  for (int k = 2; k <= npad; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int t = threadIdx.x; t < half; t += nthr()) {
+        const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1));
+        const int p = i | j;
+        const bool desc = ((i & (npad - 1)) & k) == 0;
+        const K x = key[i], y = key[p];
+        if ((x < y) == desc) {
+          key[i] = y;
+          key[p] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// balanced_packing's greedy over items sorted as composite keys
+// (load << 12 | (4095 - item)), descending; the pack keys are
+// weight << 12 | pack, so adding an item's load is one add of (key & ~4095).
+//
+// Same greedy with a node's packs spread over the lanes of a segment, in
+// sorted order: for m <= 32 a segment is the next power of two >= m lanes
+// with one position each; for larger m a segment is a whole warp and lane l
+// holds positions l*PL .. l*PL+PL-1.  Per item: position 0 (the lightest,
+// lowest index on ties) is broadcast, every position compares its key and
+// its right neighbour's with the pack's new key, and takes the neighbour's
+// key, the new key or its own -- one shuffle pair and a few selects per item
+// (a ballot + popc for the insertion point measured 45 cycles on the chain).
+// Counts move with keys.
+template <typename K, int PL>
+__device__ void pack_seg(const K *skey_base, int stride, int nseg, int n, int m, int cap,
+                         int32_t *ipack, int32_t *irank, int out_stride) {
+  const K imask = K(kIdxMask);
+  const K kmax = ~K(0);
+  int ms = 2;  // lanes per segment
+  while (ms < m && ms < 32) ms <<= 1;
+  if (PL > 1) ms = 32;
+  const int lane = threadIdx.x & 31;
+  const int li = lane & (ms - 1);            // lane within the segment
+  const int slot = static_cast<int>(threadIdx.x) / ms;
+  const int slots = nthr() / ms;
+  const int warp_first_slot = (static_cast<int>(threadIdx.x) & ~31) / ms;
+  for (int g0 = 0; g0 < nseg; g0 += slots) {
+    if (g0 + warp_first_slot >= nseg) continue;  // no segment of this warp is live: skip the chain
+    const int g = g0 + slot;
+    const bool active = g < nseg;
+    const K *skey = skey_base + (active ? g : 0) * stride;
+    K key[PL];
+    int cnt[PL];
+#pragma unroll
+    for (int r = 0; r < PL; ++r) {
+      const int pos = li * PL + r;
+      key[r] = pos < m ? K(pos) : kmax;  // pack pos, weight 0
+      cnt[r] = 0;
+    }
+    K nxt = skey[0];
+    for (int j = 0; j < n; ++j) {
+      const K c = nxt;
+      if (j + 1 < n) nxt = skey[j + 1];
+      const K best = shfl_idx(key[0], 0, ms);
+      const int bc = __shfl_sync(0xffffffffu, cnt[0], 0, ms);
+      const K up = shfl_down_k(key[0], 1, ms);  // position (li+1)*PL of the next lane
+      const int upc = __shfl_down_sync(0xffffffffu, cnt[0], 1, ms);
+      const K nk = bc + 1 < cap ? best + (c & ~imask) : kmax;
+      // lt(q) = position q >= 1 holds a key below the new one; the lt
+      // positions are a prefix 1..p.  Position q takes position q+1's key
+      // when lt(q+1), the new key when lt(q) or q == 0 (and not lt(q+1)),
+      // else keeps its own: no ballot needed, each lane sees q and q+1.
+      bool ltk[PL];
+#pragma unroll
+      for (int r = 0; r < PL; ++r) ltk[r] = (li * PL + r) >= 1 && key[r] < nk;
+      const bool lt_up = li + 1 < ms && up < nk;
+#pragma unroll
+      for (int r = 0; r < PL; ++r) {
+        const bool next_lt = r + 1 < PL ? ltk[r + 1 < PL ? r + 1 : r] : lt_up;
+        const K right = r + 1 < PL ? key[r + 1 < PL ? r + 1 : r] : up;
+        const int rightc = r + 1 < PL ? cnt[r + 1 < PL ? r + 1 : r] : upc;
+        const bool here = ltk[r] || (li * PL + r) == 0;
+        key[r] = next_lt ? right : (here ? nk : key[r]);
+        cnt[r] = next_lt ? rightc : (here ? bc + 1 : cnt[r]);
+      }
+      if (li == 0 && active) {
+        const int item = static_cast<int>(imask - (c & imask));
+        ipack[g * out_stride + item] = static_cast<int>(best & imask);
+        irank[g * out_stride + item] = bc;
+      }
+    }
+  }
+}
+
+// Same greedy for wide segments, one warp per segment: pack q is owned by
+// lane q % 32 (state in shared memory); each lane caches the composite key
+// of its lightest non-full pack; the warp takes the minimum with an xor
+// butterfly.
+template <typename K>
+__device__ void pack_warp(const K *skey, int n, int m, int cap, K *pw, int32_t *pc,
+                          int32_t *ipack, int32_t *irank) {
+  const int lane = threadIdx.x & 31;
+  const K imask = K(kIdxMask);
+  const K kmax = ~K(0);
+  for (int q = lane; q < m; q += 32) {
+    pw[q] = 0;
+    pc[q] = 0;
+  }
+  __syncwarp();
+  K best = lane < m ? K(lane) : kmax;
+  int rounds = 0;
+  while ((1 << rounds) < min(m, 32)) ++rounds;
+  for (int j = 0; j < n; ++j) {
+    const K ck = skey[j];
+    K b = best;
+    for (int r = rounds - 1; r >= 0; --r) b = kmin(b, shfl_xor(b, 1 << r));
+    const int q = static_cast<int>(b & imask);
+    if (b != kmax && lane == (q & 31)) {
+      const int rk = pc[q];
+      pc[q] = rk + 1;
+      pw[q] += ck & ~imask;  // weights kept pre-shifted
+      const int item = static_cast<int>(imask - (ck & imask));
+      ipack[item] = q;
+      irank[item] = rk;
+      K nb = kmax;
+      for (int qq = lane; qq < m; qq += 32)
+        if (pc[qq] < cap) nb = kmin(nb, pw[qq] | K(qq));
+      best = nb;
+    }
+    __syncwarp();
+  }
+}
+
+// Packs nseg segments (segment g: n sorted keys at skey + g * stride, results
+// at ipack/irank + g * out_stride) into m packs of cap items each.  Called by
+// every thread of the CTA (the lane-parallel variant needs whole warps).
+template <typename K>
+__device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
+                              int32_t *pc, int32_t *ipack, int32_t *irank, int out_stride) {
+  if (n <= 0) return;
+  if (m <= 32) {
+    pack_seg<K, 1>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
+  } else if (m <= 64) {
+    pack_seg<K, 2>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
+  } else if (m <= 128) {
+    pack_seg<K, 4>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
+  } else if (m <= 256 && sizeof(K) == 8) {
+    pack_seg<K, 8>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
+  } else {
+    for (int g = threadIdx.x >> 5; g < nseg; g += nwarps())
+      pack_warp<K>(skey + g * stride, n, m, cap, pw + g * m, pc + g * m, ipack + g * out_stride,
+                   irank + g * out_stride);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// replicate_experts.  a beats b on a larger w/c, then a lower index.
+__device__ __forceinline__ bool rep_better(int64_t aw, int ac, int ai, int64_t bw, int bc, int bi) {
+  const int64_t lhs = aw * static_cast<int64_t>(bc);
+  const int64_t rhs = bw * static_cast<int64_t>(ac);
+  return lhs > rhs || (lhs == rhs && ai < bi);
+}
+
+// D'Hondt form of the greedy: the extra replicas, in order, are the R best
+// (candidate k, divisor d) pairs by w_k / d desc, expert index asc, d asc
+// (each step takes the largest current quotient, and an expert's quotients
+// w/1, w/2, ... only decrease).  Pair (k, d) has at least k + d - 1 pairs
+// ahead of it (the k heavier candidates' first pairs and (k, 1 .. d-1)), so
+// only pairs with d <= R - k can be picked and only those are ranked.  All
+// pairs of all nodes are ranked in parallel; the picks need no serial chain.
+__device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
+                                const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
+                                int32_t *rrank) {
+  const int R = s.ppn - s.lpn, nc = num_cand(s);
+  const int grid = nc * R;
+  for (int t = threadIdx.x; t < s.N * grid; t += nthr()) {
+    const int n = t / grid;
+    const int p = t - n * grid;
+    const int k = p / R;
+    const int d = p - k * R + 1;
+    if (d > R - k) continue;
+    const int64_t w = cand_w[n * nc + k];
+    const int id = cand_i[n * nc + k];
+    int rank = 0;
+    for (int k2 = 0; k2 < nc; ++k2) {
+      const int64_t w2 = cand_w[n * nc + k2];
+      const int id2 = cand_i[n * nc + k2];
+      const bool lower = id2 < id, same = id2 == id;
+      for (int d2 = 1; d2 <= R - k2; ++d2) {
+        const int64_t lhs = w2 * d, rhs = w * d2;
+        rank += (lhs > rhs || (lhs == rhs && (lower || (same && d2 < d)))) ? 1 : 0;
+      }
+    }
+    if (rank < R) {
+      p2m[n * s.ppn + s.lpn + rank] = id;
+      rrank[n * s.ppn + s.lpn + rank] = d;
+      atomicAdd(&cand_c[n * nc + k], 1);
+    }
+  }
+}
+
+// Greedy over nc <= 32 candidates, one per lane of a warp.
+__device__ void replicate_warp(const RebalanceShape &s, int n, const int64_t *cand_w,
+                               const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
+                               int32_t *rrank) {
+  const int lane = threadIdx.x & 31;
+  const int nc = num_cand(s);
+  const int bp = n * s.ppn;
+  const bool valid = lane < nc;
+  const int64_t w = valid ? cand_w[n * nc + lane] : 0;
+  const int id = valid ? cand_i[n * nc + lane] : 0x7fffffff;
+  int c = 1;
+  int rounds = 0;
+  while ((1 << rounds) < min(nc, 32)) ++rounds;
+  for (int r = 0; r < s.ppn - s.lpn; ++r) {
+    int64_t bw = w;
+    int bc = c, bi = id, bl = lane;
+    for (int k = rounds - 1; k >= 0; --k) {
+      const int64_t ow = static_cast<int64_t>(shfl_xor(static_cast<uint64_t>(bw), 1 << k));
+      const int oc = __shfl_xor_sync(0xffffffffu, bc, 1 << k);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, 1 << k);
+      const int ol = __shfl_xor_sync(0xffffffffu, bl, 1 << k);
+      if (rep_better(ow, oc, oi, bw, bc, bi)) {
+        bw = ow;
+        bc = oc;
+        bi = oi;
+        bl = ol;
+      }
+    }
+    if (valid && lane == bl) {
+      p2m[bp + s.lpn + r] = id;
+      rrank[bp + s.lpn + r] = c;
+      ++c;
+    }
+  }
+  if (valid) cand_c[n * nc + lane] = c;
+  __syncwarp();
+}
+
+// Any number of candidates (all experts of the node), counts in shared memory.
+__device__ void replicate_smem(const RebalanceShape &s, int n, const int64_t *wm, int32_t *cnt,
+                               int32_t *p2m, int32_t *rrank) {
+  const int lane = threadIdx.x & 31;
+  const int bm = n * s.lpn, bp = n * s.ppn;
+  auto local_best = [&](int64_t &bw, int &bc, int &bi) {
+    bw = 0;
+    bc = 1;
+    bi = 0x7fffffff;
+    for (int i = lane; i < s.lpn; i += 32)
+      if (rep_better(wm[bm + i], cnt[bm + i], i, bw, bc, bi)) {
+        bw = wm[bm + i];
+        bc = cnt[bm + i];
+        bi = i;
+      }
+  };
+  int64_t bw;
+  int bc, bi;
+  local_best(bw, bc, bi);
+  for (int r = 0; r < s.ppn - s.lpn; ++r) {
+    int64_t mw = bw;
+    int mc = bc, mi = bi;
+    for (int k = 16; k >= 1; k >>= 1) {
+      const int64_t ow = static_cast<int64_t>(shfl_xor(static_cast<uint64_t>(mw), k));
+      const int oc = __shfl_xor_sync(0xffffffffu, mc, k);
+      const int oi = __shfl_xor_sync(0xffffffffu, mi, k);
+      if (rep_better(ow, oc, oi, mw, mc, mi)) {
+        mw = ow;
+        mc = oc;
+        mi = oi;
+      }
+    }
+    if (lane == (mi & 31)) {
+      cnt[bm + mi] = mc + 1;
+      p2m[bp + s.lpn + r] = mi;
+      rrank[bp + s.lpn + r] = mc;
+      local_best(bw, bc, bi);
+    }
+    __syncwarp();
+  }
+}
+
+__device__ void write_error_row(const RbArgs &a, int64_t row) {
+  const RebalanceShape &s = a.s;
+  for (int t = threadIdx.x; t < s.P; t += nthr()) {
+    a.phy2log[row * s.P + t] = -1;
+    a.phyrank[row * s.P + t] = -1;
+  }
+  for (int e = threadIdx.x; e < s.E; e += nthr()) a.logcnt[row * s.E + e] = 0;
+  int32_t *gl = a.log2phy + row * static_cast<int64_t>(s.E) * s.X;
+  for (int i = threadIdx.x; i < s.E * s.X; i += nthr()) gl[i] = -1;
+}
+
+template <typename K>
+__device__ void step3(const RbArgs &a, unsigned char *smem, const Layout &lay) {
+  const RebalanceShape &s = a.s;
+  K *keys = reinterpret_cast<K *>(smem + lay.keys);
+  K *sorted = reinterpret_cast<K *>(smem + lay.sorted);
+  const int64_t *wm = reinterpret_cast<const int64_t *>(smem + lay.wm);
+  const uint64_t *lam = reinterpret_cast<const uint64_t *>(smem + lay.lam);
+  const int32_t *cnt = reinterpret_cast<const int32_t *>(smem + lay.cnt);
+  const int32_t *p2m = reinterpret_cast<const int32_t *>(smem + lay.p2m);
+  const K imask = K(kIdxMask);
+  const bool ranked = s.npad <= kRankSortMax;
+  const int per = ranked ? s.ppn : s.npad;
+  for (int t = threadIdx.x; t < s.N * per; t += nthr()) {
+    const int n = t / per;
+    const int j = t - n * per;
+    K key = 0;
+    if (j < s.ppn) {
+      const int m = n * s.lpn + p2m[n * s.ppn + j];
+      const uint32_t c = static_cast<uint32_t>(cnt[m]);
+      const uint64_t scale = c == 1 ? lam[n] : lam[n] / c;
+      key = ((K(static_cast<uint64_t>(wm[m])) * K(scale)) << kIdxBits) | (imask - K(j));
+    }
+    keys[n * s.npad + j] = key;
+  }
+  __syncthreads();
+  const K *skeys = keys;
+  if (ranked) {
+    rank_segments<K>(keys, s.npad, s.N, s.ppn,
+                     [&](int g, int, int r, K k) { sorted[g * s.npad + r] = k; });
+    skeys = sorted;
+    __syncthreads();
+  } else {
+    bitonic_desc<K>(keys, s.npad, s.N);
+  }
+  pack_segments<K>(skeys, s.npad, s.N, s.ppn, s.mpn, s.ppg, reinterpret_cast<K *>(smem + lay.pw), reinterpret_cast<int32_t *>(smem + lay.pc),
+                   reinterpret_cast<int32_t *>(smem + lay.ipack),
+                   reinterpret_cast<int32_t *>(smem + lay.irank), s.ppn);
+}
+
+// One row of rebalance_experts, by the whole CTA, in `smem` (Layout(a.s).total
+// bytes).  Called by every thread of the CTA.
+__device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsigned char *smem) {
+  __shared__ int flags[2];  // [0] 128-bit keys needed, [1] exact ratio not representable
+  const RebalanceShape &s = a.s;
+  const Layout lay(s);
+  int64_t *w = reinterpret_cast<int64_t *>(smem + lay.w);
+  int64_t *wm = reinterpret_cast<int64_t *>(smem + lay.wm);
+  uint64_t *gkey = reinterpret_cast<uint64_t *>(smem + lay.gkey);
+  uint64_t *gsorted = reinterpret_cast<uint64_t *>(smem + lay.gsorted);
+  uint64_t *lam = reinterpret_cast<uint64_t *>(smem + lay.lam);
+  int64_t *cand_w = reinterpret_cast<int64_t *>(smem + lay.cand_w);
+  int32_t *mlog2log = reinterpret_cast<int32_t *>(smem + lay.mlog2log);
+  int32_t *cnt = reinterpret_cast<int32_t *>(smem + lay.cnt);
+  int32_t *lc = reinterpret_cast<int32_t *>(smem + lay.lc);
+  int32_t *p2m = reinterpret_cast<int32_t *>(smem + lay.p2m);
+  int32_t *rrank = reinterpret_cast<int32_t *>(smem + lay.rrank);
+  int32_t *ipack = reinterpret_cast<int32_t *>(smem + lay.ipack);
+  int32_t *irank = reinterpret_cast<int32_t *>(smem + lay.irank);
+  int32_t *outp = reinterpret_cast<int32_t *>(smem + lay.outp);
+  int32_t *outr = reinterpret_cast<int32_t *>(smem + lay.outr);
+  int32_t *gpack = reinterpret_cast<int32_t *>(smem + lay.gpack);
+  int32_t *grank = reinterpret_cast<int32_t *>(smem + lay.grank);
+  int32_t *cand_i = reinterpret_cast<int32_t *>(smem + lay.cand_i);
+  int32_t *cand_c = reinterpret_cast<int32_t *>(smem + lay.cand_c);
+
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    flags[0] = 0;
+    flags[1] = 0;
+  }
+
+  // ---- load the row (the window sum over the ring); loads in [0, 2^40) --
+  // two threads per expert, each summing half of the ring rows with all its
+  // loads in flight
+  bool bad = false;
+  {
+    const int lane = tid & 31;
+    const int64_t half = (a.ring_w + 1) >> 1;
+    for (int t = tid; t - lane < 2 * s.E; t += nthr()) {  // warp-uniform for the shuffle
+      const bool live = t < 2 * s.E;
+      const int e = t >> 1;
+      const int64_t at = row * s.E + e;
+      const int64_t k0 = (t & 1) * half;
+      const int64_t k1 = min(a.ring_w, k0 + half);
+      int64_t x = 0;
+      if (live) {
+#pragma unroll 8
+        for (int64_t k = k0; k < k1; ++k) x += __ldcg(a.ring + k * a.ring_stride + at);
+      }
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      if (live && !(t & 1)) {
+        w[e] = x;
+        if (a.loads_out) a.loads_out[at] = x;
+        if (a.zero_slot >= 0) a.ring[a.zero_slot * a.ring_stride + at] = 0;
+        bad |= (x < 0) | (x >= kLoadLimit);
+      }
+    }
+  }
+  if (__syncthreads_or(bad)) {
+    write_error_row(a, row);
+    if (tid == 0) report(a.status, EPLB_ERR_RANGE);
+    return;
+  }
+
+  // ---- step 1: groups -> nodes ---------------------------------------------
+  if (s.gpn == 1) {  // one group per node: the pages' identity short-cut
+    for (int g = tid; g < s.G; g += nthr()) {
+      gpack[g] = g;
+      grank[g] = 0;
+    }
+  } else {
+    for (int g = tid >> 5; g < s.G; g += nwarps()) {  // one warp per group
+      const int lane = tid & 31;
+      uint64_t sum = 0;
+      for (int i = lane; i < s.gs; i += 32) sum += static_cast<uint64_t>(w[g * s.gs + i]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (lane == 0) gkey[g] = (sum << kIdxBits) | (kIdxMask - g);
+    }
+    __syncthreads();
+    const uint64_t *gs_keys = gsorted;
+    if (s.gpad <= kRankSortMax) {
+      rank_segments<uint64_t>(gkey, s.gpad, 1, s.G,
+                              [&](int, int, int r, uint64_t k) { gsorted[r] = k; });
+    } else {
+      for (int g = s.G + tid; g < s.gpad; g += nthr()) gkey[g] = 0;
+      __syncthreads();
+      bitonic_desc<uint64_t>(gkey, s.gpad, 1);
+      gs_keys = gkey;
+    }
+    __syncthreads();
+    pack_segments<uint64_t>(gs_keys, s.gpad, 1, s.G, s.N, s.gpn,
+                            reinterpret_cast<uint64_t *>(smem + lay.npw),
+                            reinterpret_cast<int32_t *>(smem + lay.npc), gpack, grank, s.G);
+  }
+  __syncthreads();
+  // mlog = logical order after the node permutation; replicate's initial state
+  for (int e = tid; e < s.E; e += nthr()) {
+    const int g = e / s.gs;
+    const int m = (gpack[g] * s.gpn + grank[g]) * s.gs + (e - g * s.gs);
+    mlog2log[m] = e;
+    wm[m] = w[e];
+    cnt[m] = 1;
+    const int n = m / s.lpn;
+    const int i = m - n * s.lpn;
+    p2m[n * s.ppn + i] = i;
+    rrank[n * s.ppn + i] = 0;
+  }
+  __syncthreads();
+
+  // ---- step 2: replicate_experts inside every node -------------------------
+  const int nc = num_cand(s);
+  if (nc > 0 && nc <= 32) {
+    // candidates: the nc heaviest experts of each node (ties by index)
+    uint64_t *ckey = reinterpret_cast<uint64_t *>(smem + lay.keys);
+    for (int m = tid; m < s.E; m += nthr()) {
+      const int n = m / s.lpn;
+      ckey[m] = (static_cast<uint64_t>(wm[m]) << kIdxBits) | (kIdxMask - (m - n * s.lpn));
+    }
+    __syncthreads();
+    rank_segments<uint64_t>(ckey, s.lpn, s.N, s.lpn, [&](int g, int j, int r, uint64_t) {
+      if (r < nc) {
+        cand_w[g * nc + r] = wm[g * s.lpn + j];
+        cand_i[g * nc + r] = j;
+      }
+    });
+    __syncthreads();
+    if (nc * (s.ppn - s.lpn) <= 256) {
+      for (int t = tid; t < s.N * nc; t += nthr()) cand_c[t] = 1;
+      __syncthreads();
+      replicate_pairs(s, cand_w, cand_i, cand_c, p2m, rrank);
+    } else {
+      for (int n = tid >> 5; n < s.N; n += nwarps())
+        replicate_warp(s, n, cand_w, cand_i, cand_c, p2m, rrank);
+    }
+    __syncthreads();
+    for (int t = tid; t < s.N * nc; t += nthr()) {
+      const int n = t / nc;
+      cnt[n * s.lpn + cand_i[t]] = cand_c[t];
+    }
+  } else if (nc > 32) {
+    for (int n = tid >> 5; n < s.N; n += nwarps()) replicate_smem(s, n, wm, cnt, p2m, rrank);
+  }
+  __syncthreads();
+
+  // ---- Lambda and key width per node (one thread per node) ----------------
+  if (s.ppg > 1) {
+    for (int n = tid; n < s.N; n += nthr()) {
+      int64_t wmax = 0;
+      if (nc > 0 && nc <= 32) {
+        wmax = cand_w[n * nc];
+      } else {
+        for (int i = 0; i < s.lpn; ++i) wmax = max(wmax, wm[n * s.lpn + i]);
+      }
+      auto width = [&](uint64_t l) -> int {
+        const u128 maxsum = static_cast<u128>(static_cast<uint64_t>(wmax)) * l * s.ppg;
+        if ((maxsum >> (63 - kIdxBits)) == 0) return 0;
+        if ((maxsum >> (127 - kIdxBits)) == 0) return 1;
+        return 2;
+      };
+      uint64_t l = s.lam_fixed;
+      int wd = 2;
+      if (l != 0) wd = width(l);
+      if (wd != 0) {
+        // lcm of the counts present in the node
+        l = 1;
+        bool ok = true;
+        if (nc > 0 && nc <= 32 && s.cmax < 64) {
+          uint64_t present = 0;  // bit c: some candidate has c replicas
+          for (int k = 0; k < nc; ++k) present |= uint64_t(1) << cand_c[n * nc + k];
+          present &= ~uint64_t(3);
+          while (present && ok) {
+            const int c = __ffsll(static_cast<long long>(present)) - 1;
+            present &= present - 1;
+            ok = lcm_into(l, static_cast<uint32_t>(c));
+          }
+        } else if (nc > 0 && nc <= 32) {
+          for (int k = 0; k < nc && ok; ++k) ok = lcm_into(l, static_cast<uint32_t>(cand_c[n * nc + k]));
+        } else {
+          for (int i = 0; i < s.lpn && ok; ++i) ok = lcm_into(l, static_cast<uint32_t>(cnt[n * s.lpn + i]));
+        }
+        wd = ok ? width(l) : 2;
+      }
+      lam[n] = l;
+      if (wd == 2) atomicOr(&flags[1], 1);
+      if (wd == 1) atomicOr(&flags[0], 1);
+    }
+    __syncthreads();
+  }
+  if (flags[1]) {
+    write_error_row(a, row);
+    if (tid == 0) report(a.status, EPLB_ERR_RANGE);
+    return;
+  }
+
+  // ---- step 3: replicas -> GPUs of each node ------------------------------
+  if (s.ppg == 1) {  // one replica per GPU: identity short-cut
+    for (int t = tid; t < s.P; t += nthr()) {
+      const int n = t / s.ppn;
+      ipack[t] = t - n * s.ppn;
+      irank[t] = 0;
+    }
+  } else if (flags[0] == 0) {
+    step3<uint64_t>(a, smem, lay);
+  } else {
+    step3<u128>(a, smem, lay);
+  }
+  __syncthreads();
+
+  // ---- assembly: pphy = node*ppn + gpu*ppg + rank -------------------------
+  for (int t = tid; t < s.P; t += nthr()) {
+    const int n = t / s.ppn;
+    const int pphy = n * s.ppn + ipack[t] * s.ppg + irank[t];
+    outp[pphy] = mlog2log[n * s.lpn + p2m[t]];
+    outr[pphy] = rrank[t];
+  }
+  for (int m = tid; m < s.E; m += nthr()) lc[mlog2log[m]] = cnt[m];
+  __syncthreads();
+  for (int t = tid; t < s.P; t += nthr()) {
+    a.phy2log[row * s.P + t] = outp[t];
+    a.phyrank[row * s.P + t] = outr[t];
+  }
+  for (int e = tid; e < s.E; e += nthr()) a.logcnt[row * s.E + e] = lc[e];
+  const int EX = s.E * s.X;
+  int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
+  bool slots = false;
+  if (table_in_smem(s)) {
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
+    for (int i = tid; i < EX; i += nthr()) tbl[i] = -1;
+    __syncthreads();
+    for (int t = tid; t < s.P; t += nthr()) {
+      const int k = outr[t];
+      if (k < s.X)
+        tbl[outp[t] * s.X + k] = t;
+      else
+        slots = true;
+    }
+    __syncthreads();
+    if (a.table_vec4) {
+      const int4 *src = reinterpret_cast<const int4 *>(tbl);
+      int4 *dst = reinterpret_cast<int4 *>(gl);
+      for (int i = tid; i < (EX >> 2); i += nthr()) dst[i] = src[i];
+    } else {
+      for (int i = tid; i < EX; i += nthr()) gl[i] = tbl[i];
+    }
+  } else {
+    for (int t = tid; t < s.P; t += nthr()) {
+      const int k = outr[t];
+      if (k < s.X)
+        gl[outp[t] * s.X + k] = t;
+      else
+        slots = true;
+    }
+    const uint32_t X = static_cast<uint32_t>(s.X);
+    for (int i = tid; i < EX; i += nthr()) {
+      const uint32_t e = div_magic(static_cast<uint32_t>(i), X, a.x_magic);
+      if (static_cast<int>(i - e * X) >= lc[e]) gl[i] = -1;
+    }
+  }
+  if (slots) report(a.status, EPLB_ERR_SLOTS);
+}
+
+
+}  // namespace
+}  // namespace eplb

@@ -6,7 +6,11 @@ round-trip:
 serving (default): the plan in force (built from earlier steps' loads, the
   moving-average estimate of page "DualPipe и EPLB", Part 2, section
   "Алгоритм") redirects this step's indices in the same pass that counts
-  them, so the indices cross HBM once; two launches per step:
+  them, so the indices cross HBM once; two launches per step (with
+  single_launch=True and no process group, one: serve_step builds each
+  layer's next plan as soon as that layer's indices are all counted -- on the
+  DeepSeek-V3 prefill step this measured slower, the early layers' plans
+  holding SM slots the later layers' chunks wait for):
     1. count_redirect: indices -> ring row (step % W, cleared beforehand) and
        physical indices;
     2. rebalance_window: the window sum over the ring and the next plan of
@@ -27,7 +31,7 @@ from typing import Optional, Sequence
 import torch
 
 from . import (Plan, count_loads, count_redirect, default_slots, rebalance, rebalance_window,
-               redirect, window_accumulate)
+               redirect, serve_step, window_accumulate)
 from .distributed import allreduce_loads
 
 
@@ -43,7 +47,8 @@ class EplbStep:
 
     def __init__(self, L: int, T: int, K: int, E: int, P: int, G: int, N: int, gpus: int,
                  window: int = 1, device="cuda", slots: Optional[int] = None,
-                 token_offset: int = 0, group=None, fused: bool = True):
+                 token_offset: int = 0, group=None, fused: bool = True,
+                 single_launch: bool = False):
         self.L, self.T, self.K, self.E = L, T, K, E
         self.P, self.G, self.N, self.gpus = P, G, N, gpus
         self.W = window
@@ -52,6 +57,9 @@ class EplbStep:
         self.token_offset = token_offset
         self.group = group
         self.fused = fused
+        # one launch per step needs every rank's counts before a layer's plan:
+        # only without a process group
+        self.single = fused and single_launch and group is None
         dev = self.device
         self.ring = torch.zeros((window, L, E), dtype=torch.int64, device=dev)
         self.loads = torch.zeros((1, L, E), dtype=torch.int64, device=dev)
@@ -60,13 +68,14 @@ class EplbStep:
         self.out = torch.empty((L, T, K), dtype=torch.int32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.bad = torch.zeros(1, dtype=torch.int64, device=dev)
+        self.layer_done = torch.zeros(L, dtype=torch.int32, device=dev)
         self.steps_done = 0
         self.primed = False
 
     @property
     def launches_per_step(self) -> int:
         """Kernels of this library launched per step."""
-        return 2 if self.fused else 4
+        return 1 if self.single else (2 if self.fused else 4)
 
     @property
     def plan(self) -> Plan:
@@ -96,9 +105,10 @@ class EplbStep:
         Returns (plan used for this step's redirect, redirected indices); the
         serving order's new plan is ``self.plan`` afterwards.  ``marks``: six
         CUDA events recorded on the current stream around the stages
-        count | allreduce | window | rebalance | redirect (the serving order
-        records its fused count+redirect under count, its fused
-        window+rebalance under rebalance, and empty window / redirect stages).
+        count | allreduce | window | rebalance | redirect (the two-launch
+        serving order records its fused count+redirect under count, its fused
+        window+rebalance under rebalance, and empty window / redirect stages;
+        the one-launch serving step records the whole step under count).
         """
         if self.fused and not self.primed:
             raise RuntimeError("serving order needs a plan in force: call fill_history() first")
@@ -106,6 +116,17 @@ class EplbStep:
         row = self.ring[self.steps_done % self.W]
         used = self.plans[self.cur]
         rec(0)
+        if self.single:
+            nxt = self.plans[1 - self.cur]
+            serve_step(idx, used, self.ring, self.steps_done % self.W, nxt, self.layer_done, self.G,
+                       self.N, self.gpus, zero_slot=(self.steps_done + 1) % self.W,
+                       token_offset=self.token_offset, out=self.out, loads_out=self.loads,
+                       bad=self.bad, status=self.status)
+            for k in range(1, 6):
+                rec(k)
+            self.steps_done += 1
+            self.cur = 1 - self.cur
+            return used, self.out
         if self.fused:
             # the ring row was cleared by the previous step's rebalance_window
             count_redirect(idx, self.E, used.log2phy, used.logcnt, self.token_offset, counts=row,

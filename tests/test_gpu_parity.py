@@ -464,14 +464,17 @@ def test_pipeline_fresh_order_c2(c2_idx):
     assert np.array_equal(_np(out), red)
 
 
-def test_pipeline_serving_order_c2(c2_idx):
-    """Three serving steps: each redirects with the plan in force, then rebuilds it."""
+@pytest.mark.parametrize("single", [True, False])
+def test_pipeline_serving_order_c2(c2_idx, single):
+    """Three serving steps: each redirects with the plan in force, then rebuilds it
+    (one launch per step, or count_redirect + rebalance_window)."""
     from moe_expert_load_eplb_b200.pipeline import EplbStep
     c = W.CONFIGS[2]
     W_ = 4
     hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, 2, device=DEV)
     step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV, fused=True,
-                    token_offset=1000)
+                    token_offset=1000, single_launch=single)
+    assert step.launches_per_step == (1 if single else 2)
     step.fill_history(hist)
     ring = np.concatenate([_np(hist), np.zeros((1, c.L, c.E), np.int64)], axis=0)
     plan_ref = _oracle_plan_from_ring(ring, c, step.X)
@@ -488,6 +491,105 @@ def test_pipeline_serving_order_c2(c2_idx):
         ring[(W_ - 1 + s_i) % W_] = counts
         plan_ref = _oracle_plan_from_ring(ring, c, step.X)
         _assert_plan_equal(step.plan, plan_ref)
+        assert int(step.layer_done.abs().sum().item()) == 0
+
+
+# ------------------------------------------------------- one-launch serve step --
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+@pytest.mark.parametrize("shape", [
+    (2, 4096, 2, 12, 16, 4, 2, 8),      # the worked example's sizes, many tokens
+    (3, 70001, 8, 24, 40, 6, 2, 4),     # several chunks per layer, ragged tail
+    (5, 3, 7, 24, 40, 6, 2, 4),         # fewer indices than a vector per layer
+    (4, 0, 4, 24, 40, 6, 2, 4),         # no tokens: the plan from the ring alone
+    (2, 20000, 3, 32, 48, 4, 3, 6),     # global policy (G % N != 0), K not a multiple of 4
+    (58, 8192, 8, 256, 288, 8, 4, 32),  # DeepSeek-V3 shape, decode-sized batch
+])
+@pytest.mark.parametrize("W_,slot,zero_slot", [(3, 1, 2), (1, 0, 0), (4, 3, -1)])
+def test_serve_step_matches_oracle(shape, W_, slot, zero_slot):
+    L, T, K, E, P, G, N, gpus = shape
+    X = P - E + 1
+    rng = np.random.default_rng(L * 31 + T + K + W_ * 7 + slot)
+    ring = rng.integers(0, 5000, (W_, L, E)).astype(np.int64)
+    ring[slot] = rng.integers(0, 3, (L, E))  # counts already in the slot are added to
+    plan_in = oracle.rebalance(rng.integers(0, 10000, (L, E)), P, G, N, gpus, slots=X)
+    idx = rng.integers(-1, E + 1, (L, T, K)).astype(np.int32)
+    t0 = 4321
+    ring_d = _dev(ring)
+    used = eplb.Plan(*[_dev(a) for a in plan_in])
+    nxt = eplb.Plan(*[torch.full(a.shape, 7, dtype=torch.int32, device=DEV) for a in plan_in])
+    done = torch.zeros(L, dtype=torch.int32, device=DEV)
+    loads = torch.zeros((L, E), dtype=torch.int64, device=DEV)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    st = _status()
+    out = eplb.serve_step(_dev(idx), used, ring_d, slot, nxt, done, G, N, gpus, zero_slot=zero_slot,
+                          token_offset=t0, loads_out=loads, bad=bad, status=st)
+    torch.cuda.synchronize()
+    counts, nbad = oracle.count_loads(idx, E)
+    ring_ref = ring.copy()
+    ring_ref[slot] += counts
+    loads_ref = ring_ref.sum(axis=0)
+    next_ref = oracle.rebalance(loads_ref, P, G, N, gpus, slots=X)
+    red, _ = oracle.redirect(idx, plan_in[3], plan_in[2], t0)
+    if zero_slot >= 0:
+        ring_ref[zero_slot] = 0
+    assert int(st.item()) == 0
+    assert np.array_equal(_np(out), red)
+    assert int(bad.item()) == nbad
+    assert np.array_equal(_np(loads), loads_ref)
+    _assert_plan_equal(nxt, next_ref)
+    assert np.array_equal(_np(ring_d), ring_ref)
+    assert int(done.abs().sum().item()) == 0
+
+
+def test_serve_step_reports_range_and_keeps_going():
+    """A window sum outside [0, 2^40) marks its row and sets EPLB_ERR_RANGE;
+    the counters still end at zero."""
+    L, T, K, E, P, G, N, gpus = 3, 1000, 4, 24, 40, 6, 2, 4
+    X = P - E + 1
+    rng = np.random.default_rng(5)
+    ring = rng.integers(0, 100, (2, L, E)).astype(np.int64)
+    ring[1, 1, 3] = 1 << 41
+    plan_in = oracle.rebalance(rng.integers(0, 100, (L, E)), P, G, N, gpus, slots=X)
+    used = eplb.Plan(*[_dev(a) for a in plan_in])
+    nxt = eplb.Plan(*[torch.empty(a.shape, dtype=torch.int32, device=DEV) for a in plan_in])
+    done = torch.zeros(L, dtype=torch.int32, device=DEV)
+    st = _status()
+    idx = _dev(rng.integers(0, E, (L, T, K)).astype(np.int32))
+    eplb.serve_step(idx, used, _dev(ring), 0, nxt, done, G, N, gpus, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+    assert int(done.abs().sum().item()) == 0
+    assert (_np(nxt.phy2log)[1] == -1).all()
+    loads = ring.sum(axis=0) + oracle.count_loads(_np(idx), E)[0]  # slot 0 received the counts
+    ref = oracle.rebalance(loads[[0, 2]], P, G, N, gpus, slots=X)
+    assert np.array_equal(_np(nxt.phy2log)[[0, 2]], ref[0])
+
+
+def test_serve_step_host_errors():
+    L, T, K, E, P, G, N, gpus = 2, 64, 4, 12, 16, 4, 2, 8
+    X = P - E + 1
+    plan = eplb.Plan(torch.zeros((L, P), dtype=torch.int32, device=DEV),
+                     torch.zeros((L, P), dtype=torch.int32, device=DEV),
+                     torch.ones((L, E), dtype=torch.int32, device=DEV),
+                     torch.zeros((L, E, X), dtype=torch.int32, device=DEV))
+    ring = torch.zeros((2, L, E), dtype=torch.int64, device=DEV)
+    idx = torch.zeros((L, T, K), dtype=torch.int32, device=DEV)
+    done = torch.zeros(L, dtype=torch.int32, device=DEV)
+    with pytest.raises(eplb.EplbError) as ei:  # the next plan is the plan in force
+        eplb.serve_step(idx, plan, ring, 0, plan, done, G, N, gpus)
+    assert ei.value.code == 2
+    nxt = eplb.Plan(*[torch.empty_like(t) for t in plan])
+    for slot, zero_slot in ((2, -1), (-1, 0), (0, 2), (0, -2)):
+        with pytest.raises(eplb.EplbError) as ei:
+            eplb.serve_step(idx, plan, ring, slot, nxt, done, G, N, gpus, zero_slot=zero_slot)
+        assert ei.value.code == 2
+    with pytest.raises(eplb.EplbError) as ei:  # E % G
+        eplb.serve_step(idx, plan, ring, 0, nxt, done, 5, N, gpus)
+    assert ei.value.code == 3
 
 
 # ------------------------------------------- plan stats, fold, initial map, diff --
