@@ -225,6 +225,30 @@ eplb_status eplb_serve_step(const int32_t *idx, int64_t L, int64_t T, int32_t K,
                             uint32_t *layer_done, int32_t *status, cudaStream_t stream);
 
 /*
+ * eplb_serve_step without the caller's layer_done array: the per-layer
+ * counters live in a library-owned device array (4096 layers, one per
+ * device, zero at load and left zero by every call), so the call allocates
+ * nothing and needs no work buffer.  The pages have no counterpart to this
+ * entry point; it is a convenience form of eplb_serve_step with identical
+ * results.
+ * Because all calls on one device share that array, two calls of this entry
+ * point must not be in flight at the same time on one device (e.g. on two
+ * streams without ordering between them); use eplb_serve_step with one
+ * layer_done array per stream for that.
+ * Errors: those of eplb_serve_step, and EPLB_ERR_LIMIT when L > 4096 (checked
+ * before anything else).
+ */
+eplb_status eplb_serve_step_noalloc(const int32_t *idx, int64_t L, int64_t T, int32_t K,
+                                    int32_t E, const int32_t *log2phy, int32_t X,
+                                    const int32_t *logcnt, int64_t t0, int32_t *out,
+                                    unsigned long long *bad, int64_t *ring, int64_t W,
+                                    int64_t slot, int64_t zero_slot, int32_t P, int32_t G,
+                                    int32_t N, int32_t gpus, int64_t *loads_out,
+                                    int32_t *next_phy2log, int32_t *next_phyrank,
+                                    int32_t *next_logcnt, int32_t *next_log2phy, int32_t *status,
+                                    cudaStream_t stream);
+
+/*
  * Plan quality ([EPLB] box "От переводчика: что на рисунке": per-GPU load of
  * the worked example, 86.5 .. 156, mean 129; exercise 2 of "что сделать
  * руками": compare max / mean between policies).  Per row r:

@@ -26,6 +26,7 @@ import torch
 __all__ = [
     "EplbError", "Plan", "count_loads", "window_accumulate", "rebalance", "redirect", "count_redirect",
     "plan_stats", "fold_loads", "initial_map", "plan_diff", "rebalance_window", "serve_step",
+    "serve_step_noalloc",
     "default_slots", "lib_path", "load_library", "STATUS",
 ]
 
@@ -89,6 +90,8 @@ def load_library():
         "eplb_plan_diff": ([p, p, i64, i32, i32, i32, p, p, p, p], i32),
         "eplb_serve_step": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, i64, i64, i64,
                              i32, i32, i32, i32, p, p, p, p, p, p, p, p], i32),
+        "eplb_serve_step_noalloc": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, i64, i64,
+                                     i64, i32, i32, i32, i32, p, p, p, p, p, p, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -342,6 +345,38 @@ def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, nex
             num_gpus, _ptr(loads_out), _ptr(next_plan.phy2log), _ptr(next_plan.phyrank),
             _ptr(next_plan.logcnt), _ptr(next_plan.log2phy), _ptr(layer_done), _ptr(status),
             _stream(idx.device)), "eplb_serve_step")
+    return out
+
+
+def serve_step_noalloc(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int,
+                       next_plan: Plan, num_groups: int, num_nodes: int, num_gpus: int,
+                       zero_slot: int = -1, token_offset: int = 0,
+                       out: Optional[torch.Tensor] = None,
+                       loads_out: Optional[torch.Tensor] = None,
+                       bad: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """serve_step with the library's own per-layer counters (no work array;
+    calls must not overlap on one device).  ``out`` must be given or is
+    allocated here by torch, outside the call."""
+    _cuda(idx, torch.int32, "idx")
+    _cuda(ring, torch.int64, "ring")
+    if idx.dim() != 3 or ring.dim() != 3:
+        raise ValueError("idx [L, T, K] and ring [W, L, E] expected")
+    L, T, K = idx.shape
+    Wr, Lr, E = ring.shape
+    if Lr != L:
+        raise ValueError("ring and idx disagree on L")
+    P = next_plan.phy2log.shape[1]
+    X = plan.log2phy.shape[2]
+    if out is None:
+        out = torch.empty_like(idx)
+    with torch.cuda.device(idx.device):
+        _check(load_library().eplb_serve_step_noalloc(
+            _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
+            _ptr(out), _ptr(bad), _ptr(ring), Wr, slot, zero_slot, P, num_groups, num_nodes,
+            num_gpus, _ptr(loads_out), _ptr(next_plan.phy2log), _ptr(next_plan.phyrank),
+            _ptr(next_plan.logcnt), _ptr(next_plan.log2phy), _ptr(status),
+            _stream(idx.device)), "eplb_serve_step_noalloc")
     return out
 
 

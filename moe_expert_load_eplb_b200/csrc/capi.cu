@@ -10,7 +10,6 @@
 namespace eplb {
 namespace {
 
-constexpr int kMaxDevices = 64;
 std::once_flag g_once[kMaxDevices];
 DeviceInfo g_info[kMaxDevices];
 bool g_ok[kMaxDevices];
@@ -250,6 +249,28 @@ eplb_status eplb_serve_step(const int32_t *idx, int64_t L, int64_t T, int32_t K,
   return launch_serve(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot, zero_slot,
                       loads_out, sh, next_phy2log, next_phyrank, next_logcnt, next_log2phy,
                       layer_done, status, stream);
+}
+
+eplb_status eplb_serve_step_noalloc(const int32_t *idx, int64_t L, int64_t T, int32_t K,
+                                    int32_t E, const int32_t *log2phy, int32_t X,
+                                    const int32_t *logcnt, int64_t t0, int32_t *out,
+                                    unsigned long long *bad, int64_t *ring, int64_t W,
+                                    int64_t slot, int64_t zero_slot, int32_t P, int32_t G,
+                                    int32_t N, int32_t gpus, int64_t *loads_out,
+                                    int32_t *next_phy2log, int32_t *next_phyrank,
+                                    int32_t *next_logcnt, int32_t *next_log2phy, int32_t *status,
+                                    cudaStream_t stream) {
+  if (L > kStaticLayers) return EPLB_ERR_LIMIT;
+  if (L <= 0) {
+    return eplb_serve_step(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot,
+                           zero_slot, P, G, N, gpus, loads_out, next_phy2log, next_phyrank,
+                           next_logcnt, next_log2phy, nullptr, status, stream);
+  }
+  uint32_t *counters = static_layer_done();
+  if (counters == nullptr) return cuda_fail(cudaGetLastError());
+  return eplb_serve_step(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot,
+                         zero_slot, P, G, N, gpus, loads_out, next_phy2log, next_phyrank,
+                         next_logcnt, next_log2phy, counters, status, stream);
 }
 
 eplb_status eplb_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,

@@ -78,6 +78,13 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
                          int32_t *next_logcnt, int32_t *next_log2phy, uint32_t *layer_done,
                          int32_t *status, cudaStream_t stream);
 
+// Device address of the library-owned per-layer counters of
+// eplb_serve_step_noalloc (kStaticLayers of them) on the current device;
+// nullptr if it cannot be had.
+constexpr int64_t kStaticLayers = 4096;
+constexpr int kMaxDevices = 64;
+uint32_t *static_layer_done();
+
 eplb_status launch_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,
                               int64_t R, int32_t E, int32_t P, int32_t gpus, double *gpu_load,
                               double *stats, int32_t *status, cudaStream_t stream);

@@ -16,6 +16,8 @@
 // completing CTA fences again and reads the ring through L2 (ld.global.cg)
 // only after it has seen the final count, so it sums the whole layer.  It
 // resets the layer's counter for the next call.
+#include <mutex>
+
 #include "rebalance_row.cuh"
 #include "redirect_chunk.cuh"
 
@@ -99,6 +101,22 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
   void *args[] = {&a};
   err = launch_pdl(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
+}
+
+// Per-layer counters of eplb_serve_step_noalloc: one library-owned array per
+// device, zero when the module loads and left zero by every call.  Calls of
+// that entry point share it, so two of them must not be in flight at once on
+// one device.
+static __device__ __align__(256) uint32_t g_layer_done[kStaticLayers];
+
+uint32_t *static_layer_done() {
+  static std::once_flag once[kMaxDevices];
+  static void *addr[kMaxDevices];
+  static cudaError_t err[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(once[dev], [dev] { err[dev] = cudaGetSymbolAddress(&addr[dev], g_layer_done); });
+  return err[dev] == cudaSuccess ? static_cast<uint32_t *>(addr[dev]) : nullptr;
 }
 
 }  // namespace eplb
