@@ -254,7 +254,7 @@ def run_ours(args, rank: int, world: int, group):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     hbm_peak, peak_kind = _peaks()
 
-    def make(fused, single=True):
+    def make(fused, single=False):
         st = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=WINDOW, device=dev,
                       token_offset=rank * c.T, group=group, fused=fused, single_launch=single)
         st.fill_history(hist)

@@ -415,6 +415,12 @@ __device__ __forceinline__ bool rep_better(int64_t aw, int ac, int ai, int64_t b
 __device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
                                 const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
                                 int32_t *rrank) {
+  // Pair (k, d) -- candidate k's d-th extra replica, value w_k / d -- ranks
+  // after every pair of greater value, and after equal-valued pairs of a
+  // lower expert index (same expert: lower d).  Candidate k2 has D2 = R - k2
+  // pairs; those ahead of (k, d) are d2 < w_k2 * d / w_k, plus d2 equal to it
+  // when the quotient is exact and id2 < id: one quotient per k2 instead of
+  // D2 cross-multiplied compares.
   const int R = s.ppn - s.lpn, nc = num_cand(s);
   const int grid = nc * R;
   for (int t = threadIdx.x; t < s.N * grid; t += nthr()) {
@@ -425,15 +431,33 @@ __device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
     if (d > R - k) continue;
     const int64_t w = cand_w[n * nc + k];
     const int id = cand_i[n * nc + k];
-    int rank = 0;
+    int rank = d - 1;  // the same expert's earlier replicas
     for (int k2 = 0; k2 < nc; ++k2) {
+      if (k2 == k) continue;
       const int64_t w2 = cand_w[n * nc + k2];
       const int id2 = cand_i[n * nc + k2];
-      const bool lower = id2 < id, same = id2 == id;
-      for (int d2 = 1; d2 <= R - k2; ++d2) {
-        const int64_t lhs = w2 * d, rhs = w * d2;
-        rank += (lhs > rhs || (lhs == rhs && (lower || (same && d2 < d)))) ? 1 : 0;
+      const int D2 = R - k2;
+      int ahead;
+      if (w == 0) {  // every value is >= 0: ahead if larger, or equal with a lower index
+        ahead = (w2 > 0 || id2 < id) ? D2 : 0;
+      } else {
+        const int64_t A = w2 * d;  // < 2^51
+        if (A >= w * (D2 + 1)) {
+          ahead = D2;  // even d2 = D2 is strictly ahead
+        } else {
+          // q = floor(A / w) <= D2: a float estimate, then exact integer fix-up
+          int64_t q = static_cast<int64_t>(__fmul_rn(static_cast<float>(A),
+                                                     __frcp_rn(static_cast<float>(w))));
+          int64_t r = A - q * w;
+          if (r < 0) { --q; r += w; }
+          if (r < 0) { --q; r += w; }
+          if (r >= w) { ++q; r -= w; }
+          if (r >= w) { ++q; r -= w; }
+          ahead = static_cast<int>(r == 0 ? q - 1 + (id2 < id ? 1 : 0) : q);
+          ahead = min(max(ahead, 0), D2);
+        }
       }
+      rank += ahead;
     }
     if (rank < R) {
       p2m[n * s.ppn + s.lpn + rank] = id;
@@ -638,6 +662,11 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     return;
   }
 
+  if (table_in_smem(s)) {  // the log2phy table starts all -1 (filled while step 1 runs)
+    int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
+    for (int i = tid; i < s.E * s.X; i += nthr()) tbl[i] = -1;
+  }
+
   // ---- step 1: groups -> nodes ---------------------------------------------
   if (s.gpn == 1) {  // one group per node: the pages' identity short-cut
     for (int g = tid; g < s.G; g += nthr()) {
@@ -784,34 +813,38 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   __syncthreads();
 
   // ---- assembly: pphy = node*ppn + gpu*ppg + rank -------------------------
+  // phy2log / phyrank / logcnt go straight to global memory; log2phy is
+  // scattered into the shared table (filled with -1 before step 1), then
+  // copied out row-contiguously
+  const int EX = s.E * s.X;
+  int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
+  const bool in_smem = table_in_smem(s);
+  int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
+  bool slots = false;
   for (int t = tid; t < s.P; t += nthr()) {
     const int n = t / s.ppn;
     const int pphy = n * s.ppn + ipack[t] * s.ppg + irank[t];
-    outp[pphy] = mlog2log[n * s.lpn + p2m[t]];
-    outr[pphy] = rrank[t];
-  }
-  for (int m = tid; m < s.E; m += nthr()) lc[mlog2log[m]] = cnt[m];
-  __syncthreads();
-  for (int t = tid; t < s.P; t += nthr()) {
-    a.phy2log[row * s.P + t] = outp[t];
-    a.phyrank[row * s.P + t] = outr[t];
-  }
-  for (int e = tid; e < s.E; e += nthr()) a.logcnt[row * s.E + e] = lc[e];
-  const int EX = s.E * s.X;
-  int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
-  bool slots = false;
-  if (table_in_smem(s)) {
-    int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
-    for (int i = tid; i < EX; i += nthr()) tbl[i] = -1;
-    __syncthreads();
-    for (int t = tid; t < s.P; t += nthr()) {
-      const int k = outr[t];
+    const int e = mlog2log[n * s.lpn + p2m[t]];
+    const int k = rrank[t];
+    a.phy2log[row * s.P + pphy] = e;
+    a.phyrank[row * s.P + pphy] = k;
+    if (in_smem) {
       if (k < s.X)
-        tbl[outp[t] * s.X + k] = t;
+        tbl[e * s.X + k] = pphy;
       else
         slots = true;
+    } else {
+      outp[pphy] = e;
+      outr[pphy] = k;
     }
-    __syncthreads();
+  }
+  for (int m = tid; m < s.E; m += nthr()) {
+    const int e = mlog2log[m];
+    lc[e] = cnt[m];
+    a.logcnt[row * s.E + e] = cnt[m];
+  }
+  __syncthreads();
+  if (in_smem) {
     if (a.table_vec4) {
       const int4 *src = reinterpret_cast<const int4 *>(tbl);
       int4 *dst = reinterpret_cast<int4 *>(gl);
