@@ -5,10 +5,12 @@
 // CTA that completes a layer -- the last of the layer's chunks to bump the
 // layer's counter -- then computes that layer's next plan: the window sum
 // over the ring (S2) and rebalance_experts (S3/S4, rebalance_row), into the
-// buffers of the next plan.  Layers are laid out chunk by chunk in launch
-// order, so the early layers' plans are built while later layers are still
-// streaming, and the step ends about one row's rebalance after its last
-// chunk, with no grid-wide wait or second launch in between.
+// buffers of the next plan.  Blocks run chunk-major, so the layers complete
+// together in the last wave and their plans are built side by side in the
+// tail (one row's rebalance after the last chunk) with no grid-wide wait or
+// second launch in between; a layer-major order, which lets early layers
+// plan while later ones stream, measured slower -- the planning CTAs hold
+// SM slots the streaming chunks wait for.
 //
 // Ordering: the CTA's count atomics are ordered before its counter increment
 // by a CTA barrier and a device-scope fence in the incrementing thread (the
@@ -36,8 +38,12 @@ __global__ void __launch_bounds__(kThreads) serve_kernel(ServeArgs a) {
   __shared__ int last;
   pdl_trigger();
   pdl_wait();
-  const int64_t cta = blockIdx.x;
-  const int64_t layer = cta / a.r.chunks;
+  // blocks run chunk-major (block b: layer b mod L, chunk b div L), so every
+  // layer is completed in the last wave and the layers' plans are built
+  // together in the tail instead of holding slots the streaming chunks need
+  const int64_t L = gridDim.x / a.r.chunks;
+  const int64_t layer = blockIdx.x % L;
+  const int64_t cta = layer * a.r.chunks + blockIdx.x / L;
   redirect_chunk<kVecToken, true>(a.r, smem, cta);
   __syncthreads();
   if (threadIdx.x == 0) {
