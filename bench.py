@@ -366,35 +366,66 @@ def _finish(out, args, step, idx, hist, flush, group, dev, rank, world):
             raise RuntimeError(f"device status {code} in {where}")
 
     # ---- e2e: the serving step through the public API with host buffers --
+    # Every step copies its indices from pinned host memory and reads back
+    # the redirected indices and the new plan.  Copies run on their own
+    # streams, double-buffered, so step i's upload, step i-1's compute and
+    # step i-2's download overlap (the two copy directions use separate copy
+    # engines); the timed region runs from the first upload to the last
+    # download.  No L2 flush: each step's fresh 243 MB of indices in and out
+    # exceed the L2.
     if not args.no_e2e:
         Ke = max(5, min(K, 50))
         idx_host = idx.cpu().pin_memory()
-        out_host = torch.empty(step.out.shape, dtype=torch.int32).pin_memory()
-        plan_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.plan]
-        idx_dev = torch.empty_like(idx)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(Ke)]
+        out_host = [torch.empty(step.out.shape, dtype=torch.int32).pin_memory() for _ in range(2)]
+        plan_host = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.plan]
+                     for _ in range(2)]
+        idx_dev = [torch.empty_like(idx) for _ in range(2)]
+        out_dev = [step.out, torch.empty_like(step.out)]
+        compute = torch.cuda.current_stream(dev)
+        up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = lambda: torch.cuda.Event()
+        uploaded = [ev() for _ in range(Ke)]
+        computed = [ev() for _ in range(Ke)]
+        downloaded = [ev() for _ in range(Ke)]
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
         if group is not None:
             torch.distributed.barrier(group=group)
         torch.cuda.synchronize()
+        t_start.record(up)
         for i in range(Ke):
-            flush.fill_(i & 0xff)
-            ev[i][0].record()
-            idx_dev.copy_(idx_host, non_blocking=True)
-            step(idx_dev)
-            out_host.copy_(step.out, non_blocking=True)
-            for h, d in zip(plan_host, step.plan):
-                h.copy_(d, non_blocking=True)
-            ev[i][1].record()
+            b_ = i % 2
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(computed[i - 2])  # idx_dev[b_] no longer read
+                idx_dev[b_].copy_(idx_host, non_blocking=True)
+                uploaded[i].record(up)
+            compute.wait_event(uploaded[i])
+            if i >= 2:
+                compute.wait_event(downloaded[i - 2])  # out_dev[b_] and the plan buffer read back
+            step.out = out_dev[b_]
+            step(idx_dev[b_])
+            computed[i].record(compute)
+            with torch.cuda.stream(down):
+                down.wait_event(computed[i])
+                out_host[b_].copy_(out_dev[b_], non_blocking=True)
+                for h, d in zip(plan_host[b_], step.plan):
+                    h.copy_(d, non_blocking=True)
+                downloaded[i].record(down)
+        t_end.record(down)
+        torch.cuda.synchronize()
+        step.out = out_dev[0]
         check(step, "e2e steps")
-        e2e_ms = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], dtype=torch.float64, device=dev)
+        e2e_ms = torch.tensor([t_start.elapsed_time(t_end)], dtype=torch.float64, device=dev)
         if group is not None:
             torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX, group=group)
         e2e_ms = float(e2e_ms.item())
         out["e2e"] = {"value": round(c.L * Ke / (e2e_ms / 1e3), 1), "unit": UNIT,
                       "h2d_bytes_per_step": idx.numel() * 4,
-                      "d2h_bytes_per_step": out_host.numel() * 4 + sum(t.numel() * 4 for t in plan_host),
-                      "steps": Ke, "ms_per_step": round(e2e_ms / Ke, 4)}
+                      "d2h_bytes_per_step": out_host[0].numel() * 4 + sum(t.numel() * 4 for t in plan_host[0]),
+                      "steps": Ke, "ms_per_step": round(e2e_ms / Ke, 4),
+                      "copies": "pinned host buffers, upload / compute / download on three streams, "
+                                "double-buffered"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(idx.cpu().numpy(), hist.cpu().numpy(), args.cpu_seconds)
