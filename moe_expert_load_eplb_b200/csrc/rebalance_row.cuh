@@ -228,10 +228,38 @@ __device__ void rank_pass(const K *key, int stride, int nseg, int n, int tps, Em
   }
 }
 
+// Same ranks with two threads per key when a segment has at least twice as
+// many threads as keys: each compares the key with half the segment, and the
+// pair adds its counts with one shuffle (the passes are warp-uniform).
+template <typename K, typename Emit>
+__device__ void rank_pass_split(const K *key, int stride, int nseg, int n, int tps, Emit &emit) {
+  const int segs_per_pass = nthr() / tps;
+  const int sub = threadIdx.x % tps;
+  const int j = sub >> 1, half = sub & 1;
+  const int h = (n + 1) >> 1;
+  const int i0 = half * h, i1 = min(n, i0 + h);
+  for (int g0 = 0; g0 < nseg; g0 += segs_per_pass) {
+    const int gl = static_cast<int>(threadIdx.x) / tps;
+    const int g = g0 + gl;
+    const bool live = gl < segs_per_pass && g < nseg && j < n;
+    const K *seg = key + (live ? g : 0) * stride;
+    const K me = live ? seg[j] : K(0);
+    int r = 0;
+    if (live) {
+#pragma unroll 4
+      for (int i = i0; i < i1; ++i) r += seg[i] > me ? 1 : 0;
+    }
+    r += __shfl_xor_sync(0xffffffffu, r, 1);
+    if (live && half == 0) emit(g, j, r, me);
+  }
+}
+
 template <typename K, typename Emit>
 __device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit emit) {
   const int tps = nseg >= nthr() ? 1 : nthr() / nseg;
-  if (n <= tps)
+  if (2 * n <= tps && tps % 32 == 0)
+    rank_pass_split<K>(key, stride, nseg, n, tps, emit);
+  else if (n <= tps)
     rank_pass<1, K>(key, stride, nseg, n, tps, emit);
   else if (n <= 2 * tps)
     rank_pass<2, K>(key, stride, nseg, n, tps, emit);
