@@ -47,7 +47,7 @@ typedef enum eplb_status {
                                  a logcnt outside [1, X] given to redirect */
   EPLB_ERR_SLOTS = 5,         /* an expert got more replicas than log2phy slots X */
   EPLB_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed */
-  EPLB_ERR_TIMEOUT = 7,       /* an in-kernel wait gave up (bounded, ~2 s) */
+  EPLB_ERR_TIMEOUT = 7,       /* reserved: an in-kernel wait gave up (no current kernel waits) */
   EPLB_ERR_ALIGN = 8,         /* a pointer lacks the alignment stated below */
   EPLB_ERR_LIMIT = 9          /* a size beyond this build's stated limits */
 } eplb_status;
@@ -71,7 +71,8 @@ int32_t eplb_abi_version(void);
  *          are skipped and their number is added to *bad.
  * counts   device int64 [L, E]; overwritten (accumulate == 0) or added to.
  * bad      device uint64 word, nullable; added to, never cleared.
- * status   device int32 word, nullable (EPLB_ERR_TIMEOUT only).
+ * status   device int32 word, nullable; counting has no data-dependent error,
+ *          so nothing is written to it (kept for a uniform signature).
  * Limits:  1 <= E <= 1024, K >= 1, L, T >= 0.
  * Integer atomics make the result independent of scheduling.
  */
@@ -92,6 +93,7 @@ eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K
  * snaps    device int64 [S - s_first, L, E]; must not overlap steps.
  * W >= 1 (W >= S gives running totals); 0 <= s_first < S.
  * Sums are exact; wrap-around of int64 is the caller's concern.
+ * status   nullable; nothing is written to it (no data-dependent error).
  * With a ring buffer of the last W per-step counts, s_first = S - 1 = W - 1
  * returns the current window sum (row order does not change a full sum).
  */
