@@ -73,7 +73,7 @@ int32_t eplb_abi_version(void);
  * bad      device uint64 word, nullable; added to, never cleared.
  * status   device int32 word, nullable; counting has no data-dependent error,
  *          so nothing is written to it (kept for a uniform signature).
- * Limits:  1 <= E <= 1024, K >= 1, L, T >= 0.
+ * Limits:  1 <= E <= 1024, K >= 1, 0 <= L < 2^31, T >= 0, T * K < 2^31.
  * Integer atomics make the result independent of scheduling.
  */
 eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K,
@@ -167,7 +167,7 @@ eplb_status eplb_rebalance_window(int64_t *ring, int64_t W, int64_t zero_slot, i
  *          An index outside [0, E) gives -1 and is added to *bad; a logcnt
  *          outside [1, X] gives -1 and *status = EPLB_ERR_RANGE.
  * log2phy  device int32 [L, E, X]; logcnt device int32 [L, E].
- * Limits:  1 <= E <= 1024, 1 <= X, E * X <= 32768, T * K < 2^31,
+ * Limits:  1 <= E <= 1024, 1 <= X, E * X <= 32768, T * K < 2^31, L < 2^31,
  *          0 <= t0, t0 + T < 2^31.
  */
 eplb_status eplb_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,

@@ -151,6 +151,7 @@ eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer,
   const int64_t waves = std::min(std::max<int64_t>(total / (kChunk * slots), 1), kMaxWaves);
   a.chunks = std::max<int64_t>(1, std::min(waves * slots / L, (per_layer + 4095) / 4096));
   const int64_t grid = L * a.chunks;
+  if (grid > 0x7fffffffLL) return EPLB_ERR_LIMIT;  // one block per layer chunk
   void *args[] = {&a};
   err = launch_pdl(reinterpret_cast<const void *>(count_loads_kernel), dim3(static_cast<unsigned>(grid)),
                    dim3(kThreads), smem, stream, args);

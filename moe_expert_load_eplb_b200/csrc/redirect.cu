@@ -45,6 +45,7 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
   per_sm = std::max(1, std::min(per_sm, 4));
   a.chunks = redirect_chunks(L, a.per_layer, static_cast<int64_t>(di.sms) * per_sm);
   const int64_t grid = L * a.chunks;
+  if (grid > 0x7fffffffLL) return EPLB_ERR_LIMIT;  // one block per layer chunk
   void *args[] = {&a};
   err = launch_pdl(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), sp.bytes, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
