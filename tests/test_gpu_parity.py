@@ -494,6 +494,42 @@ def test_pipeline_serving_order_c2(c2_idx, single):
         assert int(step.layer_done.abs().sum().item()) == 0
 
 
+def test_pipeline_serving_with_an_nccl_group_of_one(c1_idx):
+    """The multi-rank serving step (count+redirect, NCCL all-reduce of the
+    counts, window + rebalance) on a one-rank NCCL group: same plans and
+    redirects as the oracle."""
+    import socket
+    import torch.distributed as dist
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device(DEV))
+    try:
+        group = dist.new_group([0])
+        c = W.CONFIGS[1]
+        W_ = 3
+        hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, 1, device=DEV)
+        step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV,
+                        group=group, token_offset=77)
+        assert step.launches_per_step == 2 and not step.single
+        step.fill_history(hist)
+        ring = np.concatenate([_np(hist), np.zeros((1, c.L, c.E), np.int64)], axis=0)
+        plan_ref = _oracle_plan_from_ring(ring, c, step.X)
+        for s_i, idx in enumerate([c1_idx, c1_idx.flip(1).contiguous()]):
+            used, out = step(idx)
+            torch.cuda.synchronize()
+            assert int(step.status.item()) == 0
+            red, _ = oracle.redirect(_np(idx), plan_ref[3], plan_ref[2], 77)
+            assert np.array_equal(_np(out), red)
+            ring[(W_ - 1 + s_i) % W_] = oracle.count_loads(_np(idx), c.E)[0]
+            plan_ref = _oracle_plan_from_ring(ring, c, step.X)
+            _assert_plan_equal(step.plan, plan_ref)
+    finally:
+        dist.destroy_process_group()
+
+
 # ------------------------------------------------------- one-launch serve step --
 
 def _dev(a):
