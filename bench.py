@@ -153,6 +153,9 @@ def _kernel_sha(name: str) -> str:
     return h.hexdigest()[:16]
 
 
+# B200 HBM3e datasheet bandwidth (about 8 TB/s), reported beside the measured peak
+DATASHEET_HBM_GBS = 8000.0
+
 # the serving-step kernel's code: its file and the two headers it inlines
 SERVE_SOURCES = "serve.cu+redirect_chunk.cuh+rebalance_row.cuh"
 
@@ -297,7 +300,8 @@ def run_ours(args, rank: int, world: int, group):
                                           "count_redirect_dsv3_prefill.md", 1.0)
     roof = {"kernel": "count_redirect", "bound": "hbm", "achieved": stages["count"]["gbs"],
             "peak": hbm_peak, "peak_kind": peak_kind, "unit": "GB/s",
-            "frac": stages["count"]["frac_hbm"], "traffic": stages["count"]["traffic"]}
+            "frac": stages["count"]["frac_hbm"], "traffic": stages["count"]["traffic"],
+            "frac_of_datasheet": round(stages["count"]["gbs"] / DATASHEET_HBM_GBS, 4)}
     order = ("serving: count+redirect with the plan in force (fused, one pass over the indices) "
              + ("-> all-reduce of the counts " if world > 1 else "")
              + "-> window sum + rebalance (fused) -> next plan")
