@@ -338,6 +338,56 @@ def run_ours(args, rank: int, world: int, group):
             "traffic": _traffic(SERVE_SOURCES, "serve_step_dsv3_prefill.md", 1.0)}
         del one
 
+    # ---- decode-sized step: eager calls vs CUDA-graph replay -----------------
+    # At 8,192 tokens per layer the GPU step is short, so the host's enqueue
+    # time per step matters; a captured step is one graph launch.
+    if world == 1 and not args.no_fresh:
+        from moe_expert_load_eplb_b200.pipeline import EplbStep, StepGraphs
+        Td = 8192
+        idx_d = W.routed_indices(2, device=dev, T=Td)
+        hist_d = W.histogram_steps(WINDOW - 1, c.L, c.E, Td * c.K, 2, device=dev)
+
+        def make_d():
+            st = EplbStep(c.L, Td, c.K, c.E, c.P, c.G, c.N, c.gpus, window=WINDOW, device=dev)
+            st.fill_history(hist_d)
+            return st
+
+        eager_d = make_d()
+        graphed_d = make_d()
+        buf_d = idx_d.clone()
+        sg = StepGraphs(graphed_d, buf_d)
+
+        def run_d(fn, n):
+            for i in range(3):
+                flush.fill_(i & 0xff)
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(n)]
+            host = 0.0
+            torch.cuda.synchronize()
+            for i in range(n):
+                flush.fill_(i & 0xff)  # keeps the GPU busy while the host enqueues
+                ev[i][0].record()
+                h0 = time.perf_counter()
+                fn()
+                host += time.perf_counter() - h0
+                ev[i][1].record()
+            torch.cuda.synchronize()
+            return (sum(a.elapsed_time(b) for a, b in ev) / n, host / n * 1e6)
+
+        Kd = max(3, min(K, 500))
+        e_ms, e_host = run_d(lambda: eager_d(idx_d), Kd)
+        g_ms, g_host = run_d(sg, Kd)
+        check(eager_d, "decode eager steps")
+        check(graphed_d, "decode graph steps")
+        out["decode_8192_tokens"] = {
+            "steps": Kd, "l2": "flushed between steps (512 MB write)",
+            "eager": {"ms_per_step": round(e_ms, 5), "host_us_per_step": round(e_host, 1),
+                      "value": round(c.L / (e_ms / 1e3), 1)},
+            "graph_replay": {"ms_per_step": round(g_ms, 5), "host_us_per_step": round(g_host, 1),
+                             "value": round(c.L / (g_ms / 1e3), 1)}}
+        del eager_d, graphed_d, sg
+
     # ---- the same four stages in the fresh-plan order, for comparison -----
     if args.no_fresh:
         return _finish(out, args, step, idx, hist, flush, group, dev, rank, world)

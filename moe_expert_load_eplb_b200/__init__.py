@@ -121,8 +121,38 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device):
+    """The current stream of ``device`` as a raw handle."""
+    if _raw_stream is not None:
+        return ctypes.c_void_p(_raw_stream(device.index if device.index is not None
+                                           else torch.cuda.current_device()))
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+class _on_device:
+    """Makes ``device`` current for the call; free when it already is."""
+
+    __slots__ = ("index", "prev")
+
+    def __init__(self, device: torch.device):
+        self.index = device.index
+        self.prev = None
+
+    def __enter__(self):
+        if self.index is not None:
+            cur = torch.cuda.current_device()
+            if cur != self.index:
+                self.prev = cur
+                torch.cuda.set_device(self.index)
+        return self
+
+    def __exit__(self, *exc):
+        if self.prev is not None:
+            torch.cuda.set_device(self.prev)
+        return False
 
 
 def count_loads(idx: torch.Tensor, num_experts: int, counts: Optional[torch.Tensor] = None,
@@ -139,7 +169,7 @@ def count_loads(idx: torch.Tensor, num_experts: int, counts: Optional[torch.Tens
     _cuda(counts, torch.int64, "counts")
     if tuple(counts.shape) != (L, num_experts):
         raise ValueError("counts must be [L, E]")
-    with torch.cuda.device(idx.device):
+    with _on_device(idx.device):
         _check(load_library().eplb_count_loads(
             _ptr(idx), L, T, K, num_experts, _ptr(counts), int(bool(accumulate)),
             _ptr(bad), _ptr(status), _stream(idx.device)), "eplb_count_loads")
@@ -159,7 +189,7 @@ def window_accumulate(steps: torch.Tensor, window: int, s_first: int = 0,
     _cuda(out, torch.int64, "out")
     if tuple(out.shape) != (S - s_first, L, E):
         raise ValueError("out must be [S - s_first, L, E]")
-    with torch.cuda.device(steps.device):
+    with _on_device(steps.device):
         _check(load_library().eplb_window_accumulate(
             _ptr(steps), S, L, E, window, s_first, _ptr(out), _ptr(status),
             _stream(steps.device)), "eplb_window_accumulate")
@@ -194,7 +224,7 @@ def rebalance(loads: torch.Tensor, num_replicas: int, num_groups: int, num_nodes
         _cuda(t, torch.int32, name)
         if tuple(t.shape) != shape:
             raise ValueError(f"{name} must be {shape}")
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(load_library().eplb_rebalance(
             _ptr(loads), R, E, P, num_groups, num_nodes, num_gpus, X,
             _ptr(out.phy2log), _ptr(out.phyrank), _ptr(out.logcnt), _ptr(out.log2phy),
@@ -230,7 +260,7 @@ def rebalance_window(ring: torch.Tensor, num_replicas: int, num_groups: int, num
         _cuda(loads_out, torch.int64, "loads_out")
         if tuple(loads_out.shape) not in ((R, E), (1, R, E)):
             raise ValueError("loads_out must be [R, E]")
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(load_library().eplb_rebalance_window(
             _ptr(ring), Wr, zero_slot, R, E, P, num_groups, num_nodes, num_gpus, X, _ptr(loads_out),
             _ptr(out.phy2log), _ptr(out.phyrank), _ptr(out.logcnt), _ptr(out.log2phy),
@@ -256,7 +286,7 @@ def redirect(idx: torch.Tensor, log2phy: torch.Tensor, logcnt: torch.Tensor, tok
     _cuda(out, torch.int32, "out")
     if out.shape != idx.shape:
         raise ValueError("out must match idx")
-    with torch.cuda.device(idx.device):
+    with _on_device(idx.device):
         _check(load_library().eplb_redirect(
             _ptr(idx), L, T, K, E, _ptr(log2phy), X, _ptr(logcnt), int(token_offset),
             _ptr(out), _ptr(bad), _ptr(status), _stream(idx.device)), "eplb_redirect")
@@ -290,7 +320,7 @@ def count_redirect(idx: torch.Tensor, num_experts: int, log2phy: torch.Tensor, l
     _cuda(out, torch.int32, "out")
     if out.shape != idx.shape:
         raise ValueError("out must match idx")
-    with torch.cuda.device(idx.device):
+    with _on_device(idx.device):
         _check(load_library().eplb_count_redirect(
             _ptr(idx), L, T, K, E, _ptr(counts), int(bool(accumulate)), _ptr(log2phy), X,
             _ptr(logcnt), int(token_offset), _ptr(out), _ptr(bad), _ptr(status),
@@ -338,7 +368,7 @@ def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, nex
         _cuda(loads_out, torch.int64, "loads_out")
         if loads_out.numel() != L * E:
             raise ValueError("loads_out must be [L, E]")
-    with torch.cuda.device(idx.device):
+    with _on_device(idx.device):
         _check(load_library().eplb_serve_step(
             _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
             _ptr(out), _ptr(bad), _ptr(ring), Wr, slot, zero_slot, P, num_groups, num_nodes,
@@ -370,7 +400,7 @@ def serve_step_noalloc(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: 
     X = plan.log2phy.shape[2]
     if out is None:
         out = torch.empty_like(idx)
-    with torch.cuda.device(idx.device):
+    with _on_device(idx.device):
         _check(load_library().eplb_serve_step_noalloc(
             _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
             _ptr(out), _ptr(bad), _ptr(ring), Wr, slot, zero_slot, P, num_groups, num_nodes,
@@ -391,7 +421,7 @@ def plan_stats(loads: torch.Tensor, phy2log: torch.Tensor, logcnt: torch.Tensor,
     P = phy2log.shape[1]
     gl = torch.empty((R, num_gpus), dtype=torch.float64, device=loads.device)
     st = torch.empty((R, 4), dtype=torch.float64, device=loads.device)
-    with torch.cuda.device(loads.device):
+    with _on_device(loads.device):
         _check(load_library().eplb_plan_stats(
             _ptr(loads), _ptr(phy2log), _ptr(logcnt), R, E, P, num_gpus, _ptr(gl), _ptr(st),
             _ptr(status), _stream(loads.device)), "eplb_plan_stats")
@@ -405,7 +435,7 @@ def fold_loads(phys: torch.Tensor, phy2log: torch.Tensor, num_logical: int,
     _cuda(phy2log, torch.int32, "phy2log")
     R, P = phys.shape
     out = torch.empty((R, num_logical), dtype=torch.int64, device=phys.device)
-    with torch.cuda.device(phys.device):
+    with _on_device(phys.device):
         _check(load_library().eplb_fold_loads(
             _ptr(phys), _ptr(phy2log), R, num_logical, P, _ptr(out), _ptr(status),
             _stream(phys.device)), "eplb_fold_loads")
@@ -417,7 +447,7 @@ def initial_map(rows: int, num_logical: int, num_replicas: int, device="cuda"):
     p2l = torch.empty((rows, num_replicas), dtype=torch.int32, device=device)
     prk = torch.empty((rows, num_replicas), dtype=torch.int32, device=device)
     dev = p2l.device
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         _check(load_library().eplb_initial_map(rows, num_logical, num_replicas, _ptr(p2l), _ptr(prk),
                                                _stream(dev)), "eplb_initial_map")
     return p2l, prk
@@ -434,7 +464,7 @@ def plan_diff(old_phy2log: torch.Tensor, new_phy2log: torch.Tensor, num_logical:
     R, P = new_phy2log.shape
     src = torch.empty((R, P), dtype=torch.int32, device=new_phy2log.device)
     moves = torch.empty((R,), dtype=torch.int32, device=new_phy2log.device)
-    with torch.cuda.device(new_phy2log.device):
+    with _on_device(new_phy2log.device):
         _check(load_library().eplb_plan_diff(
             _ptr(old_phy2log), _ptr(new_phy2log), R, num_logical, P, num_gpus, _ptr(src),
             _ptr(moves), _ptr(status), _stream(new_phy2log.device)), "eplb_plan_diff")

@@ -3,7 +3,10 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
+#include <utility>
 
 #include "internal.h"
 
@@ -34,6 +37,41 @@ int next_pow2(int v) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
+
+namespace {
+std::mutex g_kernel_mu;
+std::map<std::pair<int, const void *>, size_t> g_smem_set;                 // (device, fn) -> bytes
+std::map<std::tuple<int, const void *, int, size_t>, int> g_blocks_per_sm;  // occupancy
+}  // namespace
+
+eplb_status prepare_kernel(const void *fn, int threads, size_t smem, int *per_sm) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return cuda_fail(err);
+  std::lock_guard<std::mutex> lock(g_kernel_mu);
+  const auto key = std::make_pair(dev, fn);
+  const auto it = g_smem_set.find(key);
+  if (it == g_smem_set.end() || it->second < smem) {
+    err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return cuda_fail(err);
+    g_smem_set[key] = smem;
+  }
+  if (per_sm != nullptr) {
+    const auto okey = std::make_tuple(dev, fn, threads, smem);
+    const auto oit = g_blocks_per_sm.find(okey);
+    if (oit != g_blocks_per_sm.end()) {
+      *per_sm = oit->second;
+    } else {
+      int n = 0;
+      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem);
+      if (err != cudaSuccess) return cuda_fail(err);
+      g_blocks_per_sm[okey] = n;
+      *per_sm = n;
+    }
+  }
+  return EPLB_OK;
+}
 
 bool device_info(DeviceInfo *out) {
   int dev = 0;

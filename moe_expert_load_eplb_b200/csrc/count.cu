@@ -131,13 +131,10 @@ eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer,
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
   const size_t smem = static_cast<size_t>(E + 1) * 32 * sizeof(uint32_t);
   if (smem > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
-  cudaError_t err = cudaFuncSetAttribute(count_loads_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return cuda_fail(err);
   int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, count_loads_kernel, kThreads, smem);
-  if (err != cudaSuccess) return cuda_fail(err);
+  const eplb_status st = prepare_kernel(reinterpret_cast<const void *>(count_loads_kernel),
+                                        kThreads, smem, &per_sm);
+  if (st != EPLB_OK) return st;
   per_sm = std::max(1, std::min(per_sm, 4));
   CountArgs a;
   a.idx = idx;
@@ -153,7 +150,7 @@ eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer,
   const int64_t grid = L * a.chunks;
   if (grid > 0x7fffffffLL) return EPLB_ERR_LIMIT;  // one block per layer chunk
   void *args[] = {&a};
-  err = launch_pdl(reinterpret_cast<const void *>(count_loads_kernel), dim3(static_cast<unsigned>(grid)),
+  const cudaError_t err = launch_pdl(reinterpret_cast<const void *>(count_loads_kernel), dim3(static_cast<unsigned>(grid)),
                    dim3(kThreads), smem, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }

@@ -9,6 +9,13 @@
 
 namespace eplb {
 
+// Raises fn's dynamic shared-memory limit to `smem` bytes if it is lower
+// (once per device and size) and, with per_sm, returns how many
+// `threads`-thread CTAs of fn fit on one SM with that much shared memory
+// (cached per device, kernel, CTA size and bytes): no per-launch driver
+// queries.
+eplb_status prepare_kernel(const void *fn, int threads, size_t smem, int *per_sm);
+
 // Launches fn with programmatic stream serialisation (see pdl_trigger /
 // pdl_wait in common.cuh); args as for cudaLaunchKernel.
 inline cudaError_t launch_pdl(const void *fn, dim3 grid, dim3 block, size_t smem,

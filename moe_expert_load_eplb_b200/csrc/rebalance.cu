@@ -23,10 +23,9 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
   const Layout lay(sh);
   if (lay.total > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
-  cudaError_t err = cudaFuncSetAttribute(rebalance_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(lay.total));
-  if (err != cudaSuccess) return cuda_fail(err);
+  const eplb_status pst =
+      prepare_kernel(reinterpret_cast<const void *>(rebalance_kernel), kMaxThreads, lay.total, nullptr);
+  if (pst != EPLB_OK) return pst;
   RbArgs a;
   a.ring = ring;
   a.ring_w = ring_w;
@@ -44,7 +43,7 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
                  (reinterpret_cast<uintptr_t>(log2phy) % 16 == 0);
   const int threads = R <= 2 * static_cast<int64_t>(di.sms) ? kFewRowThreads : kManyRowThreads;
   void *args[] = {&a};
-  err = launch_pdl(reinterpret_cast<const void *>(rebalance_kernel), dim3(static_cast<unsigned>(R)),
+  const cudaError_t err = launch_pdl(reinterpret_cast<const void *>(rebalance_kernel), dim3(static_cast<unsigned>(R)),
                    dim3(threads), lay.total, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }

@@ -36,18 +36,16 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
   else
     fn = vec_token ? reinterpret_cast<const void *>(redirect_kernel<true, false>)
                    : reinterpret_cast<const void *>(redirect_kernel<false, false>);
-  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sp.bytes));
-  if (err != cudaSuccess) return cuda_fail(err);
   int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, sp.bytes);
-  if (err != cudaSuccess) return cuda_fail(err);
+  const eplb_status pst = prepare_kernel(fn, kThreads, sp.bytes, &per_sm);
+  if (pst != EPLB_OK) return pst;
   per_sm = std::max(1, std::min(per_sm, 4));
   a.chunks = redirect_chunks(L, a.per_layer, static_cast<int64_t>(di.sms) * per_sm);
   const int64_t grid = L * a.chunks;
   if (grid > 0x7fffffffLL) return EPLB_ERR_LIMIT;  // one block per layer chunk
   void *args[] = {&a};
-  err = launch_pdl(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), sp.bytes, stream, args);
+  const cudaError_t err =
+      launch_pdl(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), sp.bytes, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

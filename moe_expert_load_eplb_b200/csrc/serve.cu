@@ -95,18 +95,16 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
   a.layer_done = layer_done;
   const void *fn = (K % 4) == 0 ? reinterpret_cast<const void *>(serve_kernel<true>)
                                 : reinterpret_cast<const void *>(serve_kernel<false>);
-  cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-  if (err != cudaSuccess) return cuda_fail(err);
   int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
-  if (err != cudaSuccess) return cuda_fail(err);
+  st = prepare_kernel(fn, kThreads, smem, &per_sm);
+  if (st != EPLB_OK) return st;
   per_sm = std::max(1, std::min(per_sm, 4));
   a.r.chunks = redirect_chunks(L, a.r.per_layer, static_cast<int64_t>(di.sms) * per_sm);
   const int64_t grid = L * a.r.chunks;
   if (grid > 0x7fffffffLL) return EPLB_ERR_LIMIT;  // one block per layer chunk
   void *args[] = {&a};
-  err = launch_pdl(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, args);
+  const cudaError_t err =
+      launch_pdl(fn, dim3(static_cast<unsigned>(grid)), dim3(kThreads), smem, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

@@ -160,3 +160,55 @@ class EplbStep:
             self.cur = 1 - self.cur
             return used, self.out
         return nxt, self.out
+
+
+class StepGraphs:
+    """Replays an EplbStep's steps as CUDA graphs.
+
+    A step's launches depend on its phase only: the ring slot it counts into
+    (step mod W) and which of the two plan buffers is in force (step mod 2).
+    ``lcm(W, 2)`` consecutive steps are captured once, each as one graph that
+    reads its indices from the fixed buffer ``idx``; ``step_graphs()`` then
+    replays the graph of the current phase, so a step costs one graph launch
+    on the host instead of one call per kernel.  The captured steps are not
+    executed by the capture; the EplbStep's bookkeeping advances only on
+    replay.  One GPU (no process group), as the one-process serving step.
+    """
+
+    def __init__(self, step: "EplbStep", idx: torch.Tensor):
+        if not step.primed or step.group is not None:
+            raise ValueError("capture needs a primed EplbStep without a process group")
+        if tuple(idx.shape) != (step.L, step.T, step.K) or idx.dtype != torch.int32:
+            raise ValueError("idx must be the step's int32 [L, T, K] input buffer")
+        import math
+        self.step = step
+        self.idx = idx
+        self.period = math.lcm(step.W, 2)
+        self.first = step.steps_done
+        dev = step.device
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        saved = (step.steps_done, step.cur)
+        self.graphs = []
+        with torch.cuda.stream(side):
+            for _ in range(self.period):
+                g = torch.cuda.CUDAGraph()
+                # relaxed: the library's launch set-up (function attributes,
+                # occupancy queries) is not stream work but is still allowed
+                with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+                    step(idx)
+                self.graphs.append(g)
+        torch.cuda.current_stream(dev).wait_stream(side)
+        step.steps_done, step.cur = saved  # capturing ran nothing
+
+    def __call__(self):
+        """Runs one step on the current contents of ``idx``; returns (plan used,
+        redirected indices) like EplbStep.__call__."""
+        st = self.step
+        k = (st.steps_done - self.first) % self.period
+        used = st.plans[st.cur]
+        self.graphs[k].replay()
+        st.steps_done += 1
+        if st.fused:
+            st.cur = 1 - st.cur
+        return used, st.out

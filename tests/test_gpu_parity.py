@@ -530,6 +530,37 @@ def test_pipeline_serving_with_an_nccl_group_of_one(c1_idx):
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("fused,single", [(True, False), (True, True), (False, False)])
+def test_step_graphs_replay_matches_eager(c1_idx, fused, single):
+    """CUDA-graph replay of the step (one graph per phase of the ring slot and
+    plan buffer) gives exactly the eager steps' outputs, plans and ring."""
+    from moe_expert_load_eplb_b200.pipeline import EplbStep, StepGraphs
+    c = W.CONFIGS[1]
+    hist = W.histogram_steps(2, c.L, c.E, c.T * c.K, 1, device=DEV)
+    mk = lambda: EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=3, device=DEV,
+                          fused=fused, single_launch=single, token_offset=5)
+    eager, graphed = mk(), mk()
+    eager.fill_history(hist)
+    graphed.fill_history(hist)
+    buf = torch.empty_like(c1_idx)
+    sg = StepGraphs(graphed, buf)
+    assert sg.period == 6
+    batches = [c1_idx, c1_idx.flip(1), c1_idx.roll(7, dims=1), (c1_idx + 3) % c.E]
+    for k in range(9):
+        b = batches[k % len(batches)].contiguous()
+        buf.copy_(b)
+        used_g, out_g = sg()
+        used_e, out_e = eager(b)
+        torch.cuda.synchronize()
+        assert torch.equal(out_g, out_e), f"step {k}: redirected indices"
+        for a_, b_ in zip(used_g, used_e):
+            assert torch.equal(a_, b_), f"step {k}: plan used"
+        for a_, b_ in zip(graphed.plan, eager.plan):
+            assert torch.equal(a_, b_), f"step {k}: new plan"
+        assert torch.equal(graphed.ring, eager.ring), f"step {k}: ring"
+    assert int(graphed.status.item()) == 0
+
+
 # ------------------------------------------------------- one-launch serve step --
 
 def _dev(a):
