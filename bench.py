@@ -482,7 +482,9 @@ def _finish(out, args, step, idx, hist, flush, group, dev, rank, world):
                                 "double-buffered"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(idx.cpu().numpy(), hist.cpu().numpy(), args.cpu_seconds)
+        idx_h, hist_h = idx.cpu().numpy(), hist.cpu().numpy()
+        out["cpu_baseline"] = cpu_baseline(idx_h, hist_h, args.cpu_seconds)
+        out["cpu_baseline_parallel"] = cpu_baseline_parallel(idx_h, hist_h, args.cpu_seconds)
     return out
 
 
@@ -523,6 +525,39 @@ def cpu_baseline(idx_h, hist_h, seconds: float):
     return {"value": round(CFG.L * n / el, 2), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} full serving steps (58 layers x 65,536 tokens x top-8: count and "
                       f"redirect, 16-step window, rebalance), single-thread plain C, {el:.1f} s"}
+
+
+def cpu_baseline_parallel(idx_h, hist_h, seconds: float):
+    """The same oracle step with its layers spread over the host cores:
+    ``python -m oracle.pool`` (worker processes that import only numpy and
+    the oracle) on inputs handed over in shared memory."""
+    import subprocess
+    from multiprocessing import shared_memory
+
+    import numpy as np
+    c = CFG
+    cores = min(len(os.sched_getaffinity(0)), c.L)
+    shm_i = shared_memory.SharedMemory(create=True, size=idx_h.nbytes)
+    shm_h = shared_memory.SharedMemory(create=True, size=hist_h.nbytes)
+    try:
+        np.ndarray(idx_h.shape, np.int32, buffer=shm_i.buf)[:] = idx_h
+        np.ndarray(hist_h.shape, np.int64, buffer=shm_h.buf)[:] = hist_h
+        spec = {"idx_name": shm_i.name, "idx_shape": list(idx_h.shape), "hist_name": shm_h.name,
+                "hist_shape": list(hist_h.shape), "P": c.P, "G": c.G, "N": c.N, "gpus": c.gpus,
+                "X": (c.P - c.E) // c.N + 1, "cores": cores, "seconds": seconds}
+        res = subprocess.run([sys.executable, "-m", "oracle.pool", json.dumps(spec)], cwd=ROOT,
+                             capture_output=True, text=True, timeout=seconds * 4 + 240)
+        if res.returncode != 0:
+            return {"unavailable": f"oracle pool failed: {res.stderr.strip()[-200:]}"}
+        r = json.loads(res.stdout.strip().splitlines()[-1])
+    finally:
+        shm_i.close()
+        shm_i.unlink()
+        shm_h.close()
+        shm_h.unlink()
+    return {"value": round(r["layers_per_s"], 2), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{r['steps']} full serving steps, the 58 layers spread over {cores} worker "
+                      f"processes (plain C oracle per layer), {r['seconds']:.1f} s"}
 
 
 def run_reference(args):
