@@ -57,7 +57,8 @@ def layer_step(layer: int) -> int:
 
 def main(argv=None):
     """``python -m oracle.pool '<json>'``: times the pool on inputs already in
-    shared memory and prints one JSON object (value in layers per second)."""
+    shared memory -- for ``seconds``, or ``steps`` steps after ``warmup`` --
+    and prints one JSON object (value in layers per second)."""
     import json
     import multiprocessing as mp
     import sys
@@ -70,12 +71,14 @@ def main(argv=None):
                             tuple(a["hist_shape"]), a["P"], a["G"], a["N"], a["gpus"],
                             a["X"])) as p:
         p.map(layer_step, range(L), chunksize=1)  # plans in force, libraries loaded
+        for _ in range(a.get("warmup", 0)):
+            p.map(layer_step, range(L), chunksize=1)
         n, t0 = 0, time.perf_counter()
         while True:
             p.map(layer_step, range(L), chunksize=1)
             n += 1
             el = time.perf_counter() - t0
-            if el >= a["seconds"]:
+            if ("steps" in a and n >= a["steps"]) or ("steps" not in a and el >= a["seconds"]):
                 break
     print(json.dumps({"steps": n, "seconds": el, "layers_per_s": L * n / el}), flush=True)
 
