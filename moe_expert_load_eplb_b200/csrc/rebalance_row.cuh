@@ -403,6 +403,38 @@ __device__ void pack_warp(const K *skey, int n, int m, int cap, K *pw, int32_t *
   }
 }
 
+// The greedy in closed form when every pack takes exactly two items
+// (n == 2m) and the m heaviest items all weigh more than zero.  Round 1:
+// item j (sorted, 0-based) finds packs 0..j-1 heavier than the empty ones,
+// so it opens pack j.  Round 2: no pack changes weight until it is full, so
+// the packs take their second item lightest first -- ascending (weight,
+// index) of their first item -- and pack p takes item m + pos(p).  One
+// thread per pack, no dependent chain.
+template <typename K>
+__device__ void pack_cap2(const K *skey_base, int stride, int nseg, int m, int32_t *ipack,
+                          int32_t *irank, int out_stride) {
+  const K imask = K(kIdxMask);
+  for (int t = threadIdx.x; t < nseg * m; t += nthr()) {
+    const int g = t / m;
+    const int p = t - g * m;
+    const K *skey = skey_base + g * stride;
+    const K kp = skey[p];
+    const K wp = kp >> kIdxBits;
+    int item = static_cast<int>(imask - (kp & imask));
+    ipack[g * out_stride + item] = p;
+    irank[g * out_stride + item] = 0;
+    int pos = 0;
+    for (int q = 0; q < m; ++q) {
+      const K wq = skey[q] >> kIdxBits;
+      pos += (wq < wp || (wq == wp && q < p)) ? 1 : 0;
+    }
+    const K k2 = skey[m + pos];
+    item = static_cast<int>(imask - (k2 & imask));
+    ipack[g * out_stride + item] = p;
+    irank[g * out_stride + item] = 1;
+  }
+}
+
 // Packs nseg segments (segment g: n sorted keys at skey + g * stride, results
 // at ipack/irank + g * out_stride) into m packs of cap items each.  Called by
 // every thread of the CTA (the lane-parallel variant needs whole warps).
@@ -410,6 +442,17 @@ template <typename K>
 __device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
                               int32_t *pc, int32_t *ipack, int32_t *irank, int out_stride) {
   if (n <= 0) return;
+  // closed form only for long chains: on a few packs (8 groups onto 4 nodes)
+  // the vote cost more than the short greedy it replaces (measured)
+  if (cap == 2 && n == 2 * m && m >= 16) {  // uniform: every segment has the same shape
+    bool ok = true;
+    for (int g = threadIdx.x; g < nseg; g += nthr())
+      ok &= (skey[g * stride + m - 1] >> kIdxBits) != K(0);
+    if (__syncthreads_and(ok)) {
+      pack_cap2<K>(skey, stride, nseg, m, ipack, irank, out_stride);
+      return;
+    }
+  }
   if (m <= 32) {
     pack_seg<K, 1>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
   } else if (m <= 64) {
