@@ -6,11 +6,12 @@
 namespace eplb {
 namespace {
 
+template <bool kCap2>
 __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_trigger();
   pdl_wait();
-  rebalance_row(a, blockIdx.x, smem);
+  rebalance_row<kCap2>(a, blockIdx.x, smem);
 }
 
 }  // namespace
@@ -23,8 +24,9 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
   if (!device_info(&di)) return cuda_fail(cudaGetLastError());
   const Layout lay(sh);
   if (lay.total > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
-  const eplb_status pst =
-      prepare_kernel(reinterpret_cast<const void *>(rebalance_kernel), kMaxThreads, lay.total, nullptr);
+  const void *fn = cap2_shape(sh) ? reinterpret_cast<const void *>(rebalance_kernel<true>)
+                                  : reinterpret_cast<const void *>(rebalance_kernel<false>);
+  const eplb_status pst = prepare_kernel(fn, kMaxThreads, lay.total, nullptr);
   if (pst != EPLB_OK) return pst;
   RbArgs a;
   a.ring = ring;
@@ -43,8 +45,8 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
                  (reinterpret_cast<uintptr_t>(log2phy) % 16 == 0);
   const int threads = R <= 2 * static_cast<int64_t>(di.sms) ? kFewRowThreads : kManyRowThreads;
   void *args[] = {&a};
-  const cudaError_t err = launch_pdl(reinterpret_cast<const void *>(rebalance_kernel), dim3(static_cast<unsigned>(R)),
-                   dim3(threads), lay.total, stream, args);
+  const cudaError_t err =
+      launch_pdl(fn, dim3(static_cast<unsigned>(R)), dim3(threads), lay.total, stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

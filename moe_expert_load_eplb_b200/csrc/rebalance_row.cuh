@@ -410,6 +410,15 @@ __device__ void pack_warp(const K *skey, int n, int m, int cap, K *pw, int32_t *
 // the packs take their second item lightest first -- ascending (weight,
 // index) of their first item -- and pack p takes item m + pos(p).  One
 // thread per pack, no dependent chain.
+constexpr int kCap2MinPacks = 16;
+
+// True when either packing step of rebalance_experts on shape s has two items
+// per pack over at least kCap2MinPacks packs (the closed form may apply).
+__host__ __device__ inline bool cap2_shape(const RebalanceShape &s) {
+  return (s.ppg == 2 && s.ppn == 2 * s.mpn && s.mpn >= kCap2MinPacks) ||
+         (s.gpn == 2 && s.G == 2 * s.N && s.N >= kCap2MinPacks);
+}
+
 template <typename K>
 __device__ void pack_cap2(const K *skey_base, int stride, int nseg, int m, int32_t *ipack,
                           int32_t *irank, int out_stride) {
@@ -438,19 +447,24 @@ __device__ void pack_cap2(const K *skey_base, int stride, int nseg, int m, int32
 // Packs nseg segments (segment g: n sorted keys at skey + g * stride, results
 // at ipack/irank + g * out_stride) into m packs of cap items each.  Called by
 // every thread of the CTA (the lane-parallel variant needs whole warps).
-template <typename K>
+// kCap2 compiles in the two-items-per-pack closed form; kernels for shapes
+// that can never take it are built without it (its code alone, never run,
+// slowed the row by about 2 us: the kernel is instruction-fetch bound).
+template <typename K, bool kCap2>
 __device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
                               int32_t *pc, int32_t *ipack, int32_t *irank, int out_stride) {
   if (n <= 0) return;
-  // closed form only for long chains: on a few packs (8 groups onto 4 nodes)
-  // the vote cost more than the short greedy it replaces (measured)
-  if (cap == 2 && n == 2 * m && m >= 16) {  // uniform: every segment has the same shape
-    bool ok = true;
-    for (int g = threadIdx.x; g < nseg; g += nthr())
-      ok &= (skey[g * stride + m - 1] >> kIdxBits) != K(0);
-    if (__syncthreads_and(ok)) {
-      pack_cap2<K>(skey, stride, nseg, m, ipack, irank, out_stride);
-      return;
+  if constexpr (kCap2) {
+    // closed form only for long chains: on a few packs (8 groups onto 4
+    // nodes) the vote cost more than the short greedy it replaces (measured)
+    if (cap == 2 && n == 2 * m && m >= kCap2MinPacks) {  // every segment has this shape
+      bool ok = true;
+      for (int g = threadIdx.x; g < nseg; g += nthr())
+        ok &= (skey[g * stride + m - 1] >> kIdxBits) != K(0);
+      if (__syncthreads_and(ok)) {
+        pack_cap2<K>(skey, stride, nseg, m, ipack, irank, out_stride);
+        return;
+      }
     }
   }
   if (m <= 32) {
@@ -629,7 +643,7 @@ __device__ void write_error_row(const RbArgs &a, int64_t row) {
   for (int i = threadIdx.x; i < s.E * s.X; i += nthr()) gl[i] = -1;
 }
 
-template <typename K>
+template <typename K, bool kCap2>
 __device__ void step3(const RbArgs &a, unsigned char *smem, const Layout &lay) {
   const RebalanceShape &s = a.s;
   K *keys = reinterpret_cast<K *>(smem + lay.keys);
@@ -663,13 +677,15 @@ __device__ void step3(const RbArgs &a, unsigned char *smem, const Layout &lay) {
   } else {
     bitonic_desc<K>(keys, s.npad, s.N);
   }
-  pack_segments<K>(skeys, s.npad, s.N, s.ppn, s.mpn, s.ppg, reinterpret_cast<K *>(smem + lay.pw), reinterpret_cast<int32_t *>(smem + lay.pc),
+  pack_segments<K, kCap2>(skeys, s.npad, s.N, s.ppn, s.mpn, s.ppg, reinterpret_cast<K *>(smem + lay.pw), reinterpret_cast<int32_t *>(smem + lay.pc),
                    reinterpret_cast<int32_t *>(smem + lay.ipack),
                    reinterpret_cast<int32_t *>(smem + lay.irank), s.ppn);
 }
 
 // One row of rebalance_experts, by the whole CTA, in `smem` (Layout(a.s).total
-// bytes).  Called by every thread of the CTA.
+// bytes).  Called by every thread of the CTA; kCap2 = cap2_shape(a.s) (a
+// kernel built without it is correct on every shape, only slower on those).
+template <bool kCap2>
 __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsigned char *smem) {
   __shared__ int flags[2];  // [0] 128-bit keys needed, [1] exact ratio not representable
   const RebalanceShape &s = a.s;
@@ -765,7 +781,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       gs_keys = gkey;
     }
     __syncthreads();
-    pack_segments<uint64_t>(gs_keys, s.gpad, 1, s.G, s.N, s.gpn,
+    pack_segments<uint64_t, kCap2>(gs_keys, s.gpad, 1, s.G, s.N, s.gpn,
                             reinterpret_cast<uint64_t *>(smem + lay.npw),
                             reinterpret_cast<int32_t *>(smem + lay.npc), gpack, grank, s.G);
   }
@@ -877,9 +893,9 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       irank[t] = 0;
     }
   } else if (flags[0] == 0) {
-    step3<uint64_t>(a, smem, lay);
+    step3<uint64_t, kCap2>(a, smem, lay);
   } else {
-    step3<u128>(a, smem, lay);
+    step3<u128, kCap2>(a, smem, lay);
   }
   __syncthreads();
 

@@ -32,7 +32,7 @@ struct ServeArgs {
   uint32_t *layer_done;
 };
 
-template <bool kVecToken>
+template <bool kVecToken, bool kCap2>
 __global__ void __launch_bounds__(kThreads) serve_kernel(ServeArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int last;
@@ -54,7 +54,7 @@ __global__ void __launch_bounds__(kThreads) serve_kernel(ServeArgs a) {
   if (!last) return;
   __threadfence();
   if (threadIdx.x == 0) a.layer_done[layer] = 0;
-  rebalance_row(a.b, layer, smem);
+  rebalance_row<kCap2>(a.b, layer, smem);
 }
 
 }  // namespace
@@ -93,8 +93,12 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
   a.b.table_vec4 = ((static_cast<int64_t>(sh.E) * sh.X) % 4 == 0) &&
                    (reinterpret_cast<uintptr_t>(next_log2phy) % 16 == 0);
   a.layer_done = layer_done;
-  const void *fn = (K % 4) == 0 ? reinterpret_cast<const void *>(serve_kernel<true>)
-                                : reinterpret_cast<const void *>(serve_kernel<false>);
+  const bool vec = (K % 4) == 0, cap2 = cap2_shape(sh);
+  const void *fn =
+      vec ? (cap2 ? reinterpret_cast<const void *>(serve_kernel<true, true>)
+                  : reinterpret_cast<const void *>(serve_kernel<true, false>))
+          : (cap2 ? reinterpret_cast<const void *>(serve_kernel<false, true>)
+                  : reinterpret_cast<const void *>(serve_kernel<false, false>));
   int per_sm = 0;
   st = prepare_kernel(fn, kThreads, smem, &per_sm);
   if (st != EPLB_OK) return st;

@@ -210,6 +210,9 @@ SHAPES = [
     (1, 1, 1, 1, 1), (1, 1, 64, 1, 4), (2, 2, 2, 2, 2), (1024, 32, 2048, 8, 64), (1024, 1, 1024, 1, 1),
     (384, 12, 448, 4, 64), (160, 10, 200, 5, 40), (128, 16, 160, 16, 32), (256, 8, 320, 1, 160),
     (96, 3, 2048, 2, 8), (300, 5, 602, 7, 7),
+    # two groups per node over 16+ nodes / two replicas per GPU over 16+ GPUs
+    # per node: the balanced_packing closed form for two items per pack
+    (64, 32, 128, 16, 32), (96, 48, 192, 24, 48), (64, 16, 128, 1, 64),
 ]
 
 
@@ -574,6 +577,8 @@ def _dev(a):
     (4, 0, 4, 24, 40, 6, 2, 4),         # no tokens: the plan from the ring alone
     (2, 20000, 3, 32, 48, 4, 3, 6),     # global policy (G % N != 0), K not a multiple of 4
     (58, 8192, 8, 256, 288, 8, 4, 32),  # DeepSeek-V3 shape, decode-sized batch
+    (3, 5000, 8, 256, 288, 1, 2, 144),  # global policy, two replicas per GPU on 144 GPUs
+    (2, 3000, 6, 64, 128, 32, 16, 32),  # two groups per node on 16 nodes
 ])
 @pytest.mark.parametrize("W_,slot,zero_slot", [(3, 1, 2), (1, 0, 0), (4, 3, -1)])
 def test_serve_step_matches_oracle(shape, W_, slot, zero_slot):
