@@ -1,6 +1,7 @@
 // rebalance.cu -- S3/S4 (and, in ring mode, S2): rebalance_experts over R
 // rows, one CTA per row.  The row's work is rebalance_row (rebalance_row.cuh),
 // shared with the serving-step kernel.
+#define EPLB_RB_COLD __noinline__  // cold paths out of line (rebalance_row.cuh)
 #include "rebalance_row.cuh"
 
 namespace eplb {

@@ -46,6 +46,17 @@
 #include "common.cuh"
 #include "internal.h"
 
+// Paths the common shapes never take (128-entry packs, bitonic sorts, wide
+// replication, the two-items-per-pack closed form) carry EPLB_RB_COLD.  The
+// rebalance kernel defines it as __noinline__ before including this header:
+// the row's code is then compact in the instruction cache, which made the
+// 58-row DeepSeek-V3 rebalance about 2 us faster (measured).  The serving
+// kernel keeps them inline: there the calls raised its register spills from
+// 12 to 64 bytes a thread.
+#ifndef EPLB_RB_COLD
+#define EPLB_RB_COLD
+#endif
+
 namespace eplb {
 namespace {
 
@@ -270,7 +281,7 @@ __device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit em
 // CTA-wide bitonic sort, descending, of nseg segments of npad (power of two)
 // keys each, in place; padding keys must be 0.
 template <typename K>
-__device__ void bitonic_desc(K *key, int npad, int nseg) {
+__device__ EPLB_RB_COLD void bitonic_desc(K *key, int npad, int nseg) {
   const int half = (npad * nseg) >> 1;
   for (int k = 2; k <= npad; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
@@ -369,7 +380,7 @@ __device__ void pack_seg(const K *skey_base, int stride, int nseg, int n, int m,
 // of its lightest non-full pack; the warp takes the minimum with an xor
 // butterfly.
 template <typename K>
-__device__ void pack_warp(const K *skey, int n, int m, int cap, K *pw, int32_t *pc,
+__device__ EPLB_RB_COLD void pack_warp(const K *skey, int n, int m, int cap, K *pw, int32_t *pc,
                           int32_t *ipack, int32_t *irank) {
   const int lane = threadIdx.x & 31;
   const K imask = K(kIdxMask);
@@ -420,7 +431,7 @@ __host__ __device__ inline bool cap2_shape(const RebalanceShape &s) {
 }
 
 template <typename K>
-__device__ void pack_cap2(const K *skey_base, int stride, int nseg, int m, int32_t *ipack,
+__device__ EPLB_RB_COLD void pack_cap2(const K *skey_base, int stride, int nseg, int m, int32_t *ipack,
                           int32_t *irank, int out_stride) {
   const K imask = K(kIdxMask);
   for (int t = threadIdx.x; t < nseg * m; t += nthr()) {
@@ -450,6 +461,11 @@ __device__ void pack_cap2(const K *skey_base, int stride, int nseg, int m, int32
 // kCap2 compiles in the two-items-per-pack closed form; kernels for shapes
 // that can never take it are built without it (its code alone, never run,
 // slowed the row by about 2 us: the kernel is instruction-fetch bound).
+template <typename K>
+__device__ EPLB_RB_COLD void pack_segments_wide(const K *skey, int stride, int nseg, int n, int m,
+                                                int cap, K *pw, int32_t *pc, int32_t *ipack,
+                                                int32_t *irank, int out_stride);
+
 template <typename K, bool kCap2>
 __device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
                               int32_t *pc, int32_t *ipack, int32_t *irank, int out_stride) {
@@ -469,7 +485,16 @@ __device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m,
   }
   if (m <= 32) {
     pack_seg<K, 1>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
-  } else if (m <= 64) {
+  } else {
+    pack_segments_wide<K>(skey, stride, nseg, n, m, cap, pw, pc, ipack, irank, out_stride);
+  }
+}
+
+template <typename K>
+__device__ EPLB_RB_COLD void pack_segments_wide(const K *skey, int stride, int nseg, int n, int m,
+                                                int cap, K *pw, int32_t *pc, int32_t *ipack,
+                                                int32_t *irank, int out_stride) {
+  if (m <= 64) {
     pack_seg<K, 2>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
   } else if (m <= 128) {
     pack_seg<K, 4>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
@@ -553,19 +578,18 @@ __device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
 }
 
 // Greedy over nc <= 32 candidates, one per lane of a warp.
-__device__ void replicate_warp(const RebalanceShape &s, int n, const int64_t *cand_w,
-                               const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
-                               int32_t *rrank) {
+__device__ EPLB_RB_COLD void replicate_warp(int nc, int lpn, int ppn, int n, const int64_t *cand_w,
+                                            const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
+                                            int32_t *rrank) {
   const int lane = threadIdx.x & 31;
-  const int nc = num_cand(s);
-  const int bp = n * s.ppn;
+  const int bp = n * ppn;
   const bool valid = lane < nc;
   const int64_t w = valid ? cand_w[n * nc + lane] : 0;
   const int id = valid ? cand_i[n * nc + lane] : 0x7fffffff;
   int c = 1;
   int rounds = 0;
   while ((1 << rounds) < min(nc, 32)) ++rounds;
-  for (int r = 0; r < s.ppn - s.lpn; ++r) {
+  for (int r = 0; r < ppn - lpn; ++r) {
     int64_t bw = w;
     int bc = c, bi = id, bl = lane;
     for (int k = rounds - 1; k >= 0; --k) {
@@ -581,8 +605,8 @@ __device__ void replicate_warp(const RebalanceShape &s, int n, const int64_t *ca
       }
     }
     if (valid && lane == bl) {
-      p2m[bp + s.lpn + r] = id;
-      rrank[bp + s.lpn + r] = c;
+      p2m[bp + lpn + r] = id;
+      rrank[bp + lpn + r] = c;
       ++c;
     }
   }
@@ -591,15 +615,15 @@ __device__ void replicate_warp(const RebalanceShape &s, int n, const int64_t *ca
 }
 
 // Any number of candidates (all experts of the node), counts in shared memory.
-__device__ void replicate_smem(const RebalanceShape &s, int n, const int64_t *wm, int32_t *cnt,
+__device__ EPLB_RB_COLD void replicate_smem(int lpn, int ppn, int n, const int64_t *wm, int32_t *cnt,
                                int32_t *p2m, int32_t *rrank) {
   const int lane = threadIdx.x & 31;
-  const int bm = n * s.lpn, bp = n * s.ppn;
+  const int bm = n * lpn, bp = n * ppn;
   auto local_best = [&](int64_t &bw, int &bc, int &bi) {
     bw = 0;
     bc = 1;
     bi = 0x7fffffff;
-    for (int i = lane; i < s.lpn; i += 32)
+    for (int i = lane; i < lpn; i += 32)
       if (rep_better(wm[bm + i], cnt[bm + i], i, bw, bc, bi)) {
         bw = wm[bm + i];
         bc = cnt[bm + i];
@@ -609,7 +633,7 @@ __device__ void replicate_smem(const RebalanceShape &s, int n, const int64_t *wm
   int64_t bw;
   int bc, bi;
   local_best(bw, bc, bi);
-  for (int r = 0; r < s.ppn - s.lpn; ++r) {
+  for (int r = 0; r < ppn - lpn; ++r) {
     int64_t mw = bw;
     int mc = bc, mi = bi;
     for (int k = 16; k >= 1; k >>= 1) {
@@ -624,62 +648,85 @@ __device__ void replicate_smem(const RebalanceShape &s, int n, const int64_t *wm
     }
     if (lane == (mi & 31)) {
       cnt[bm + mi] = mc + 1;
-      p2m[bp + s.lpn + r] = mi;
-      rrank[bp + s.lpn + r] = mc;
+      p2m[bp + lpn + r] = mi;
+      rrank[bp + lpn + r] = mc;
       local_best(bw, bc, bi);
     }
     __syncwarp();
   }
 }
 
-__device__ void write_error_row(const RbArgs &a, int64_t row) {
-  const RebalanceShape &s = a.s;
-  for (int t = threadIdx.x; t < s.P; t += nthr()) {
-    a.phy2log[row * s.P + t] = -1;
-    a.phyrank[row * s.P + t] = -1;
+// The plan of a row that cannot be computed: no replicas, log2phy all -1.
+__device__ void write_error_row(int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
+                                             int32_t *log2phy, int P, int E, int X, int64_t row) {
+  for (int t = threadIdx.x; t < P; t += nthr()) {
+    phy2log[row * P + t] = -1;
+    phyrank[row * P + t] = -1;
   }
-  for (int e = threadIdx.x; e < s.E; e += nthr()) a.logcnt[row * s.E + e] = 0;
-  int32_t *gl = a.log2phy + row * static_cast<int64_t>(s.E) * s.X;
-  for (int i = threadIdx.x; i < s.E * s.X; i += nthr()) gl[i] = -1;
+  for (int e = threadIdx.x; e < E; e += nthr()) logcnt[row * E + e] = 0;
+  int32_t *gl = log2phy + row * static_cast<int64_t>(E) * X;
+  for (int i = threadIdx.x; i < E * X; i += nthr()) gl[i] = -1;
 }
 
+// Operands of step 3 as plain values (an out-of-line instance then needs no
+// copy of the kernel's parameter block or of the layout on the stack).
+struct Step3Ops {
+  unsigned char *keys, *sorted, *pw;
+  const int64_t *wm;
+  const uint64_t *lam;
+  const int32_t *cnt, *p2m;
+  int32_t *pc, *ipack, *irank;
+  int N, npad, lpn, ppn, mpn, ppg;
+};
+
 template <typename K, bool kCap2>
-__device__ void step3(const RbArgs &a, unsigned char *smem, const Layout &lay) {
-  const RebalanceShape &s = a.s;
-  K *keys = reinterpret_cast<K *>(smem + lay.keys);
-  K *sorted = reinterpret_cast<K *>(smem + lay.sorted);
-  const int64_t *wm = reinterpret_cast<const int64_t *>(smem + lay.wm);
-  const uint64_t *lam = reinterpret_cast<const uint64_t *>(smem + lay.lam);
-  const int32_t *cnt = reinterpret_cast<const int32_t *>(smem + lay.cnt);
-  const int32_t *p2m = reinterpret_cast<const int32_t *>(smem + lay.p2m);
+__device__ void step3(const Step3Ops &o) {
+  K *keys = reinterpret_cast<K *>(o.keys);
+  K *sorted = reinterpret_cast<K *>(o.sorted);
+  const int64_t *wm = o.wm;
+  const uint64_t *lam = o.lam;
+  const int32_t *cnt = o.cnt;
+  const int32_t *p2m = o.p2m;
+  const int N = o.N, npad = o.npad, lpn = o.lpn, ppn = o.ppn;
   const K imask = K(kIdxMask);
-  const bool ranked = s.npad <= kRankSortMax;
-  const int per = ranked ? s.ppn : s.npad;
-  for (int t = threadIdx.x; t < s.N * per; t += nthr()) {
+  const bool ranked = npad <= kRankSortMax;
+  const int per = ranked ? ppn : npad;
+  for (int t = threadIdx.x; t < N * per; t += nthr()) {
     const int n = t / per;
     const int j = t - n * per;
     K key = 0;
-    if (j < s.ppn) {
-      const int m = n * s.lpn + p2m[n * s.ppn + j];
+    if (j < ppn) {
+      const int m = n * lpn + p2m[n * ppn + j];
       const uint32_t c = static_cast<uint32_t>(cnt[m]);
       const uint64_t scale = c == 1 ? lam[n] : lam[n] / c;
       key = ((K(static_cast<uint64_t>(wm[m])) * K(scale)) << kIdxBits) | (imask - K(j));
     }
-    keys[n * s.npad + j] = key;
+    keys[n * npad + j] = key;
   }
   __syncthreads();
   const K *skeys = keys;
   if (ranked) {
-    rank_segments<K>(keys, s.npad, s.N, s.ppn,
-                     [&](int g, int, int r, K k) { sorted[g * s.npad + r] = k; });
+    rank_segments<K>(keys, npad, N, ppn,
+                     [&](int g, int, int r, K k) { sorted[g * npad + r] = k; });
     skeys = sorted;
     __syncthreads();
   } else {
-    bitonic_desc<K>(keys, s.npad, s.N);
+    bitonic_desc<K>(keys, npad, N);
   }
-  pack_segments<K, kCap2>(skeys, s.npad, s.N, s.ppn, s.mpn, s.ppg, reinterpret_cast<K *>(smem + lay.pw), reinterpret_cast<int32_t *>(smem + lay.pc),
-                   reinterpret_cast<int32_t *>(smem + lay.ipack),
-                   reinterpret_cast<int32_t *>(smem + lay.irank), s.ppn);
+  pack_segments<K, kCap2>(skeys, npad, N, ppn, o.mpn, o.ppg, reinterpret_cast<K *>(o.pw), o.pc,
+                          o.ipack, o.irank, ppn);
+}
+
+// step 3 with 128-bit keys (rows whose weights times Lambda overflow 64 bits);
+// left inline: out of line, its call made the kernel spill around it
+template <bool kCap2>
+__device__ void step3_wide(unsigned char *keys, unsigned char *sorted, unsigned char *pw,
+                                        const int64_t *wm, const uint64_t *lam, const int32_t *cnt,
+                                        const int32_t *p2m, int32_t *pc, int32_t *ipack,
+                                        int32_t *irank, int N, int npad, int lpn, int ppn, int mpn,
+                                        int ppg) {
+  step3<u128, kCap2>(Step3Ops{keys, sorted, pw, wm, lam, cnt, p2m, pc, ipack, irank, N, npad, lpn,
+                              ppn, mpn, ppg});
 }
 
 // One row of rebalance_experts, by the whole CTA, in `smem` (Layout(a.s).total
@@ -744,7 +791,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     }
   }
   if (__syncthreads_or(bad)) {
-    write_error_row(a, row);
+    write_error_row(a.phy2log, a.phyrank, a.logcnt, a.log2phy, s.P, s.E, s.X, row);
     if (tid == 0) report(a.status, EPLB_ERR_RANGE);
     return;
   }
@@ -823,7 +870,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       replicate_pairs(s, cand_w, cand_i, cand_c, p2m, rrank);
     } else {
       for (int n = tid >> 5; n < s.N; n += nwarps())
-        replicate_warp(s, n, cand_w, cand_i, cand_c, p2m, rrank);
+        replicate_warp(nc, s.lpn, s.ppn, n, cand_w, cand_i, cand_c, p2m, rrank);
     }
     __syncthreads();
     for (int t = tid; t < s.N * nc; t += nthr()) {
@@ -831,7 +878,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       cnt[n * s.lpn + cand_i[t]] = cand_c[t];
     }
   } else if (nc > 32) {
-    for (int n = tid >> 5; n < s.N; n += nwarps()) replicate_smem(s, n, wm, cnt, p2m, rrank);
+    for (int n = tid >> 5; n < s.N; n += nwarps()) replicate_smem(s.lpn, s.ppn, n, wm, cnt, p2m, rrank);
   }
   __syncthreads();
 
@@ -880,7 +927,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     __syncthreads();
   }
   if (flags[1]) {
-    write_error_row(a, row);
+    write_error_row(a.phy2log, a.phyrank, a.logcnt, a.log2phy, s.P, s.E, s.X, row);
     if (tid == 0) report(a.status, EPLB_ERR_RANGE);
     return;
   }
@@ -893,9 +940,13 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       irank[t] = 0;
     }
   } else if (flags[0] == 0) {
-    step3<uint64_t, kCap2>(a, smem, lay);
+    step3<uint64_t, kCap2>(Step3Ops{smem + lay.keys, smem + lay.sorted, smem + lay.pw, wm, lam, cnt,
+                                    p2m, reinterpret_cast<int32_t *>(smem + lay.pc), ipack, irank,
+                                    s.N, s.npad, s.lpn, s.ppn, s.mpn, s.ppg});
   } else {
-    step3<u128, kCap2>(a, smem, lay);
+    step3_wide<kCap2>(smem + lay.keys, smem + lay.sorted, smem + lay.pw, wm, lam, cnt, p2m,
+                      reinterpret_cast<int32_t *>(smem + lay.pc), ipack, irank, s.N, s.npad, s.lpn,
+                      s.ppn, s.mpn, s.ppg);
   }
   __syncthreads();
 
