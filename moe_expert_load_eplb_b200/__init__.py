@@ -107,14 +107,58 @@ def _check(code: int, where: str):
         raise EplbError(code, where, detail)
 
 
-def _cuda(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
+def _cuda(t: torch.Tensor, dtype: torch.dtype, name: str,
+          device: Optional[torch.device] = None) -> torch.Tensor:
+    """t must be a contiguous CUDA tensor of dtype (on ``device`` if given):
+    the C ABI takes bare pointers and cannot check any of it."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}; the call runs on {device}")
     return t
+
+
+_BAD_DTYPES = (torch.int64, torch.uint64)
+
+
+def _word(t: Optional[torch.Tensor], dtypes, name: str, device: torch.device):
+    """An optional device word: the bad-index tally (64-bit) or the status
+    word (int32).  None passes a null pointer (the word is not written)."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be one of {dtypes}, got {t.dtype}")
+    if t.numel() < 1:
+        raise ValueError(f"{name} must hold at least one element")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}; the call runs on {device}")
+    return t
+
+
+def _words(device: torch.device, bad=None, status=None):
+    _word(bad, _BAD_DTYPES, "bad", device)
+    _word(status, (torch.int32,), "status", device)
+
+
+def _check_plan(plan, name: str, R: int, E: int, X: int, P: Optional[int],
+                device: torch.device):
+    """The four plan tensors: log2phy [R, E, X], logcnt [R, E] and, if P is
+    given, phy2log / phyrank [R, P]; all int32 on ``device``."""
+    _cuda(plan.log2phy, torch.int32, f"{name}.log2phy", device)
+    _cuda(plan.logcnt, torch.int32, f"{name}.logcnt", device)
+    if tuple(plan.log2phy.shape) != (R, E, X) or tuple(plan.logcnt.shape) != (R, E):
+        raise ValueError(f"{name}: log2phy must be {(R, E, X)} and logcnt {(R, E)}")
+    if P is not None:
+        _cuda(plan.phy2log, torch.int32, f"{name}.phy2log", device)
+        _cuda(plan.phyrank, torch.int32, f"{name}.phyrank", device)
+        if tuple(plan.phy2log.shape) != (R, P) or tuple(plan.phyrank.shape) != (R, P):
+            raise ValueError(f"{name}: phy2log and phyrank must be {(R, P)}")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -166,9 +210,10 @@ def count_loads(idx: torch.Tensor, num_experts: int, counts: Optional[torch.Tens
     if counts is None:
         counts = torch.empty((L, num_experts), dtype=torch.int64, device=idx.device)
         accumulate = False
-    _cuda(counts, torch.int64, "counts")
+    _cuda(counts, torch.int64, "counts", idx.device)
     if tuple(counts.shape) != (L, num_experts):
         raise ValueError("counts must be [L, E]")
+    _words(idx.device, bad, status)
     with _on_device(idx.device):
         _check(load_library().eplb_count_loads(
             _ptr(idx), L, T, K, num_experts, _ptr(counts), int(bool(accumulate)),
@@ -186,9 +231,10 @@ def window_accumulate(steps: torch.Tensor, window: int, s_first: int = 0,
     S, L, E = steps.shape
     if out is None:
         out = torch.empty((max(S - s_first, 0), L, E), dtype=torch.int64, device=steps.device)
-    _cuda(out, torch.int64, "out")
+    _cuda(out, torch.int64, "out", steps.device)
     if tuple(out.shape) != (S - s_first, L, E):
         raise ValueError("out must be [S - s_first, L, E]")
+    _words(steps.device, status=status)
     with _on_device(steps.device):
         _check(load_library().eplb_window_accumulate(
             _ptr(steps), S, L, E, window, s_first, _ptr(out), _ptr(status),
@@ -221,9 +267,10 @@ def rebalance(loads: torch.Tensor, num_replicas: int, num_groups: int, num_nodes
                    torch.empty((R, E, X), dtype=torch.int32, device=dev))
     for name, t, shape in (("phy2log", out.phy2log, (R, P)), ("phyrank", out.phyrank, (R, P)),
                            ("logcnt", out.logcnt, (R, E)), ("log2phy", out.log2phy, (R, E, X))):
-        _cuda(t, torch.int32, name)
+        _cuda(t, torch.int32, name, dev)
         if tuple(t.shape) != shape:
             raise ValueError(f"{name} must be {shape}")
+    _words(dev, status=status)
     with _on_device(dev):
         _check(load_library().eplb_rebalance(
             _ptr(loads), R, E, P, num_groups, num_nodes, num_gpus, X,
@@ -253,11 +300,12 @@ def rebalance_window(ring: torch.Tensor, num_replicas: int, num_groups: int, num
                    torch.empty((R, E, X), dtype=torch.int32, device=dev))
     for name, t, shape in (("phy2log", out.phy2log, (R, P)), ("phyrank", out.phyrank, (R, P)),
                            ("logcnt", out.logcnt, (R, E)), ("log2phy", out.log2phy, (R, E, X))):
-        _cuda(t, torch.int32, name)
+        _cuda(t, torch.int32, name, dev)
         if tuple(t.shape) != shape:
             raise ValueError(f"{name} must be {shape}")
+    _words(dev, status=status)
     if loads_out is not None:
-        _cuda(loads_out, torch.int64, "loads_out")
+        _cuda(loads_out, torch.int64, "loads_out", dev)
         if tuple(loads_out.shape) not in ((R, E), (1, R, E)):
             raise ValueError("loads_out must be [R, E]")
     with _on_device(dev):
@@ -273,8 +321,8 @@ def redirect(idx: torch.Tensor, log2phy: torch.Tensor, logcnt: torch.Tensor, tok
              status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """S5: out[l, t, k] = log2phy[l, e, (token_offset + t) mod logcnt[l, e]], e = idx[l, t, k]."""
     _cuda(idx, torch.int32, "idx")
-    _cuda(log2phy, torch.int32, "log2phy")
-    _cuda(logcnt, torch.int32, "logcnt")
+    _cuda(log2phy, torch.int32, "log2phy", idx.device)
+    _cuda(logcnt, torch.int32, "logcnt", idx.device)
     if idx.dim() != 3 or log2phy.dim() != 3 or logcnt.dim() != 2:
         raise ValueError("idx [L, T, K], log2phy [L, E, X], logcnt [L, E] expected")
     L, T, K = idx.shape
@@ -283,9 +331,10 @@ def redirect(idx: torch.Tensor, log2phy: torch.Tensor, logcnt: torch.Tensor, tok
         raise ValueError("table shapes do not match idx")
     if out is None:
         out = torch.empty_like(idx)
-    _cuda(out, torch.int32, "out")
+    _cuda(out, torch.int32, "out", idx.device)
     if out.shape != idx.shape:
         raise ValueError("out must match idx")
+    _words(idx.device, bad, status)
     with _on_device(idx.device):
         _check(load_library().eplb_redirect(
             _ptr(idx), L, T, K, E, _ptr(log2phy), X, _ptr(logcnt), int(token_offset),
@@ -301,8 +350,8 @@ def count_redirect(idx: torch.Tensor, num_experts: int, log2phy: torch.Tensor, l
     """S1 + S5 in one pass over idx: counts (+)= histogram of idx and
     out = redirect(idx, log2phy, logcnt, token_offset).  Returns (counts, out)."""
     _cuda(idx, torch.int32, "idx")
-    _cuda(log2phy, torch.int32, "log2phy")
-    _cuda(logcnt, torch.int32, "logcnt")
+    _cuda(log2phy, torch.int32, "log2phy", idx.device)
+    _cuda(logcnt, torch.int32, "logcnt", idx.device)
     if idx.dim() != 3 or log2phy.dim() != 3 or logcnt.dim() != 2:
         raise ValueError("idx [L, T, K], log2phy [L, E, X], logcnt [L, E] expected")
     L, T, K = idx.shape
@@ -312,20 +361,52 @@ def count_redirect(idx: torch.Tensor, num_experts: int, log2phy: torch.Tensor, l
     if counts is None:
         counts = torch.empty((L, E), dtype=torch.int64, device=idx.device)
         accumulate = False
-    _cuda(counts, torch.int64, "counts")
+    _cuda(counts, torch.int64, "counts", idx.device)
     if tuple(counts.shape) != (L, E):
         raise ValueError("counts must be [L, E]")
     if out is None:
         out = torch.empty_like(idx)
-    _cuda(out, torch.int32, "out")
+    _cuda(out, torch.int32, "out", idx.device)
     if out.shape != idx.shape:
         raise ValueError("out must match idx")
+    _words(idx.device, bad, status)
     with _on_device(idx.device):
         _check(load_library().eplb_count_redirect(
             _ptr(idx), L, T, K, E, _ptr(counts), int(bool(accumulate)), _ptr(log2phy), X,
             _ptr(logcnt), int(token_offset), _ptr(out), _ptr(bad), _ptr(status),
             _stream(idx.device)), "eplb_count_redirect")
     return counts, out
+
+
+def _serve_args(idx, plan, ring, next_plan, out, loads_out, bad, status):
+    """Checks shared by both one-launch entry points; returns (L, T, K, W, E,
+    P, X, out)."""
+    _cuda(idx, torch.int32, "idx")
+    dev = idx.device
+    _cuda(ring, torch.int64, "ring", dev)
+    if idx.dim() != 3 or ring.dim() != 3:
+        raise ValueError("idx [L, T, K] and ring [W, L, E] expected")
+    L, T, K = idx.shape
+    Wr, Lr, E = ring.shape
+    if Lr != L:
+        raise ValueError("ring and idx disagree on L")
+    if next_plan.phy2log.dim() != 2 or plan.log2phy.dim() != 3:
+        raise ValueError("plan.log2phy [L, E, X] and next_plan.phy2log [L, P] expected")
+    P = next_plan.phy2log.shape[1]
+    X = plan.log2phy.shape[2]
+    _check_plan(plan, "plan", L, E, X, None, dev)
+    _check_plan(next_plan, "next_plan", L, E, X, P, dev)
+    if out is None:
+        out = torch.empty_like(idx)
+    _cuda(out, torch.int32, "out", dev)
+    if out.shape != idx.shape:
+        raise ValueError("out must match idx")
+    if loads_out is not None:
+        _cuda(loads_out, torch.int64, "loads_out", dev)
+        if loads_out.numel() != L * E:
+            raise ValueError("loads_out must be [L, E]")
+    _words(dev, bad, status)
+    return L, T, K, Wr, E, P, X, out
 
 
 def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, next_plan: Plan,
@@ -337,37 +418,13 @@ def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, nex
     with ``plan`` (the plan in force), then rebuild every layer's plan from the
     window sum over the ring into ``next_plan`` (clearing ring[zero_slot]).
     ``layer_done``: uint32 [L] work array, zero before and after.  Returns out."""
-    _cuda(idx, torch.int32, "idx")
-    _cuda(ring, torch.int64, "ring")
-    if idx.dim() != 3 or ring.dim() != 3:
-        raise ValueError("idx [L, T, K] and ring [W, L, E] expected")
-    L, T, K = idx.shape
-    Wr, Lr, E = ring.shape
-    if Lr != L:
-        raise ValueError("ring and idx disagree on L")
-    for name, pl in (("plan", plan), ("next_plan", next_plan)):
-        _cuda(pl.log2phy, torch.int32, f"{name}.log2phy")
-        _cuda(pl.logcnt, torch.int32, f"{name}.logcnt")
-        _cuda(pl.phy2log, torch.int32, f"{name}.phy2log")
-        _cuda(pl.phyrank, torch.int32, f"{name}.phyrank")
-    P = next_plan.phy2log.shape[1]
-    X = plan.log2phy.shape[2]
-    if (tuple(plan.log2phy.shape) != (L, E, X) or tuple(next_plan.log2phy.shape) != (L, E, X)
-            or tuple(plan.logcnt.shape) != (L, E) or tuple(next_plan.logcnt.shape) != (L, E)
-            or tuple(next_plan.phy2log.shape) != (L, P) or tuple(next_plan.phyrank.shape) != (L, P)):
-        raise ValueError("plan shapes do not match idx / ring")
+    L, T, K, Wr, E, P, X, out = _serve_args(idx, plan, ring, next_plan, out, loads_out, bad,
+                                            status)
     if not isinstance(layer_done, torch.Tensor) or not layer_done.is_cuda or \
             layer_done.dtype not in (torch.int32, torch.uint32) or layer_done.numel() != L:
         raise TypeError("layer_done must be a CUDA int32/uint32 tensor of L elements")
-    if out is None:
-        out = torch.empty_like(idx)
-    _cuda(out, torch.int32, "out")
-    if out.shape != idx.shape:
-        raise ValueError("out must match idx")
-    if loads_out is not None:
-        _cuda(loads_out, torch.int64, "loads_out")
-        if loads_out.numel() != L * E:
-            raise ValueError("loads_out must be [L, E]")
+    if not layer_done.is_contiguous() or layer_done.device != idx.device:
+        raise ValueError("layer_done must be contiguous and on the device of idx")
     with _on_device(idx.device):
         _check(load_library().eplb_serve_step(
             _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
@@ -388,18 +445,8 @@ def serve_step_noalloc(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: 
     """serve_step with the library's own per-layer counters (no work array;
     calls must not overlap on one device).  ``out`` must be given or is
     allocated here by torch, outside the call."""
-    _cuda(idx, torch.int32, "idx")
-    _cuda(ring, torch.int64, "ring")
-    if idx.dim() != 3 or ring.dim() != 3:
-        raise ValueError("idx [L, T, K] and ring [W, L, E] expected")
-    L, T, K = idx.shape
-    Wr, Lr, E = ring.shape
-    if Lr != L:
-        raise ValueError("ring and idx disagree on L")
-    P = next_plan.phy2log.shape[1]
-    X = plan.log2phy.shape[2]
-    if out is None:
-        out = torch.empty_like(idx)
+    L, T, K, Wr, E, P, X, out = _serve_args(idx, plan, ring, next_plan, out, loads_out, bad,
+                                            status)
     with _on_device(idx.device):
         _check(load_library().eplb_serve_step_noalloc(
             _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
@@ -415,10 +462,15 @@ def plan_stats(loads: torch.Tensor, phy2log: torch.Tensor, logcnt: torch.Tensor,
     """Per-GPU load (fp64, sum of w/logcnt over the GPU's slots in order) and
     per-row stats {min, max, mean, mean/max}.  Returns (gpu_load [R, gpus], stats [R, 4])."""
     _cuda(loads, torch.int64, "loads")
-    _cuda(phy2log, torch.int32, "phy2log")
-    _cuda(logcnt, torch.int32, "logcnt")
+    _cuda(phy2log, torch.int32, "phy2log", loads.device)
+    _cuda(logcnt, torch.int32, "logcnt", loads.device)
+    if loads.dim() != 2 or phy2log.dim() != 2:
+        raise ValueError("loads [R, E] and phy2log [R, P] expected")
     R, E = loads.shape
     P = phy2log.shape[1]
+    if phy2log.shape[0] != R or tuple(logcnt.shape) != (R, E):
+        raise ValueError("phy2log must be [R, P] and logcnt [R, E]")
+    _words(loads.device, status=status)
     gl = torch.empty((R, num_gpus), dtype=torch.float64, device=loads.device)
     st = torch.empty((R, 4), dtype=torch.float64, device=loads.device)
     with _on_device(loads.device):
@@ -432,8 +484,11 @@ def fold_loads(phys: torch.Tensor, phy2log: torch.Tensor, num_logical: int,
                status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """logical[r, e] = sum of phys[r, p] over slots with phy2log[r, p] == e."""
     _cuda(phys, torch.int64, "phys")
-    _cuda(phy2log, torch.int32, "phy2log")
+    _cuda(phy2log, torch.int32, "phy2log", phys.device)
+    if phys.dim() != 2 or phy2log.shape != phys.shape:
+        raise ValueError("phys and phy2log must both be [R, P]")
     R, P = phys.shape
+    _words(phys.device, status=status)
     out = torch.empty((R, num_logical), dtype=torch.int64, device=phys.device)
     with _on_device(phys.device):
         _check(load_library().eplb_fold_loads(
@@ -457,11 +512,12 @@ def plan_diff(old_phy2log: torch.Tensor, new_phy2log: torch.Tensor, num_logical:
               status: Optional[torch.Tensor] = None):
     """src[r, p] = -1 where the new slot keeps its expert on its GPU, else the old slot
     to copy from; moves[r] = number of copies.  Returns (src, moves)."""
-    _cuda(old_phy2log, torch.int32, "old_phy2log")
     _cuda(new_phy2log, torch.int32, "new_phy2log")
-    if old_phy2log.shape != new_phy2log.shape:
-        raise ValueError("plans must have the same shape")
+    _cuda(old_phy2log, torch.int32, "old_phy2log", new_phy2log.device)
+    if new_phy2log.dim() != 2 or old_phy2log.shape != new_phy2log.shape:
+        raise ValueError("plans must both be [R, P]")
     R, P = new_phy2log.shape
+    _words(new_phy2log.device, status=status)
     src = torch.empty((R, P), dtype=torch.int32, device=new_phy2log.device)
     moves = torch.empty((R,), dtype=torch.int32, device=new_phy2log.device)
     with _on_device(new_phy2log.device):

@@ -664,6 +664,47 @@ def test_serve_step_host_errors():
     assert ei.value.code == 3
 
 
+def test_binding_rejects_malformed_arguments():
+    """The C ABI takes bare pointers; the binding refuses, before any launch,
+    tensors whose shape, dtype or device would let a kernel run off a buffer."""
+    L, T, K, E, P, G, N, gpus = 2, 64, 4, 12, 16, 4, 2, 8
+    X = P - E + 1
+    mk = lambda shape, dt=torch.int32: torch.zeros(shape, dtype=dt, device=DEV)
+    plan = eplb.Plan(mk((L, P)), mk((L, P)), torch.ones((L, E), dtype=torch.int32, device=DEV),
+                     mk((L, E, X)))
+    nxt = eplb.Plan(*[torch.empty_like(t) for t in plan])
+    ring = mk((2, L, E), torch.int64)
+    idx = mk((L, T, K))
+    short = eplb.Plan(nxt.phy2log, nxt.phyrank, nxt.logcnt, mk((L, E, X - 1)))
+    call = eplb.serve_step_noalloc
+    with pytest.raises(ValueError):  # next plan's log2phy narrower than the plan in force
+        call(idx, plan, ring, 0, short, G, N, gpus)
+    with pytest.raises(ValueError):  # phyrank of the wrong width
+        call(idx, plan, ring, 0, eplb.Plan(nxt.phy2log, mk((L, P - 1)), nxt.logcnt, nxt.log2phy),
+             G, N, gpus)
+    with pytest.raises(TypeError):  # ring of the wrong dtype
+        call(idx, plan, ring.to(torch.int32), 0, nxt, G, N, gpus)
+    with pytest.raises(ValueError):  # loads_out too small
+        call(idx, plan, ring, 0, nxt, G, N, gpus, loads_out=mk((L, E - 1), torch.int64))
+    with pytest.raises(ValueError):
+        eplb.serve_step(idx, plan, ring, 0, short, mk(L), G, N, gpus)
+    with pytest.raises(TypeError):  # bad is a 64-bit word
+        eplb.redirect(idx, plan.log2phy, plan.logcnt, bad=mk(1))
+    with pytest.raises(TypeError):  # status is an int32 word
+        eplb.count_loads(idx, E, status=mk(1, torch.int64))
+    with pytest.raises(ValueError):
+        eplb.count_redirect(idx, E, plan.log2phy, plan.logcnt, status=mk(0))
+    with pytest.raises(TypeError):  # a table left on the host
+        eplb.count_redirect(idx, E, plan.log2phy.cpu(), plan.logcnt)
+    with pytest.raises(ValueError):
+        eplb.plan_stats(mk((L, E), torch.int64), plan.phy2log, mk((L, E + 1)), gpus)
+    with pytest.raises(ValueError):
+        eplb.fold_loads(mk((L, P), torch.int64), mk((L, P + 1)), E)
+    with pytest.raises(ValueError):
+        eplb.plan_diff(plan.phy2log, mk((L, P - 1)), E, gpus)
+    torch.cuda.synchronize()
+
+
 # ------------------------------------------- plan stats, fold, initial map, diff --
 
 def _plans_for(c, loads_np):
