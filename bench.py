@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 import workloads as W  # noqa: E402
 
-CFG = W.CONFIGS[2]
+CFG = W.DSV3_PREFILL
 WINDOW = 16
 METRIC = "EPLB layer-rebalances/sec on 1 B200 + load-count GB/s vs HBM peak"
 UNIT = "layer-rebalances/s"
@@ -252,8 +252,8 @@ def run_ours(args, rank: int, world: int, group):
 
     dev = torch.device("cuda", torch.cuda.current_device())
     c = CFG
-    idx = W.routed_indices(2, device=dev, shard=rank)
-    hist = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K * world, 2, device=dev)
+    idx = W.routed_indices("dsv3_prefill", device=dev, shard=rank)
+    hist = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K * world, c.stream, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     hbm_peak, peak_kind = _peaks()
 
@@ -344,8 +344,8 @@ def run_ours(args, rank: int, world: int, group):
     if world == 1 and not args.no_fresh:
         from moe_expert_load_eplb_b200.pipeline import EplbStep, StepGraphs
         Td = 8192
-        idx_d = W.routed_indices(2, device=dev, T=Td)
-        hist_d = W.histogram_steps(WINDOW - 1, c.L, c.E, Td * c.K, 2, device=dev)
+        idx_d = W.routed_indices("dsv3_prefill", device=dev, T=Td)
+        hist_d = W.histogram_steps(WINDOW - 1, c.L, c.E, Td * c.K, c.stream, device=dev)
 
         def make_d():
             st = EplbStep(c.L, Td, c.K, c.E, c.P, c.G, c.N, c.gpus, window=WINDOW, device=dev)
@@ -573,8 +573,8 @@ def run_reference(args):
     full serving step, its 58 layers spread over worker processes (one per
     core, up to 58); one core if no process pool can be had."""
     c = CFG
-    idx_h = W.routed_indices(2, device="cpu", T=c.T).numpy()
-    hist_h = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K, 2).numpy()
+    idx_h = W.routed_indices("dsv3_prefill", device="cpu", T=c.T).numpy()
+    hist_h = W.histogram_steps(WINDOW - 1, c.L, c.E, c.T * c.K, c.stream).numpy()
     try:
         r, cores = _oracle_pool(idx_h, hist_h, {"steps": args.steps, "warmup": args.warmup})
         layers, el = c.L, r["seconds"]

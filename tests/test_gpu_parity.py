@@ -73,27 +73,27 @@ def _assert_plan_equal(plan, ref):
 # ---------------------------------------------------------------- fixtures --
 
 @pytest.fixture(scope="module")
-def c1_idx():
-    return W.c1_indices(device=DEV)
+def tiny_idx():
+    return W.tiny_indices(device=DEV)
 
 
 @pytest.fixture(scope="module")
-def c2_idx():
-    return W.routed_indices(2, device=DEV)
+def dsv3_idx():
+    return W.routed_indices("dsv3_prefill", device=DEV)
 
 
 @pytest.fixture(scope="module")
-def c5_idx():
+def hbm_idx():
     torch.cuda.empty_cache()
-    return W.routed_indices(5, device=DEV)
+    return W.routed_indices("hbm_stream", device=DEV)
 
 
 # ------------------------------------------------------------------ count --
 
-@pytest.mark.parametrize("cfg", [1, 2, 5])
-def test_count_configs(cfg, request):
-    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
-    E = W.CONFIGS[cfg].E
+@pytest.mark.parametrize("cfg", ["tiny", "dsv3_prefill", "hbm_stream"])
+def test_count_workloads(cfg, request):
+    idx = request.getfixturevalue({"tiny": "tiny_idx", "dsv3_prefill": "dsv3_idx", "hbm_stream": "hbm_idx"}[cfg])
+    E = W.WORKLOADS[cfg].E
     bad = torch.zeros(1, dtype=torch.int64, device=DEV)
     counts = eplb.count_loads(idx, E, bad=bad)
     ref, nbad = oracle.count_loads(_np(idx), E)
@@ -137,14 +137,14 @@ def test_count_misaligned_pointer_rejected():
 # ----------------------------------------------------------------- window --
 
 @pytest.fixture(scope="module")
-def c4_steps():
-    return W.c4_steps(device=DEV)
+def sweep_steps():
+    return W.window_sweep_steps(device=DEV)
 
 
 @pytest.mark.parametrize("window", [1000, 128, 1])
-def test_window_c4(c4_steps, window):
-    snaps = eplb.window_accumulate(c4_steps, window)
-    ref = oracle.window(_np(c4_steps), window)
+def test_window_sweep(sweep_steps, window):
+    snaps = eplb.window_accumulate(sweep_steps, window)
+    ref = oracle.window(_np(sweep_steps), window)
     assert np.array_equal(_np(snaps), ref)
 
 
@@ -176,10 +176,10 @@ def test_rebalance_readme_example():
     assert _np(plan.phy2log).tolist() == ex["phy2log"]["value"]
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 5])
+@pytest.mark.parametrize("cfg", ["tiny", "dsv3_prefill", "hbm_stream"])
 def test_rebalance_on_counted_loads(cfg, request):
-    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
-    c = W.CONFIGS[cfg]
+    idx = request.getfixturevalue({"tiny": "tiny_idx", "dsv3_prefill": "dsv3_idx", "hbm_stream": "hbm_idx"}[cfg])
+    c = W.WORKLOADS[cfg]
     loads = _np(eplb.count_loads(idx, c.E))
     plan, ref, st = _rebalance_both(loads, c.P, c.G, c.N, c.gpus)
     assert st == 0
@@ -187,17 +187,17 @@ def test_rebalance_on_counted_loads(cfg, request):
     check_plan(loads[:4], *(p[:4] for p in ref), c.P, c.G, c.N, c.gpus)
 
 
-def test_rebalance_c3_global():
-    c = W.CONFIGS[3]
-    loads = W.c3_loads()
+def test_rebalance_global_policy():
+    c = W.GLOBAL_POLICY
+    loads = W.global_policy_loads()
     plan, ref, st = _rebalance_both(loads, c.P, c.G, c.N, c.gpus)
     assert st == 0
     _assert_plan_equal(plan, ref)
 
 
-def test_rebalance_c4_sweep(c4_steps):
-    c = W.CONFIGS[4]
-    snaps = eplb.window_accumulate(c4_steps, c.W)
+def test_rebalance_window_sweep_rows(sweep_steps):
+    c = W.WINDOW_SWEEP
+    snaps = eplb.window_accumulate(sweep_steps, c.W)
     loads = _np(snaps).reshape(-1, c.E)
     plan, ref, st = _rebalance_both(loads, c.P, c.G, c.N, c.gpus)
     assert st == 0
@@ -313,10 +313,10 @@ def test_rebalance_host_errors():
 
 # --------------------------------------------------------------- redirect --
 
-@pytest.mark.parametrize("cfg", [1, 2, 5])
-def test_redirect_configs(cfg, request):
-    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
-    c = W.CONFIGS[cfg]
+@pytest.mark.parametrize("cfg", ["tiny", "dsv3_prefill", "hbm_stream"])
+def test_redirect_workloads(cfg, request):
+    idx = request.getfixturevalue({"tiny": "tiny_idx", "dsv3_prefill": "dsv3_idx", "hbm_stream": "hbm_idx"}[cfg])
+    c = W.WORKLOADS[cfg]
     counts = eplb.count_loads(idx, c.E)
     plan = eplb.rebalance(counts, c.P, c.G, c.N, c.gpus)
     bad = torch.zeros(1, dtype=torch.int64, device=DEV)
@@ -386,14 +386,14 @@ def test_redirect_arbitrary_tables(E, X, K, fused):
     assert int(bad.item()) == nbad and int(st.item()) == 0
 
 
-def test_redirect_sharded_equals_whole(c2_idx):
-    c = W.CONFIGS[2]
-    counts = eplb.count_loads(c2_idx, c.E)
+def test_redirect_sharded_equals_whole(dsv3_idx):
+    c = W.DSV3_PREFILL
+    counts = eplb.count_loads(dsv3_idx, c.E)
     plan = eplb.rebalance(counts, c.P, c.G, c.N, c.gpus)
-    whole = eplb.redirect(c2_idx, plan.log2phy, plan.logcnt)
+    whole = eplb.redirect(dsv3_idx, plan.log2phy, plan.logcnt)
     h = c.T // 2
-    a = eplb.redirect(c2_idx[:, :h].contiguous(), plan.log2phy, plan.logcnt, 0)
-    b = eplb.redirect(c2_idx[:, h:].contiguous(), plan.log2phy, plan.logcnt, h)
+    a = eplb.redirect(dsv3_idx[:, :h].contiguous(), plan.log2phy, plan.logcnt, 0)
+    b = eplb.redirect(dsv3_idx[:, h:].contiguous(), plan.log2phy, plan.logcnt, h)
     assert torch.equal(torch.cat([a, b], dim=1), whole)
 
 
@@ -404,11 +404,11 @@ def _plan_in_force(c, seed):
     return eplb.rebalance(loads, c.P, c.G, c.N, c.gpus)
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 5])
-def test_count_redirect_configs(cfg, request):
-    idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx", 5: "c5_idx"}[cfg])
-    c = W.CONFIGS[cfg]
-    plan = _plan_in_force(c, 100 + cfg)
+@pytest.mark.parametrize("cfg", ["tiny", "dsv3_prefill", "hbm_stream"])
+def test_count_redirect_workloads(cfg, request):
+    idx = request.getfixturevalue({"tiny": "tiny_idx", "dsv3_prefill": "dsv3_idx", "hbm_stream": "hbm_idx"}[cfg])
+    c = W.WORKLOADS[cfg]
+    plan = _plan_in_force(c, 100 + c.stream)
     bad = torch.zeros(1, dtype=torch.int64, device=DEV)
     st = _status()
     counts, out = eplb.count_redirect(idx, c.E, plan.log2phy, plan.logcnt, bad=bad, status=st)
@@ -451,30 +451,30 @@ def _oracle_plan_from_ring(ring, c, X):
     return oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=X)
 
 
-def test_pipeline_fresh_order_c2(c2_idx):
+def test_pipeline_fresh_order_dsv3_prefill(dsv3_idx):
     from moe_expert_load_eplb_b200.pipeline import EplbStep
-    c = W.CONFIGS[2]
-    hist = W.histogram_steps(15, c.L, c.E, c.T * c.K, 2, device=DEV)
+    c = W.DSV3_PREFILL
+    hist = W.histogram_steps(15, c.L, c.E, c.T * c.K, c.stream, device=DEV)
     step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=16, device=DEV, fused=False)
     step.fill_history(hist)
-    plan, out = step(c2_idx)
+    plan, out = step(dsv3_idx)
     torch.cuda.synchronize()
     assert int(step.status.item()) == 0
-    counts, _ = oracle.count_loads(_np(c2_idx), c.E)
+    counts, _ = oracle.count_loads(_np(dsv3_idx), c.E)
     ref = _oracle_plan_from_ring(np.concatenate([_np(hist), counts[None]], axis=0), c, step.X)
     _assert_plan_equal(plan, ref)
-    red, _ = oracle.redirect(_np(c2_idx), ref[3], ref[2])
+    red, _ = oracle.redirect(_np(dsv3_idx), ref[3], ref[2])
     assert np.array_equal(_np(out), red)
 
 
 @pytest.mark.parametrize("single", [True, False])
-def test_pipeline_serving_order_c2(c2_idx, single):
+def test_pipeline_serving_order_dsv3_prefill(dsv3_idx, single):
     """Three serving steps: each redirects with the plan in force, then rebuilds it
     (one launch per step, or count_redirect + rebalance_window)."""
     from moe_expert_load_eplb_b200.pipeline import EplbStep
-    c = W.CONFIGS[2]
+    c = W.DSV3_PREFILL
     W_ = 4
-    hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, 2, device=DEV)
+    hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, c.stream, device=DEV)
     step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV, fused=True,
                     token_offset=1000, single_launch=single)
     assert step.launches_per_step == (1 if single else 2)
@@ -482,7 +482,7 @@ def test_pipeline_serving_order_c2(c2_idx, single):
     ring = np.concatenate([_np(hist), np.zeros((1, c.L, c.E), np.int64)], axis=0)
     plan_ref = _oracle_plan_from_ring(ring, c, step.X)
     _assert_plan_equal(step.plan, plan_ref)
-    batches = [c2_idx, W.routed_indices(2, device=DEV, shard=1), c2_idx.flip(1).contiguous()]
+    batches = [dsv3_idx, W.routed_indices("dsv3_prefill", device=DEV, shard=1), dsv3_idx.flip(1).contiguous()]
     for s_i, idx in enumerate(batches):
         used, out = step(idx)
         torch.cuda.synchronize()
@@ -497,7 +497,7 @@ def test_pipeline_serving_order_c2(c2_idx, single):
         assert int(step.layer_done.abs().sum().item()) == 0
 
 
-def test_pipeline_serving_with_an_nccl_group_of_one(c1_idx):
+def test_pipeline_serving_with_an_nccl_group_of_one(tiny_idx):
     """The multi-rank serving step (count+redirect, NCCL all-reduce of the
     counts, window + rebalance) on a one-rank NCCL group: same plans and
     redirects as the oracle."""
@@ -511,16 +511,16 @@ def test_pipeline_serving_with_an_nccl_group_of_one(c1_idx):
                             device_id=torch.device(DEV))
     try:
         group = dist.new_group([0])
-        c = W.CONFIGS[1]
+        c = W.TINY
         W_ = 3
-        hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, 1, device=DEV)
+        hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, c.stream, device=DEV)
         step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV,
                         group=group, token_offset=77)
         assert step.launches_per_step == 2 and not step.single
         step.fill_history(hist)
         ring = np.concatenate([_np(hist), np.zeros((1, c.L, c.E), np.int64)], axis=0)
         plan_ref = _oracle_plan_from_ring(ring, c, step.X)
-        for s_i, idx in enumerate([c1_idx, c1_idx.flip(1).contiguous()]):
+        for s_i, idx in enumerate([tiny_idx, tiny_idx.flip(1).contiguous()]):
             used, out = step(idx)
             torch.cuda.synchronize()
             assert int(step.status.item()) == 0
@@ -534,21 +534,21 @@ def test_pipeline_serving_with_an_nccl_group_of_one(c1_idx):
 
 
 @pytest.mark.parametrize("fused,single", [(True, False), (True, True), (False, False)])
-def test_step_graphs_replay_matches_eager(c1_idx, fused, single):
+def test_step_graphs_replay_matches_eager(tiny_idx, fused, single):
     """CUDA-graph replay of the step (one graph per phase of the ring slot and
     plan buffer) gives exactly the eager steps' outputs, plans and ring."""
     from moe_expert_load_eplb_b200.pipeline import EplbStep, StepGraphs
-    c = W.CONFIGS[1]
-    hist = W.histogram_steps(2, c.L, c.E, c.T * c.K, 1, device=DEV)
+    c = W.TINY
+    hist = W.histogram_steps(2, c.L, c.E, c.T * c.K, c.stream, device=DEV)
     mk = lambda: EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=3, device=DEV,
                           fused=fused, single_launch=single, token_offset=5)
     eager, graphed = mk(), mk()
     eager.fill_history(hist)
     graphed.fill_history(hist)
-    buf = torch.empty_like(c1_idx)
+    buf = torch.empty_like(tiny_idx)
     sg = StepGraphs(graphed, buf)
     assert sg.period == 6
-    batches = [c1_idx, c1_idx.flip(1), c1_idx.roll(7, dims=1), (c1_idx + 3) % c.E]
+    batches = [tiny_idx, tiny_idx.flip(1), tiny_idx.roll(7, dims=1), (tiny_idx + 3) % c.E]
     for k in range(9):
         b = batches[k % len(batches)].contiguous()
         buf.copy_(b)
@@ -711,13 +711,13 @@ def _plans_for(c, loads_np):
     return oracle.rebalance(loads_np, c.P, c.G, c.N, c.gpus)
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3])
+@pytest.mark.parametrize("cfg", ["tiny", "dsv3_prefill", "global_policy"])
 def test_plan_stats_matches_oracle(cfg, request):
-    c = W.CONFIGS[cfg]
-    if cfg == 3:
-        loads_np = W.c3_loads()
+    c = W.WORKLOADS[cfg]
+    if cfg == "global_policy":
+        loads_np = W.global_policy_loads()
     else:
-        idx = request.getfixturevalue({1: "c1_idx", 2: "c2_idx"}[cfg])
+        idx = request.getfixturevalue({"tiny": "tiny_idx", "dsv3_prefill": "dsv3_idx"}[cfg])
         loads_np, _ = oracle.count_loads(_np(idx), c.E)
     p2l, _, cnt, _ = _plans_for(c, loads_np)
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
@@ -751,11 +751,11 @@ def test_fold_loads_matches_oracle(shape):
     assert np.array_equal(_np(got), oracle.fold_loads(phys, p2l, E))
 
 
-def test_fold_of_physical_counts_after_redirect(c2_idx):
-    c = W.CONFIGS[2]
-    counts = eplb.count_loads(c2_idx, c.E)
+def test_fold_of_physical_counts_after_redirect(dsv3_idx):
+    c = W.DSV3_PREFILL
+    counts = eplb.count_loads(dsv3_idx, c.E)
     plan = eplb.rebalance(counts, c.P, c.G, c.N, c.gpus)
-    out = eplb.redirect(c2_idx, plan.log2phy, plan.logcnt)
+    out = eplb.redirect(dsv3_idx, plan.log2phy, plan.logcnt)
     phys = eplb.count_loads(out, c.P)
     assert torch.equal(eplb.fold_loads(phys, plan.phy2log, c.E), counts)
 
@@ -766,14 +766,14 @@ def test_initial_map_matches_oracle():
     assert np.array_equal(_np(p2l), ref_p) and np.array_equal(_np(prk), ref_r)
 
 
-@pytest.mark.parametrize("cfg", [2, 3])
-def test_plan_diff_matches_oracle(cfg, c4_steps):
-    c = W.CONFIGS[cfg]
-    if cfg == 3:
-        old_l = W.c3_loads()
+@pytest.mark.parametrize("cfg", ["dsv3_prefill", "global_policy"])
+def test_plan_diff_matches_oracle(cfg, sweep_steps):
+    c = W.WORKLOADS[cfg]
+    if cfg == "global_policy":
+        old_l = W.global_policy_loads()
         new_l = np.roll(old_l, 1, axis=1)
     else:
-        snaps = _np(c4_steps)
+        snaps = _np(sweep_steps)
         old_l, new_l = snaps[10], snaps[900]
     old = _plans_for(c, old_l)[0]
     new = _plans_for(c, new_l)[0]
@@ -783,10 +783,10 @@ def test_plan_diff_matches_oracle(cfg, c4_steps):
     assert np.array_equal(_np(src), ref_src) and np.array_equal(_np(moves), ref_moves)
 
 
-def test_plan_diff_initial_to_first_plan(c2_idx):
-    c = W.CONFIGS[2]
+def test_plan_diff_initial_to_first_plan(dsv3_idx):
+    c = W.DSV3_PREFILL
     init, _ = eplb.initial_map(c.L, c.E, c.P, device=DEV)
-    plan = eplb.rebalance(eplb.count_loads(c2_idx, c.E), c.P, c.G, c.N, c.gpus)
+    plan = eplb.rebalance(eplb.count_loads(dsv3_idx, c.E), c.P, c.G, c.N, c.gpus)
     src, moves = eplb.plan_diff(init, plan.phy2log, c.E, c.gpus)
     ref_src, ref_moves = oracle.plan_diff(_np(init), _np(plan.phy2log), c.E, c.gpus)
     assert np.array_equal(_np(src), ref_src) and np.array_equal(_np(moves), ref_moves)
@@ -796,7 +796,7 @@ def test_plan_diff_initial_to_first_plan(c2_idx):
 
 @pytest.mark.parametrize("W_,zero", [(16, 3), (1, -1), (4, 0), (7, -1)])
 def test_rebalance_window_matches_window_then_rebalance(W_, zero):
-    c = W.CONFIGS[2]
+    c = W.DSV3_PREFILL
     ring = W.histogram_steps(W_, c.L, c.E, c.T * c.K, 7, device=DEV).contiguous()
     ring_h = _np(ring).copy()
     loads_out = torch.empty((c.L, c.E), dtype=torch.int64, device=DEV)

@@ -6,14 +6,19 @@ describe, and is the only code that the CUDA path's tests, the bench and the
 CPU oracle share.
 """
 from .gen import (  # noqa: F401
-    CONFIGS,
-    Config,
-    c1_indices,
-    c3_loads,
-    c4_steps,
+    DSV3_PREFILL,
+    GLOBAL_POLICY,
+    HBM_STREAM,
+    TINY,
+    WINDOW_SWEEP,
+    WORKLOADS,
+    Workload,
+    global_policy_loads,
     group_limited_indices,
     histogram_steps,
     routed_indices,
     seed_for,
+    tiny_indices,
+    window_sweep_steps,
     zipf_indices,
 )

@@ -18,14 +18,15 @@ import torch
 BASE_SEED = 20250227
 
 
-def seed_for(config: int, sub: int = 0) -> int:
-    """Seed of sub-stream ``sub`` (layer, step, ...) of workload ``config``."""
-    return BASE_SEED + 1000 * config + sub
+def seed_for(stream: int, sub: int = 0) -> int:
+    """Seed of sub-stream ``sub`` (layer, step, ...) of seed stream ``stream``
+    (each workload draws from its own stream, ``Workload.stream``)."""
+    return BASE_SEED + 1000 * stream + sub
 
 
 @dataclass(frozen=True)
-class Config:
-    index: int
+class Workload:
+    stream: int     # seed stream (seed_for)
     name: str
     L: int          # MoE layers (rows of one rebalance call)
     E: int          # logical experts per layer
@@ -50,13 +51,16 @@ class Config:
         return (self.P - self.E) // n + 1
 
 
-CONFIGS = {
-    1: Config(1, "tiny_hierarchical", L=2, E=12, G=4, P=16, N=2, gpus=8, T=4096, K=2),
-    2: Config(2, "dsv3_prefill_hierarchical", L=58, E=256, G=8, P=288, N=4, gpus=32, T=65536, K=8),
-    3: Config(3, "global_policy", L=58, E=256, G=1, P=288, N=2, gpus=144),
-    4: Config(4, "window_sweep", L=58, E=256, G=8, P=288, N=4, gpus=32, T=8192, K=8, S=1000, W=1000),
-    5: Config(5, "hbm_stream", L=58, E=256, G=8, P=288, N=4, gpus=32, T=1048576, K=8),
-}
+# The workloads by name: the pages' worked-example sizes, DeepSeek-V3-shaped
+# prefill, the global policy over 144 GPUs, a 1000-step window sweep, and a
+# 16x larger routed batch that streams ~2 GB of indices.
+TINY = Workload(1, "tiny", L=2, E=12, G=4, P=16, N=2, gpus=8, T=4096, K=2)
+DSV3_PREFILL = Workload(2, "dsv3_prefill", L=58, E=256, G=8, P=288, N=4, gpus=32, T=65536, K=8)
+GLOBAL_POLICY = Workload(3, "global_policy", L=58, E=256, G=1, P=288, N=2, gpus=144)
+WINDOW_SWEEP = Workload(4, "window_sweep", L=58, E=256, G=8, P=288, N=4, gpus=32, T=8192, K=8,
+                        S=1000, W=1000)
+HBM_STREAM = Workload(5, "hbm_stream", L=58, E=256, G=8, P=288, N=4, gpus=32, T=1048576, K=8)
+WORKLOADS = {w.name: w for w in (TINY, DSV3_PREFILL, GLOBAL_POLICY, WINDOW_SWEEP, HBM_STREAM)}
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -65,7 +69,7 @@ def _gen(seed: int, device) -> torch.Generator:
     return g
 
 
-def zipf_indices(L: int, T: int, K: int, E: int, s: float, config: int, device="cpu") -> torch.Tensor:
+def zipf_indices(L: int, T: int, K: int, E: int, s: float, stream: int, device="cpu") -> torch.Tensor:
     """int32 [L, T, K]: per layer, expert popularity p_r ∝ r^-s over ranks r = 1..E
     mapped to experts through a seeded permutation; each token draws K distinct
     experts (sampling without replacement, as a router's top-k is distinct)."""
@@ -73,7 +77,7 @@ def zipf_indices(L: int, T: int, K: int, E: int, s: float, config: int, device="
     ranks = torch.arange(1, E + 1, dtype=torch.float64)
     base = ranks.pow(-s)
     for l in range(L):
-        g = _gen(seed_for(config, l), "cpu")
+        g = _gen(seed_for(stream, l), "cpu")
         perm = torch.randperm(E, generator=g)
         p = torch.empty(E, dtype=torch.float64)
         p[perm] = base / base.sum()
@@ -83,10 +87,10 @@ def zipf_indices(L: int, T: int, K: int, E: int, s: float, config: int, device="
     return out
 
 
-def c1_indices(device="cpu") -> torch.Tensor:
-    """Tiny config: 2 layers x 4096 tokens x top-2 over 12 experts, Zipf(s=1.2)."""
-    c = CONFIGS[1]
-    return zipf_indices(c.L, c.T, c.K, c.E, 1.2, 1, device)
+def tiny_indices(device="cpu") -> torch.Tensor:
+    """Tiny workload: 2 layers x 4096 tokens x top-2 over 12 experts, Zipf(s=1.2)."""
+    c = TINY
+    return zipf_indices(c.L, c.T, c.K, c.E, 1.2, c.stream, device)
 
 
 def group_limited_indices(popularity: torch.Tensor, T: int, K: int, G: int, groups_per_token: int,
@@ -117,38 +121,39 @@ def group_limited_indices(popularity: torch.Tensor, T: int, K: int, G: int, grou
     return out
 
 
-def routed_indices(config: int, device="cpu", T: int | None = None, L: int | None = None,
+def routed_indices(workload: str, device="cpu", T: int | None = None, L: int | None = None,
                    shard: int = 0) -> torch.Tensor:
-    """Routed indices of configs 2 and 5 (optionally with fewer tokens / layers).
+    """Routed indices of the dsv3_prefill and hbm_stream workloads (optionally
+    with fewer tokens / layers).
 
-    Config 2: popularity LogNormal(mu=0, sigma=1) per expert per layer.
-    Config 5: popularity ∝ rank^-1.0 (Zipf s=1.0) through a seeded permutation.
+    dsv3_prefill: popularity LogNormal(mu=0, sigma=1) per expert per layer.
+    hbm_stream: popularity ∝ rank^-1.0 (Zipf s=1.0) through a seeded permutation.
     Both: 8 groups of 32, 4 groups per token, top-8.  ``shard`` selects an
     independent token stream with the same popularity (one per data-parallel
     rank).
     """
-    c = CONFIGS[config]
+    c = WORKLOADS[workload]
     L = c.L if L is None else L
     T = c.T if T is None else T
-    g = _gen(seed_for(config, 999), "cpu")
-    if config == 2:
+    g = _gen(seed_for(c.stream, 999), "cpu")
+    if c is DSV3_PREFILL:
         pop = torch.empty((L, c.E), dtype=torch.float64).log_normal_(0.0, 1.0, generator=g)
-    elif config == 5:
+    elif c is HBM_STREAM:
         base = torch.arange(1, c.E + 1, dtype=torch.float64).pow(-1.0)
         pop = torch.stack([base[torch.randperm(c.E, generator=g)] for _ in range(L)])
     else:
-        raise ValueError("routed indices exist for configs 2 and 5")
-    return group_limited_indices(pop.float(), T, c.K, c.G, 4, seed_for(config, 0) + 100000 * shard,
-                                 device)
+        raise ValueError("routed indices exist for dsv3_prefill and hbm_stream")
+    return group_limited_indices(pop.float(), T, c.K, c.G, 4,
+                                 seed_for(c.stream, 0) + 100000 * shard, device)
 
 
-def c3_loads(L: int = 58, E: int = 256) -> np.ndarray:
-    """Config 3: loads int64 [L, E] = round(1e4 * Pareto(alpha=1.5)), x_m = 1."""
-    rng = np.random.default_rng(seed_for(3))
+def global_policy_loads(L: int = 58, E: int = 256) -> np.ndarray:
+    """global_policy workload: loads int64 [L, E] = round(1e4 * Pareto(alpha=1.5)), x_m = 1."""
+    rng = np.random.default_rng(seed_for(GLOBAL_POLICY.stream))
     return np.round(1e4 * (rng.pareto(1.5, size=(L, E)) + 1.0)).astype(np.int64)
 
 
-def histogram_steps(S: int, L: int, E: int, draws: int, config: int, sigma: float = 0.05,
+def histogram_steps(S: int, L: int, E: int, draws: int, stream: int, sigma: float = 0.05,
                     device="cpu") -> torch.Tensor:
     """int64 [S, L, E]: per step, the histogram of ``draws`` expert choices.
 
@@ -157,7 +162,7 @@ def histogram_steps(S: int, L: int, E: int, draws: int, config: int, sigma: floa
     ``draws`` choices from softmax(log-popularity), sampled exactly as a
     chain of conditional binomials (counts add up to ``draws``).
     """
-    g = _gen(seed_for(config, 0), device)
+    g = _gen(seed_for(stream, 0), device)
     theta = torch.randn((1, L, E), generator=g, device=device, dtype=torch.float64)
     walk = torch.randn((S, L, E), generator=g, device=device, dtype=torch.float64) * sigma
     walk[0] = 0
@@ -176,7 +181,8 @@ def histogram_steps(S: int, L: int, E: int, draws: int, config: int, sigma: floa
     return counts.view(S, L, E)
 
 
-def c4_steps(device="cpu", S: int | None = None) -> torch.Tensor:
-    """Config 4: 1000 steps x 58 layers x 256 experts, 8192 tokens x top-8 per step."""
-    c = CONFIGS[4]
-    return histogram_steps(c.S if S is None else S, c.L, c.E, c.T * c.K, 4, device=device)
+def window_sweep_steps(device="cpu", S: int | None = None) -> torch.Tensor:
+    """window_sweep workload: 1000 steps x 58 layers x 256 experts, 8192 tokens
+    x top-8 per step."""
+    c = WINDOW_SWEEP
+    return histogram_steps(c.S if S is None else S, c.L, c.E, c.T * c.K, c.stream, device=device)
