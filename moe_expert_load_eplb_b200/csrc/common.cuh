@@ -40,6 +40,13 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Brings the 128-byte line holding p into L2.  It reads nothing into the
+// thread and L2 is the point of coherence for global memory, so it may be
+// issued before pdl_wait, even on data the previous grid is still writing.
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // x mod d for 0 <= x < 2^31 and 1 <= d < 2^31 with m = floor((2^32-1)/d):
 // q = floor(x*m / 2^32) undershoots floor(x/d) by at most 1 (the deficit
 // x*(2^32/d - m)/2^32 < 2x/2^32 < 1), so one conditional subtraction fixes

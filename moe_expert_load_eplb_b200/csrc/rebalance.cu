@@ -11,6 +11,15 @@ template <bool kCap2>
 __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
   pdl_trigger();
+  // warm L2 with this row's ring rows while the previous kernel finishes:
+  // the row's first phase sums them (one 128-byte line per thread)
+  {
+    const int E = a.s.E;
+    const int lines = (E + 15) >> 4;  // 16 int64 per line
+    const int64_t *row = a.ring + static_cast<int64_t>(blockIdx.x) * E;
+    for (int64_t w = 0; w < a.ring_w; ++w, row += a.ring_stride)
+      for (int j = threadIdx.x; j < lines; j += blockDim.x) prefetch_l2(row + min(j << 4, E - 1));
+  }
   pdl_wait();
   rebalance_row<kCap2>(a, blockIdx.x, smem);
 }
