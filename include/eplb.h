@@ -49,7 +49,7 @@ typedef enum eplb_status {
   EPLB_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed */
   EPLB_ERR_TIMEOUT = 7,       /* reserved: an in-kernel wait gave up (no current kernel waits) */
   EPLB_ERR_ALIGN = 8,         /* a pointer lacks the alignment stated below */
-  EPLB_ERR_LIMIT = 9          /* a size beyond this build's stated limits */
+  EPLB_ERR_LIMIT = 9          /* a size beyond the limits stated in this header */
 } eplb_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
