@@ -180,13 +180,15 @@ def _traffic(kernel_file: str, profile: str, scale: float):
 STAGES = ("count", "allreduce", "window", "rebalance", "redirect")
 
 
-def _timed_steps(step, idx, flush, K, group, dev, staged=False):
+def _timed_steps(step, idx, flush, K, group, dev, staged=False, scrub=None):
     """Runs K steps, each between a start and an end event (the L2 flush
     before each step stays outside them); returns (total ms, max over ranks,
     per-stage mean ms or None, clock summary).  With ``staged`` the step also
     records events between its stages for the per-stage breakdown -- those
     extra records cost time of their own, so the headline is taken without
-    them."""
+    them.  ``scrub`` (a buffer larger than L2): read after the flush write,
+    so that L2 holds clean lines and none of the flush's dirty lines is
+    written back inside the timed step."""
     n_ev = 6 if staged else 2
     marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
     if group is not None:
@@ -195,6 +197,8 @@ def _timed_steps(step, idx, flush, K, group, dev, staged=False):
     with ClockSampler(dev.index) as clocks:
         for i in range(K):
             flush.fill_(i & 0xff)
+            if scrub is not None:
+                scrub.max()
             if staged:
                 step(idx, marks[i])
             else:
@@ -314,6 +318,26 @@ def run_ours(args, rank: int, world: int, group):
            "gpu_launches": step.launches_per_step * K,
            "tokens_per_s": round(world * c.T * K / (total_ms / 1e3), 1),
            "stages": stages, "roofline": roof, "clocks": clocks}
+
+    # ---- the same step after a clean flush, one GPU only --------------------
+    # The headline's flush (a 512 MB write) leaves L2 full of dirty lines that
+    # are written back while the timed step runs.  Here a 256 MB read follows
+    # the write, so L2 starts the step holding clean lines of another buffer,
+    # as ncu's cold-cache replays do (they write back and invalidate L2).
+    if world == 1 and not args.no_fresh:
+        scrub = torch.zeros(FLUSH_BYTES // 2, dtype=torch.uint8, device=dev)
+        Kc = max(3, min(K, 500))
+        c_total, _, _ = _timed_steps(step, idx, flush, Kc, group, dev, scrub=scrub)
+        _, c_stage, _ = _timed_steps(step, idx, flush, Kc, group, dev, staged=True, scrub=scrub)
+        check(step, "clean-flush steps")
+        cst = _stage_report(c_stage, True, step.X, world, hbm_peak)
+        out["clean_l2"] = {
+            "steps": Kc, "ms_per_step": round(c_total / Kc, 5),
+            "value": round(c.L * Kc / (c_total / 1e3), 1),
+            "l2": "512 MB write, then a 256 MB read (clean lines), between steps",
+            "count_redirect": {k: cst["count"][k] for k in ("ms", "gbs", "frac_hbm")},
+            "rebalance_ms": cst["rebalance"]["ms"]}
+        del scrub
 
     # ---- the same step in one launch (serve_step), one GPU only -------------
     if world == 1 and not args.no_fresh:
