@@ -94,6 +94,31 @@ class EplbStep:
         self._plan_from_ring(self.plans[self.cur])
         self.primed = True
 
+    def state_dict(self) -> dict:
+        """The step's state, copied to the host: the ring of per-step counts,
+        the plan in force, the number of steps done.  A step restored from it
+        (``load_state_dict``, on any device) continues bit for bit as this one
+        would: the plan is an exact function of the ring, and the ring and the
+        step count are all the window keeps."""
+        return {"shape": self._shape(), "steps_done": self.steps_done, "primed": self.primed,
+                "cur": self.cur, "token_offset": self.token_offset,
+                "ring": self.ring.cpu(), "plan": [t.cpu() for t in self.plans[self.cur]]}
+
+    def load_state_dict(self, state: dict):
+        """Restore a state taken by ``state_dict`` from a step of the same shape."""
+        if tuple(state["shape"]) != self._shape():
+            raise ValueError(f"state of shape {tuple(state['shape'])}, step of shape {self._shape()}")
+        self.ring.copy_(state["ring"])
+        self.cur = int(state["cur"])
+        for dst, src in zip(self.plans[self.cur], state["plan"]):
+            dst.copy_(src)
+        self.steps_done = int(state["steps_done"])
+        self.primed = bool(state["primed"])
+        self.token_offset = int(state["token_offset"])
+
+    def _shape(self):
+        return (self.L, self.T, self.K, self.E, self.P, self.G, self.N, self.gpus, self.W, self.X)
+
     def _plan_from_ring(self, plan: Plan):
         window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads, status=self.status)
         rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=plan,

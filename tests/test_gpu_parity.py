@@ -564,6 +564,97 @@ def test_step_graphs_replay_matches_eager(tiny_idx, fused, single):
     assert int(graphed.status.item()) == 0
 
 
+@pytest.mark.parametrize("single", [False, True])
+def test_pipeline_checkpoint_resume(tiny_idx, single):
+    """A step restored mid-sweep from state_dict (through torch.save) continues
+    exactly as the step it was taken from: outputs, plans and ring."""
+    import io
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+    c = W.TINY
+    W_ = 3
+    hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, c.stream, device=DEV)
+    mk = lambda: EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV,
+                          fused=True, single_launch=single)
+    batches = [tiny_idx, tiny_idx.flip(1).contiguous(), tiny_idx.roll(1, 2).contiguous(),
+               tiny_idx.flip(2).contiguous(), tiny_idx.roll(7, 1).contiguous()]
+    a = mk()
+    a.fill_history(hist)
+    for b in batches[:2]:
+        a(b)
+    buf = io.BytesIO()
+    torch.save(a.state_dict(), buf)
+    buf.seek(0)
+    ref = []
+    for b in batches[2:]:
+        _, out = a(b)
+        ref.append((out.clone(), [t.clone() for t in a.plan]))
+    r = mk()
+    r.load_state_dict(torch.load(buf))
+    for b, (out_ref, plan_ref) in zip(batches[2:], ref):
+        _, out = r(b)
+        assert torch.equal(out, out_ref)
+        for x, y in zip(r.plan, plan_ref):
+            assert torch.equal(x, y)
+    assert torch.equal(r.ring, a.ring)
+    assert int(a.status.item()) == 0 and int(r.status.item()) == 0
+
+
+# ---------------------------------------------------------- guard bands --
+
+_GUARD = 64  # elements on each side (256 B for int32: keeps 16-byte alignment)
+
+
+def _guarded(shape, dtype, fill=-7):
+    n = int(np.prod(shape))
+    buf = torch.full((n + 2 * _GUARD,), fill, dtype=dtype, device=DEV)
+    return buf, buf[_GUARD:_GUARD + n].view(shape)
+
+
+def _intact(buf, fill=-7):
+    return bool((buf[:_GUARD] == fill).all()) and bool((buf[-_GUARD:] == fill).all())
+
+
+@pytest.mark.parametrize("shape", [(3, 1001, 3, 12, 16, 4, 2, 8), (2, 70001, 5, 256, 288, 8, 4, 32),
+                                   (1, 1, 1, 12, 16, 4, 2, 8), (5, 3, 7, 24, 40, 6, 2, 4)])
+def test_outputs_stay_inside_their_buffers(shape):
+    """Every entry point writing caller-owned memory, on ragged shapes, leaves
+    guard bands around each output untouched."""
+    L, T, K, E, P, G, N, gpus = shape
+    X = P - E + 1
+    rng = np.random.default_rng(T + E)
+    idx = _dev(rng.integers(-1, E + 1, (L, T, K)).astype(np.int32))
+    bufs = []
+
+    def g(shape_, dtype):
+        b, t = _guarded(shape_, dtype)
+        bufs.append(b)
+        return t
+
+    def gplan():
+        return eplb.Plan(g((L, P), torch.int32), g((L, P), torch.int32), g((L, E), torch.int32),
+                         g((L, E, X), torch.int32))
+
+    st = _status()
+    counts = eplb.count_loads(idx, E, counts=g((L, E), torch.int64), status=st)
+    plan = eplb.rebalance(counts, P, G, N, gpus, slots=X, out=gplan(), status=st)
+    eplb.redirect(idx, plan.log2phy, plan.logcnt, 5, out=g((L, T, K), torch.int32), status=st)
+    eplb.count_redirect(idx, E, plan.log2phy, plan.logcnt, 5, counts=g((L, E), torch.int64),
+                        out=g((L, T, K), torch.int32), status=st)
+    steps = _dev(rng.integers(0, 1000, (4, L, E)).astype(np.int64))
+    eplb.window_accumulate(steps, 2, out=g((4, L, E), torch.int64), status=st)
+    ring = g((3, L, E), torch.int64)
+    ring.copy_(steps[:3])
+    eplb.rebalance_window(ring, P, G, N, gpus, zero_slot=1, slots=X, out=gplan(),
+                          loads_out=g((L, E), torch.int64), status=st)
+    done = g((L,), torch.int32)
+    done.zero_()
+    eplb.serve_step(idx, plan, ring, 1, gplan(), done, G, N, gpus, zero_slot=2, token_offset=9,
+                    out=g((L, T, K), torch.int32), loads_out=g((L, E), torch.int64), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert all(_intact(b) for b in bufs)
+
+
 # ------------------------------------------------------- one-launch serve step --
 
 def _dev(a):
