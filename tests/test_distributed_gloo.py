@@ -88,22 +88,25 @@ def test_token_shards_cover_and_balance():
             assert max(sizes) - min(sizes) <= 1
 
 
-def test_two_ranks_sum_loads_and_agree_on_the_plan():
+@pytest.mark.parametrize("world", [2, 3])
+def test_ranks_sum_loads_and_agree_on_the_plan(world):
+    """World 3 splits the 1001 tokens unevenly (334, 334, 333)."""
     import oracle
-    results, (L, T, K, E, P, G, N, gpus) = _run(2)
-    assert set(results) == {0, 1}, results
-    for r in (0, 1):
+    results, (L, T, K, E, P, G, N, gpus) = _run(world)
+    ranks = tuple(range(world))
+    assert set(results) == set(ranks), results
+    for r in ranks:
         assert results[r][0] == "ok", results[r]
     rng = np.random.default_rng(123)
     idx = rng.integers(0, E, (L, T, K)).astype(np.int32)
     counts, _ = oracle.count_loads(idx, E)
     plan = oracle.rebalance(counts, P, G, N, gpus)
     full, _ = oracle.redirect(idx, plan[3], plan[2], 0)
-    for r in (0, 1):
+    for r in ranks:
         assert np.array_equal(np.array(results[r][1]), counts)
         for got, want in zip(results[r][2], plan):
             assert np.array_equal(np.array(got), want)
-    shards = sorted((results[r][4], np.array(results[r][3])) for r in (0, 1))
+    shards = sorted((results[r][4], np.array(results[r][3])) for r in ranks)
     assert np.array_equal(np.concatenate([s for _, s in shards], axis=1), full)
 
 
