@@ -92,3 +92,24 @@ def test_binding_fails_loudly_without_a_gpu_tensor():
     import moe_expert_load_eplb_b200 as eplb
     with pytest.raises(TypeError):
         eplb.count_loads(torch.zeros((1, 4, 2), dtype=torch.int32), 8)
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No CPU fallback: without libeplb.so every call raises."""
+    import moe_expert_load_eplb_b200 as eplb
+    monkeypatch.setattr(eplb, "_lib", None)
+    monkeypatch.setattr(eplb, "_LIB_PATH", "/nonexistent/libeplb.so")
+    with pytest.raises(ImportError, match="build"):
+        eplb.load_library()
+
+
+def test_host_tensors_are_refused():
+    """The binding never computes on host tensors: it refuses them."""
+    import torch
+
+    import moe_expert_load_eplb_b200 as eplb
+    idx = torch.zeros((1, 4, 2), dtype=torch.int32)
+    with pytest.raises(TypeError, match="CUDA"):
+        eplb.count_loads(idx, 8)
+    with pytest.raises(TypeError, match="CUDA"):
+        eplb.rebalance(torch.zeros((1, 8), dtype=torch.int64), 8, 1, 1, 1)
