@@ -458,8 +458,12 @@ void oracle_fold_loads(const int64_t *phys, const int32_t *phy2log, int64_t R, i
     for (int p = 0; p < P; ++p) logical[r * E + phy2log[r * P + p]] += phys[r * P + p];
 }
 
-/* Initial map: routed experts first, then the redundant slots cycle through */
-/* the experts from 0 (phy2log[p] = p mod E, phyrank[p] = p div E).          */
+/* Initial map, the plan before any load is measured: the physical experts  */
+/* are the routed ones followed by the redundant ones (vLLM eplb_state        */
+/* glossary), and with every expert taken as equally loaded replicate_experts */
+/* gives each redundant slot to the lowest-index expert with the fewest       */
+/* replicas, so the redundant slots cycle through the experts from 0:         */
+/* phy2log[p] = p mod E, phyrank[p] = p div E.                                */
 void oracle_initial_map(int64_t R, int32_t E, int32_t P, int32_t *phy2log, int32_t *phyrank) {
   for (int64_t r = 0; r < R; ++r)
     for (int p = 0; p < P; ++p) {

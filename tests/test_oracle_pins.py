@@ -442,9 +442,45 @@ def test_fold_of_redirected_counts_is_the_logical_count():
     assert (oracle.fold_loads(phys, p2l, E) == logical).all()
 
 
-def test_initial_map_closed_form():
-    p2l, prk = oracle.initial_map(3, 256, 288)
-    assert (p2l == np.arange(288) % 256).all() and (prk == np.arange(288) // 256).all()
+@pytest.mark.parametrize("E,P", [(256, 288), (12, 16), (4, 13), (1, 5), (7, 7), (32, 100)])
+def test_initial_map_routed_experts_first(E, P):
+    # vLLM eplb_state glossary prose: the physical experts are the routed
+    # (logical) experts followed by the redundant ones (256 routed + 32
+    # redundant = 288 on DeepSeek-V3), so slot p < E holds expert p, rank 0
+    p2l, prk = oracle.initial_map(2, E, P)
+    assert (p2l[:, :E] == np.arange(E)).all() and (prk[:, :E] == 0).all()
+
+
+@pytest.mark.parametrize("E,P", [(256, 288), (12, 16), (4, 13), (1, 5), (7, 7), (32, 100)])
+def test_initial_map_is_a_valid_plan(E, P):
+    # every slot names an expert, every expert has a replica, and a slot's
+    # rank counts the earlier slots of its expert (ranks 0 .. cnt-1 in slot
+    # order), so logcnt = bincount(phy2log) sums to P
+    p2l, prk = oracle.initial_map(3, E, P)
+    for r in range(3):
+        assert ((p2l[r] >= 0) & (p2l[r] < E)).all()
+        cnt = np.bincount(p2l[r], minlength=E)
+        assert cnt.sum() == P and (cnt >= 1).all()
+        seen = np.zeros(E, dtype=np.int64)
+        for p in range(P):
+            e = p2l[r, p]
+            assert prk[r, p] == seen[e]
+            seen[e] += 1
+
+
+@pytest.mark.parametrize("E,P", [(256, 288), (12, 16), (4, 13), (1, 5), (7, 7), (32, 100), (5, 23)])
+def test_initial_map_is_replicate_experts_on_equal_loads(E, P):
+    # Before any load is measured every expert is taken as equally loaded.
+    # The appendix's replicate_experts (pinned to textbook D'Hondt above)
+    # then hands each redundant slot to the lowest-index expert among those
+    # with the fewest replicas: the initial map's cycle from expert 0.  A
+    # different cycle (another start, a reversed order, two redundant slots
+    # for one expert before another gets its first) fails here.
+    p2l, prk = oracle.initial_map(1, E, P)
+    want_p2l, want_rank, want_cnt = oracle.replicate_experts(np.full(E, 1000, np.int64), P)
+    assert (p2l[0] == want_p2l).all() and (prk[0] == want_rank).all()
+    assert (np.bincount(p2l[0], minlength=E) == want_cnt).all()
+    assert want_cnt.max() - want_cnt.min() <= 1  # the redundant slots are spread evenly
 
 
 def test_plan_diff_identity_and_swap():
