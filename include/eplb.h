@@ -71,15 +71,13 @@ int32_t eplb_abi_version(void);
  *          are skipped and their number is added to *bad.
  * counts   device int64 [L, E]; overwritten (accumulate == 0) or added to.
  * bad      device uint64 word, nullable; added to, never cleared.
- * status   device int32 word, nullable; counting has no data-dependent error,
- *          so nothing is written to it (kept for a uniform signature).
+ * Counting has no data-dependent error: the call takes no status word.
  * Limits:  1 <= E <= 1024, K >= 1, 0 <= L < 2^31, T >= 0, T * K < 2^31.
  * Integer atomics make the result independent of scheduling.
  */
 eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K,
                              int32_t E, int64_t *counts, int32_t accumulate,
-                             unsigned long long *bad, int32_t *status,
-                             cudaStream_t stream);
+                             unsigned long long *bad, cudaStream_t stream);
 
 /*
  * S2 -- sliding-window accumulation.  [EPLB] "Алгоритм": expert load is
@@ -92,14 +90,14 @@ eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K
  * steps    device int64 [S, L, E].
  * snaps    device int64 [S - s_first, L, E]; must not overlap steps.
  * W >= 1 (W >= S gives running totals); 0 <= s_first < S.
- * Sums are exact; wrap-around of int64 is the caller's concern.
- * status   nullable; nothing is written to it (no data-dependent error).
+ * Sums are exact; wrap-around of int64 is the caller's concern.  No
+ * data-dependent error exists, so the call takes no status word.
  * With a ring buffer of the last W per-step counts, s_first = S - 1 = W - 1
  * returns the current window sum (row order does not change a full sum).
  */
 eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, int32_t E,
                                    int64_t W, int64_t s_first, int64_t *snaps,
-                                   int32_t *status, cudaStream_t stream);
+                                   cudaStream_t stream);
 
 /*
  * S3/S4 -- rebalance_experts over R independent rows ([EPLB] "Алгоритм",
@@ -281,8 +279,10 @@ eplb_status eplb_fold_loads(const int64_t *phys, const int32_t *phy2log, int64_t
                             int32_t P, int64_t *logical, int32_t *status, cudaStream_t stream);
 
 /*
- * The plan before any load is known: routed experts first, then the
- * redundant slots cycle through the experts from 0:
+ * The plan before any load is known (vLLM eplb_state glossary, context only:
+ * the routed experts in slots 0 .. E-1, then the redundant slots).  With every expert taken as
+ * equally loaded, replicate_experts gives each redundant slot to the
+ * lowest-index expert with the fewest replicas, so they cycle from expert 0:
  *   phy2log[r, p] = p mod E,  phyrank[r, p] = p div E  (phyrank nullable).
  */
 eplb_status eplb_initial_map(int64_t R, int32_t E, int32_t P, int32_t *phy2log, int32_t *phyrank,

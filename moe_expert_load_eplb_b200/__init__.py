@@ -77,8 +77,8 @@ def load_library():
         "eplb_status_string": ([i32], ctypes.c_char_p),
         "eplb_last_cuda_error": ([], ctypes.c_char_p),
         "eplb_abi_version": ([], i32),
-        "eplb_count_loads": ([p, i64, i64, i32, i32, p, i32, p, p, p], i32),
-        "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, p, p], i32),
+        "eplb_count_loads": ([p, i64, i64, i32, i32, p, i32, p, p], i32),
+        "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, p], i32),
         "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p], i32),
         "eplb_redirect": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, p], i32),
         "eplb_count_redirect": ([p, i64, i64, i32, i32, p, i32, p, i32, p, i64, p, p, p, p], i32),
@@ -200,8 +200,7 @@ class _on_device:
 
 
 def count_loads(idx: torch.Tensor, num_experts: int, counts: Optional[torch.Tensor] = None,
-                accumulate: bool = False, bad: Optional[torch.Tensor] = None,
-                status: Optional[torch.Tensor] = None) -> torch.Tensor:
+                accumulate: bool = False, bad: Optional[torch.Tensor] = None) -> torch.Tensor:
     """S1: counts[l, e] (+)= #{(t, k): idx[l, t, k] == e} for int32 idx [L, T, K]."""
     _cuda(idx, torch.int32, "idx")
     if idx.dim() != 3:
@@ -213,17 +212,16 @@ def count_loads(idx: torch.Tensor, num_experts: int, counts: Optional[torch.Tens
     _cuda(counts, torch.int64, "counts", idx.device)
     if tuple(counts.shape) != (L, num_experts):
         raise ValueError("counts must be [L, E]")
-    _words(idx.device, bad, status)
+    _words(idx.device, bad)
     with _on_device(idx.device):
         _check(load_library().eplb_count_loads(
             _ptr(idx), L, T, K, num_experts, _ptr(counts), int(bool(accumulate)),
-            _ptr(bad), _ptr(status), _stream(idx.device)), "eplb_count_loads")
+            _ptr(bad), _stream(idx.device)), "eplb_count_loads")
     return counts
 
 
 def window_accumulate(steps: torch.Tensor, window: int, s_first: int = 0,
-                      out: Optional[torch.Tensor] = None,
-                      status: Optional[torch.Tensor] = None) -> torch.Tensor:
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """S2: out[s - s_first] = sum of steps[max(0, s-window+1) .. s] (int64 [S, L, E])."""
     _cuda(steps, torch.int64, "steps")
     if steps.dim() != 3:
@@ -234,11 +232,10 @@ def window_accumulate(steps: torch.Tensor, window: int, s_first: int = 0,
     _cuda(out, torch.int64, "out", steps.device)
     if tuple(out.shape) != (S - s_first, L, E):
         raise ValueError("out must be [S - s_first, L, E]")
-    _words(steps.device, status=status)
     with _on_device(steps.device):
         _check(load_library().eplb_window_accumulate(
-            _ptr(steps), S, L, E, window, s_first, _ptr(out), _ptr(status),
-            _stream(steps.device)), "eplb_window_accumulate")
+            _ptr(steps), S, L, E, window, s_first, _ptr(out), _stream(steps.device)),
+            "eplb_window_accumulate")
     return out
 
 
@@ -421,8 +418,8 @@ def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, nex
     L, T, K, Wr, E, P, X, out = _serve_args(idx, plan, ring, next_plan, out, loads_out, bad,
                                             status)
     if not isinstance(layer_done, torch.Tensor) or not layer_done.is_cuda or \
-            layer_done.dtype not in (torch.int32, torch.uint32) or layer_done.numel() != L:
-        raise TypeError("layer_done must be a CUDA int32/uint32 tensor of L elements")
+            layer_done.dtype != torch.uint32 or layer_done.numel() != L:
+        raise TypeError("layer_done must be a CUDA uint32 tensor of L elements")
     if not layer_done.is_contiguous() or layer_done.device != idx.device:
         raise ValueError("layer_done must be contiguous and on the device of idx")
     with _on_device(idx.device):

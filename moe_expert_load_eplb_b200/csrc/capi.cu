@@ -15,7 +15,7 @@ namespace {
 
 std::once_flag g_once[kMaxDevices];
 DeviceInfo g_info[kMaxDevices];
-bool g_ok[kMaxDevices];
+cudaError_t g_err[kMaxDevices];
 
 thread_local char g_last_error[256] = "no error";
 
@@ -73,18 +73,23 @@ eplb_status prepare_kernel(const void *fn, int threads, size_t smem, int *per_sm
   return EPLB_OK;
 }
 
-bool device_info(DeviceInfo *out) {
+eplb_status device_info(DeviceInfo *out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  const cudaError_t gerr = cudaGetDevice(&dev);
+  if (gerr != cudaSuccess) return cuda_fail(gerr);
+  if (dev < 0 || dev >= kMaxDevices) return EPLB_ERR_LIMIT;
   std::call_once(g_once[dev], [dev]() {
     DeviceInfo d;
-    g_ok[dev] = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-                cudaDeviceGetAttribute(&d.max_smem_optin,
-                                       cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess;
+    g_err[dev] = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_err[dev] == cudaSuccess)
+      g_err[dev] = cudaDeviceGetAttribute(&d.max_smem_optin,
+                                          cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
     g_info[dev] = d;
   });
+  // the queries' own error, kept for every later call on this device
+  if (g_err[dev] != cudaSuccess) return cuda_fail(g_err[dev]);
   *out = g_info[dev];
-  return g_ok[dev];
+  return EPLB_OK;
 }
 
 eplb_status cuda_fail(cudaError_t err) {
@@ -117,11 +122,11 @@ const char *eplb_status_string(int32_t status) {
 
 const char *eplb_last_cuda_error(void) { return g_last_error; }
 
-int32_t eplb_abi_version(void) { return (1 << 16) | 1; }
+int32_t eplb_abi_version(void) { return (2 << 16) | 0; }
 
 eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
                              int64_t *counts, int32_t accumulate, unsigned long long *bad,
-                             int32_t *status, cudaStream_t stream) {
+                             cudaStream_t stream) {
   if (L < 0 || T < 0 || K < 1 || E < 1) return EPLB_ERR_SHAPE;
   if (E > 1024 || T > (int64_t(1) << 31) / K) return EPLB_ERR_LIMIT;
   if (L == 0) return EPLB_OK;
@@ -134,13 +139,12 @@ eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K
     if (err != cudaSuccess) return cuda_fail(err);
   }
   if (T == 0) return EPLB_OK;
-  return launch_count_loads(idx, L, T * K, E, counts, bad, status, stream);
+  return launch_count_loads(idx, L, T * K, E, counts, bad, stream);
 }
 
 eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, int32_t E,
-                                   int64_t W, int64_t s_first, int64_t *snaps, int32_t *status,
+                                   int64_t W, int64_t s_first, int64_t *snaps,
                                    cudaStream_t stream) {
-  (void)status;
   if (S < 0 || L < 0 || E < 1 || W < 1 || s_first < 0) return EPLB_ERR_SHAPE;
   if (S == 0 || L == 0) return s_first == 0 ? EPLB_OK : EPLB_ERR_SHAPE;
   if (s_first >= S) return EPLB_ERR_SHAPE;
@@ -304,8 +308,9 @@ eplb_status eplb_serve_step_noalloc(const int32_t *idx, int64_t L, int64_t T, in
                            zero_slot, P, G, N, gpus, loads_out, next_phy2log, next_phyrank,
                            next_logcnt, next_log2phy, nullptr, status, stream);
   }
-  uint32_t *counters = static_layer_done();
-  if (counters == nullptr) return cuda_fail(cudaGetLastError());
+  uint32_t *counters = nullptr;
+  const eplb_status cst = static_layer_done(&counters);
+  if (cst != EPLB_OK) return cst;
   return eplb_serve_step(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot,
                          zero_slot, P, G, N, gpus, loads_out, next_phy2log, next_phyrank,
                          next_logcnt, next_log2phy, counters, status, stream);

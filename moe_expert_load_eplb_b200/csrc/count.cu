@@ -124,11 +124,10 @@ __global__ void __launch_bounds__(kThreads) count_loads_kernel(CountArgs a) {
 }  // namespace
 
 eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer, int32_t E,
-                               int64_t *counts, unsigned long long *bad, int32_t *status,
-                               cudaStream_t stream) {
-  (void)status;  // this kernel has no wait that could run out
+                               int64_t *counts, unsigned long long *bad, cudaStream_t stream) {
   DeviceInfo di;
-  if (!device_info(&di)) return cuda_fail(cudaGetLastError());
+  const eplb_status dst = device_info(&di);
+  if (dst != EPLB_OK) return dst;
   const size_t smem = static_cast<size_t>(E + 1) * 32 * sizeof(uint32_t);
   if (smem > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
   int per_sm = 0;

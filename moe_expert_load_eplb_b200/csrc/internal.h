@@ -34,20 +34,23 @@ inline cudaError_t launch_pdl(const void *fn, dim3 grid, dim3 block, size_t smem
 }
 
 
+// Devices this library keeps per-device state for (indices 0 .. kMaxDevices-1).
+constexpr int kMaxDevices = 64;
+
 struct DeviceInfo {
   int sms = 0;
   int max_smem_optin = 0;
 };
 
-// Cached per device; returns false when the runtime query fails.
-bool device_info(DeviceInfo *out);
+// Cached per device (queried once); EPLB_ERR_CUDA with the query's own error
+// when it failed, EPLB_ERR_LIMIT for a device index of kMaxDevices or more.
+eplb_status device_info(DeviceInfo *out);
 
 // Records a CUDA error message for eplb_last_cuda_error() and maps it.
 eplb_status cuda_fail(cudaError_t err);
 
 eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer, int32_t E,
-                               int64_t *counts, unsigned long long *bad, int32_t *status,
-                               cudaStream_t stream);
+                               int64_t *counts, unsigned long long *bad, cudaStream_t stream);
 
 eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
                           int64_t *snaps, cudaStream_t stream);
@@ -86,11 +89,11 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
                          int32_t *status, cudaStream_t stream);
 
 // Device address of the library-owned per-layer counters of
-// eplb_serve_step_noalloc (kStaticLayers of them) on the current device;
-// nullptr if it cannot be had.
+// eplb_serve_step_noalloc (kStaticLayers of them) on the current device,
+// looked up once per device; EPLB_ERR_LIMIT for a device index of
+// kMaxDevices or more, EPLB_ERR_CUDA with the look-up's own error otherwise.
 constexpr int64_t kStaticLayers = 4096;
-constexpr int kMaxDevices = 64;
-uint32_t *static_layer_done();
+eplb_status static_layer_done(uint32_t **out);
 
 eplb_status launch_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,
                               int64_t R, int32_t E, int32_t P, int32_t gpus, double *gpu_load,

@@ -175,7 +175,8 @@ eplb_status launch_fold_loads(const int64_t *phys, const int32_t *phy2log, int64
 eplb_status launch_initial_map(int64_t R, int32_t E, int32_t P, int32_t *phy2log,
                                int32_t *phyrank, cudaStream_t stream) {
   DeviceInfo di;
-  if (!device_info(&di)) return cuda_fail(cudaGetLastError());
+  const eplb_status dst = device_info(&di);
+  if (dst != EPLB_OK) return dst;
   const int64_t total = R * P;
   const int64_t blocks = std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(di.sms) * 8);
   initial_map_kernel<<<static_cast<unsigned>(std::max<int64_t>(blocks, 1)), 256, 0, stream>>>(

@@ -31,7 +31,8 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
                              int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
                              cudaStream_t stream) {
   DeviceInfo di;
-  if (!device_info(&di)) return cuda_fail(cudaGetLastError());
+  const eplb_status dst = device_info(&di);
+  if (dst != EPLB_OK) return dst;
   const Layout lay(sh);
   if (lay.total > static_cast<size_t>(di.max_smem_optin)) return EPLB_ERR_LIMIT;
   const void *fn = cap2_shape(sh) ? reinterpret_cast<const void *>(rebalance_kernel<true>)

@@ -21,7 +21,8 @@ eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K,
                             int32_t *out, int64_t *counts, unsigned long long *bad,
                             int32_t *status, cudaStream_t stream) {
   DeviceInfo di;
-  if (!device_info(&di)) return cuda_fail(cudaGetLastError());
+  const eplb_status dst = device_info(&di);
+  if (dst != EPLB_OK) return dst;
   const bool count = counts != nullptr;
   RedirectSmem sp;
   const eplb_status st = redirect_plan(E, count, di, &sp);

@@ -67,7 +67,8 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
                          int32_t *next_logcnt, int32_t *next_log2phy, uint32_t *layer_done,
                          int32_t *status, cudaStream_t stream) {
   DeviceInfo di;
-  if (!device_info(&di)) return cuda_fail(cudaGetLastError());
+  const eplb_status dst = device_info(&di);
+  if (dst != EPLB_OK) return dst;
   RedirectSmem sp;
   eplb_status st = redirect_plan(E, true, di, &sp);
   if (st != EPLB_OK) return st;
@@ -118,14 +119,19 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
 // one device.
 static __device__ __align__(256) uint32_t g_layer_done[kStaticLayers];
 
-uint32_t *static_layer_done() {
+eplb_status static_layer_done(uint32_t **out) {
   static std::once_flag once[kMaxDevices];
   static void *addr[kMaxDevices];
   static cudaError_t err[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  const cudaError_t gerr = cudaGetDevice(&dev);
+  if (gerr != cudaSuccess) return cuda_fail(gerr);
+  if (dev < 0 || dev >= kMaxDevices) return EPLB_ERR_LIMIT;
   std::call_once(once[dev], [dev] { err[dev] = cudaGetSymbolAddress(&addr[dev], g_layer_done); });
-  return err[dev] == cudaSuccess ? static_cast<uint32_t *>(addr[dev]) : nullptr;
+  // the look-up's own error, kept for every later call on this device
+  if (err[dev] != cudaSuccess) return cuda_fail(err[dev]);
+  *out = static_cast<uint32_t *>(addr[dev]);
+  return EPLB_OK;
 }
 
 }  // namespace eplb

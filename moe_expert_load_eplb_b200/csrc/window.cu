@@ -73,7 +73,8 @@ __global__ void window_kernel(const int64_t *__restrict__ steps, int64_t S, int6
 eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
                           int64_t *snaps, cudaStream_t stream) {
   DeviceInfo di;
-  if (!device_info(&di)) return cuda_fail(cudaGetLastError());
+  const eplb_status dst = device_info(&di);
+  if (dst != EPLB_OK) return dst;
   // Pick the strip width cw and row groups rg: rg never exceeds the row
   // blocks there are (short rings), the strip count fills the SMs evenly
   // (strips per SM rounded up cost the tail), and enough threads per SM keep

@@ -68,7 +68,7 @@ class EplbStep:
         self.out = torch.empty((L, T, K), dtype=torch.int32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.bad = torch.zeros(1, dtype=torch.int64, device=dev)
-        self.layer_done = torch.zeros(L, dtype=torch.int32, device=dev)
+        self.layer_done = torch.zeros(L, dtype=torch.uint32, device=dev)
         self.steps_done = 0
         self.primed = False
 
@@ -82,15 +82,25 @@ class EplbStep:
         """The plan in force (the newest one built)."""
         return self.plans[self.cur]
 
-    def fill_history(self, history: torch.Tensor, steps_done: Optional[int] = None):
-        """Load earlier per-step counts (at most W - 1 rows kept) into the ring,
-        clear the slot the next step counts into, and build the plan in force."""
+    def load_history(self, history: torch.Tensor, steps_done: Optional[int] = None):
+        """Put earlier per-step counts (int64 [S, L, E], oldest first; the last
+        W - 1 rows are kept) into the ring where the steps that made them
+        would have left them: with s = steps_done (default: the rows kept),
+        row i of the n kept rows is step s - n + i and sits in slot
+        (s - n + i) mod W; slot s mod W, which the next step counts into, is
+        cleared.  Host-side bookkeeping only: no kernel runs."""
         n = min(history.shape[0], self.W - 1)
+        s = n if steps_done is None else int(steps_done)
+        if s < n:
+            raise ValueError(f"steps_done={s} is less than the {n} history rows kept")
         self.ring.zero_()
-        if n:
-            self.ring[:n].copy_(history[history.shape[0] - n:])
-        self.steps_done = n if steps_done is None else steps_done
-        self.ring[self.steps_done % self.W].zero_()
+        for i in range(n):
+            self.ring[(s - n + i) % self.W].copy_(history[history.shape[0] - n + i])
+        self.steps_done = s
+
+    def fill_history(self, history: torch.Tensor, steps_done: Optional[int] = None):
+        """load_history, then build the plan in force from the ring."""
+        self.load_history(history, steps_done)
         self._plan_from_ring(self.plans[self.cur])
         self.primed = True
 
@@ -120,7 +130,7 @@ class EplbStep:
         return (self.L, self.T, self.K, self.E, self.P, self.G, self.N, self.gpus, self.W, self.X)
 
     def _plan_from_ring(self, plan: Plan):
-        window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads, status=self.status)
+        window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads)
         rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=plan,
                   status=self.status)
 
@@ -157,7 +167,7 @@ class EplbStep:
             count_redirect(idx, self.E, used.log2phy, used.logcnt, self.token_offset, counts=row,
                            accumulate=True, out=self.out, bad=self.bad, status=self.status)
         else:
-            count_loads(idx, self.E, counts=row, bad=self.bad, status=self.status)
+            count_loads(idx, self.E, counts=row, bad=self.bad)
         rec(1)
         if self.group is not None:
             allreduce_loads(row, self.group)
@@ -169,8 +179,7 @@ class EplbStep:
                              zero_slot=(self.steps_done + 1) % self.W, slots=self.X, out=nxt,
                              loads_out=self.loads, status=self.status)
         else:
-            window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads,
-                              status=self.status)
+            window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads)
             rec(3)
             nxt = used
             rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=nxt,

@@ -50,23 +50,23 @@ def test_status_strings(lib):
     for code, name in STATUS.items():
         assert lib.eplb_status_string(code).decode() == name
     assert lib.eplb_status_string(1234).decode() == "EPLB_ERR_UNKNOWN"
-    assert lib.eplb_abi_version() >> 16 == 1
+    assert lib.eplb_abi_version() >> 16 == 2
 
 
 def test_host_argument_checks(lib):
     p = ctypes.c_void_p
     one = p(16)  # never dereferenced: every call below fails its checks first
     # count: bad shapes, limits, null, alignment
-    assert lib.eplb_count_loads(one, -1, 4, 2, 8, one, 0, None, None, None) == 2
-    assert lib.eplb_count_loads(one, 1, 4, 0, 8, one, 0, None, None, None) == 2
-    assert lib.eplb_count_loads(one, 1, 4, 2, 2000, one, 0, None, None, None) == 9
-    assert lib.eplb_count_loads(None, 1, 4, 2, 8, one, 1, None, None, None) == 1
-    assert lib.eplb_count_loads(p(20), 1, 4, 2, 8, one, 1, None, None, None) == 8
-    assert lib.eplb_count_loads(one, 0, 4, 2, 8, None, 0, None, None, None) == 0  # nothing to do
+    assert lib.eplb_count_loads(one, -1, 4, 2, 8, one, 0, None, None) == 2
+    assert lib.eplb_count_loads(one, 1, 4, 0, 8, one, 0, None, None) == 2
+    assert lib.eplb_count_loads(one, 1, 4, 2, 2000, one, 0, None, None) == 9
+    assert lib.eplb_count_loads(None, 1, 4, 2, 8, one, 1, None, None) == 1
+    assert lib.eplb_count_loads(p(20), 1, 4, 2, 8, one, 1, None, None) == 8
+    assert lib.eplb_count_loads(one, 0, 4, 2, 8, None, 0, None, None) == 0  # nothing to do
     # window
-    assert lib.eplb_window_accumulate(one, 4, 2, 3, 0, 0, one, None, None) == 2
-    assert lib.eplb_window_accumulate(one, 4, 2, 3, 2, 4, one, None, None) == 2
-    assert lib.eplb_window_accumulate(None, 4, 2, 3, 2, 0, one, None, None) == 1
+    assert lib.eplb_window_accumulate(one, 4, 2, 3, 0, 0, one, None) == 2
+    assert lib.eplb_window_accumulate(one, 4, 2, 3, 2, 4, one, None) == 2
+    assert lib.eplb_window_accumulate(None, 4, 2, 3, 2, 0, one, None) == 1
     # rebalance: divisibility, shape, limits; R == 0 needs no device
     rb = lib.eplb_rebalance
     assert rb(one, 1, 12, 16, 5, 2, 8, 5, one, one, one, one, None, None) == 3   # 12 % 5

@@ -494,7 +494,41 @@ def test_pipeline_serving_order_dsv3_prefill(dsv3_idx, single):
         ring[(W_ - 1 + s_i) % W_] = counts
         plan_ref = _oracle_plan_from_ring(ring, c, step.X)
         _assert_plan_equal(step.plan, plan_ref)
-        assert int(step.layer_done.abs().sum().item()) == 0
+        assert int(step.layer_done.cpu().numpy().astype("int64").sum()) == 0
+
+
+@pytest.mark.parametrize("single", [True, False])
+@pytest.mark.parametrize("steps_done", [2, 7, 13])
+def test_pipeline_history_with_a_step_count(tiny_idx, single, steps_done):
+    """A step primed with history at any step count keeps the last W - 1
+    steps in its window: the oracle, given the same per-step counts in step
+    order, sums the same window before and after each new step."""
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+    c = W.TINY
+    W_ = 4
+    hist = W.histogram_steps(2, c.L, c.E, c.T * c.K, c.stream, device=DEV)
+    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV, fused=True,
+                    single_launch=single)
+    step.fill_history(hist, steps_done=steps_done)
+    steps = [_np(hist[0]), _np(hist[1])]  # per-step counts in step order
+
+    def ref_plan():
+        win = np.stack(steps[-(W_ - 1):] + [np.zeros((c.L, c.E), np.int64)], axis=0)
+        return _oracle_plan_from_ring(win, c, step.X)
+
+    plan_ref = ref_plan()
+    _assert_plan_equal(step.plan, plan_ref)
+    for s_i, idx in enumerate([tiny_idx, tiny_idx.flip(1).contiguous(), tiny_idx,
+                               tiny_idx.flip(2).contiguous()]):
+        used, out = step(idx)
+        torch.cuda.synchronize()
+        assert int(step.status.item()) == 0
+        red, _ = oracle.redirect(_np(idx), plan_ref[3], plan_ref[2])
+        assert np.array_equal(_np(out), red), f"step {s_i}: redirect"
+        steps.append(oracle.count_loads(_np(idx), c.E)[0])
+        plan_ref = ref_plan()
+        _assert_plan_equal(step.plan, plan_ref)
+    assert step.steps_done == steps_done + 4
 
 
 def test_pipeline_serving_with_an_nccl_group_of_one(tiny_idx):
@@ -635,18 +669,18 @@ def test_outputs_stay_inside_their_buffers(shape):
                          g((L, E, X), torch.int32))
 
     st = _status()
-    counts = eplb.count_loads(idx, E, counts=g((L, E), torch.int64), status=st)
+    counts = eplb.count_loads(idx, E, counts=g((L, E), torch.int64))
     plan = eplb.rebalance(counts, P, G, N, gpus, slots=X, out=gplan(), status=st)
     eplb.redirect(idx, plan.log2phy, plan.logcnt, 5, out=g((L, T, K), torch.int32), status=st)
     eplb.count_redirect(idx, E, plan.log2phy, plan.logcnt, 5, counts=g((L, E), torch.int64),
                         out=g((L, T, K), torch.int32), status=st)
     steps = _dev(rng.integers(0, 1000, (4, L, E)).astype(np.int64))
-    eplb.window_accumulate(steps, 2, out=g((4, L, E), torch.int64), status=st)
+    eplb.window_accumulate(steps, 2, out=g((4, L, E), torch.int64))
     ring = g((3, L, E), torch.int64)
     ring.copy_(steps[:3])
     eplb.rebalance_window(ring, P, G, N, gpus, zero_slot=1, slots=X, out=gplan(),
                           loads_out=g((L, E), torch.int64), status=st)
-    done = g((L,), torch.int32)
+    done = g((L,), torch.int32).view(torch.uint32)
     done.zero_()
     eplb.serve_step(idx, plan, ring, 1, gplan(), done, G, N, gpus, zero_slot=2, token_offset=9,
                     out=g((L, T, K), torch.int32), loads_out=g((L, E), torch.int64), status=st)
@@ -684,7 +718,7 @@ def test_serve_step_matches_oracle(shape, W_, slot, zero_slot):
     ring_d = _dev(ring)
     used = eplb.Plan(*[_dev(a) for a in plan_in])
     nxt = eplb.Plan(*[torch.full(a.shape, 7, dtype=torch.int32, device=DEV) for a in plan_in])
-    done = torch.zeros(L, dtype=torch.int32, device=DEV)
+    done = torch.zeros(L, dtype=torch.uint32, device=DEV)
     loads = torch.zeros((L, E), dtype=torch.int64, device=DEV)
     bad = torch.zeros(1, dtype=torch.int64, device=DEV)
     st = _status()
@@ -719,7 +753,7 @@ def test_serve_step_reports_range_and_keeps_going():
     plan_in = oracle.rebalance(rng.integers(0, 100, (L, E)), P, G, N, gpus, slots=X)
     used = eplb.Plan(*[_dev(a) for a in plan_in])
     nxt = eplb.Plan(*[torch.empty(a.shape, dtype=torch.int32, device=DEV) for a in plan_in])
-    done = torch.zeros(L, dtype=torch.int32, device=DEV)
+    done = torch.zeros(L, dtype=torch.uint32, device=DEV)
     st = _status()
     idx = _dev(rng.integers(0, E, (L, T, K)).astype(np.int32))
     eplb.serve_step(idx, used, _dev(ring), 0, nxt, done, G, N, gpus, status=st)
@@ -741,7 +775,7 @@ def test_serve_step_host_errors():
                      torch.zeros((L, E, X), dtype=torch.int32, device=DEV))
     ring = torch.zeros((2, L, E), dtype=torch.int64, device=DEV)
     idx = torch.zeros((L, T, K), dtype=torch.int32, device=DEV)
-    done = torch.zeros(L, dtype=torch.int32, device=DEV)
+    done = torch.zeros(L, dtype=torch.uint32, device=DEV)
     with pytest.raises(eplb.EplbError) as ei:  # the next plan is the plan in force
         eplb.serve_step(idx, plan, ring, 0, plan, done, G, N, gpus)
     assert ei.value.code == 2
@@ -782,7 +816,7 @@ def test_binding_rejects_malformed_arguments():
     with pytest.raises(TypeError):  # bad is a 64-bit word
         eplb.redirect(idx, plan.log2phy, plan.logcnt, bad=mk(1))
     with pytest.raises(TypeError):  # status is an int32 word
-        eplb.count_loads(idx, E, status=mk(1, torch.int64))
+        eplb.redirect(idx, plan.log2phy, plan.logcnt, status=mk(1, torch.int64))
     with pytest.raises(ValueError):
         eplb.count_redirect(idx, E, plan.log2phy, plan.logcnt, status=mk(0))
     with pytest.raises(TypeError):  # a table left on the host

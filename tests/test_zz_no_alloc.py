@@ -42,7 +42,7 @@ def test_noalloc_matches_serve_step_on_two_calls_in_a_row(shape):
         ring = _dev(ring0)
         plans = [eplb.Plan(*[_dev(a) for a in plan_in]),
                  eplb.Plan(*[torch.zeros(a.shape, dtype=torch.int32, device="cuda:0") for a in plan_in])]
-        done = torch.zeros(L, dtype=torch.int32, device="cuda:0")
+        done = torch.zeros(L, dtype=torch.uint32, device="cuda:0")
         st = torch.zeros(1, dtype=torch.int32, device="cuda:0")
         outs = []
         for k, idx in enumerate(batches):  # two calls in a row, the plans swapping
