@@ -191,101 +191,93 @@ static i128 gcd128(i128 a, i128 b) {
 }
 
 /* ------------------------------------------------------------------------ */
-/* rebalance_experts_hierarchical ([EPLB] section "Иерархическая             */
-/* балансировка" and the appendix function of that name), for one row.       */
-/*   step 1: group loads -> balanced_packing over num_nodes (groups->nodes);  */
-/*   step 2: replicate_experts inside every node;                            */
-/*   step 3: per-replica load w/cnt -> balanced_packing over the node's GPUs; */
-/*   then the index bookkeeping (mlog = logical order after the node         */
-/*   permutation, pphy = physical order after GPU packing).                  */
+/* One row of the hierarchical policy ([EPLB] section "Иерархическая         */
+/* балансировка" and its flowchart), in three steps:                          */
+/*   1. spread the expert groups over the nodes so that the nodes' loads are  */
+/*      balanced (balanced_packing of the G group loads into N nodes, G/N     */
+/*      groups each); a node's experts are then its groups in the order the   */
+/*      packing seated them, each group's experts in index order;             */
+/*   2. copy experts inside every node (replicate_experts of the node's E/N   */
+/*      loads to its P/N slots);                                               */
+/*   3. lay each node's copies onto the node's GPUs so that the GPUs' loads   */
+/*      are balanced (balanced_packing of the copies' loads w / copies into   */
+/*      gpus/N GPUs, P/gpus copies each).                                      */
+/* Physical slot of a copy: node * (P/N) + GPU-in-node * (P/gpus) + its seat  */
+/* on that GPU.  The global policy calls this with one group on one node.     */
 /* ------------------------------------------------------------------------ */
-static int rebalance_hierarchical_row(const int64_t *weight, int E, int P,
-                                      int G, int N, int gpus, int32_t *phy2log,
-                                      int32_t *phyrank, int32_t *logcnt) {
+static int plan_row(const int64_t *weight, int E, int P, int G, int N, int gpus,
+                    int32_t *phy2log, int32_t *phyrank, int32_t *logcnt) {
   if (E % G != 0 || G % N != 0 || gpus % N != 0 || P % gpus != 0)
     return ORACLE_ERR_DIVISIBILITY;
-  const int group_size = E / G;
-  const int groups_per_node = G / N;
-  const int lpn = E / N;              /* logical experts per node */
-  const int ppn = P / N;              /* physical experts per node */
-  const int ppg = P / gpus;           /* physical experts per GPU */
+  const int gsize = E / G;              /* experts per group */
+  const int per_node = E / N;           /* experts per node */
+  const int slots_per_node = P / N;
+  const int slots_per_gpu = P / gpus;
   const int gpus_per_node = gpus / N;
   int rc = ORACLE_OK;
 
-  i128 *tokens_per_group = (i128 *)calloc((size_t)G, sizeof(i128));
-  int *group_pack = (int *)malloc(sizeof(int) * (size_t)G);
-  int *group_rank = (int *)malloc(sizeof(int) * (size_t)G);
-  int *log2mlog = (int *)malloc(sizeof(int) * (size_t)E);
-  int *mlog2log = (int *)malloc(sizeof(int) * (size_t)E);
-  int64_t *tokens_per_mlog = (int64_t *)malloc(sizeof(int64_t) * (size_t)lpn);
-  int *phy2mlog = (int *)malloc(sizeof(int) * (size_t)ppn);
-  int *rank = (int *)malloc(sizeof(int) * (size_t)ppn);
-  int *mlogcnt = (int *)malloc(sizeof(int) * (size_t)E); /* all nodes */
-  i128 *tokens_per_phy = (i128 *)malloc(sizeof(i128) * (size_t)ppn);
-  int *pack = (int *)malloc(sizeof(int) * (size_t)ppn);
-  int *rank_in_pack = (int *)malloc(sizeof(int) * (size_t)ppn);
-  int *pphy2phy = (int *)malloc(sizeof(int) * (size_t)ppn);
-  if (!tokens_per_group || !group_pack || !group_rank || !log2mlog ||
-      !mlog2log || !tokens_per_mlog || !phy2mlog || !rank || !mlogcnt ||
-      !tokens_per_phy || !pack || !rank_in_pack || !pphy2phy) {
+  i128 *group_load = (i128 *)calloc((size_t)G, sizeof(i128));
+  int *node_of_group = (int *)malloc(sizeof(int) * (size_t)G);
+  int *seat_of_group = (int *)malloc(sizeof(int) * (size_t)G);
+  int *member = (int *)malloc(sizeof(int) * (size_t)E);       /* [N][per_node] expert ids */
+  int64_t *node_w = (int64_t *)malloc(sizeof(int64_t) * (size_t)per_node);
+  int *owner = (int *)malloc(sizeof(int) * (size_t)slots_per_node);   /* copy -> member */
+  int *copy_rank = (int *)malloc(sizeof(int) * (size_t)slots_per_node);
+  int *copies = (int *)malloc(sizeof(int) * (size_t)per_node);
+  i128 *copy_w = (i128 *)malloc(sizeof(i128) * (size_t)slots_per_node);
+  int *gpu_of_copy = (int *)malloc(sizeof(int) * (size_t)slots_per_node);
+  int *seat_of_copy = (int *)malloc(sizeof(int) * (size_t)slots_per_node);
+  if (!group_load || !node_of_group || !seat_of_group || !member || !node_w || !owner ||
+      !copy_rank || !copies || !copy_w || !gpu_of_copy || !seat_of_copy) {
     rc = ORACLE_ERR_ALLOC;
-    goto done;
+    goto out;
   }
 
-  /* step 1: groups -> nodes */
-  for (int g = 0; g < G; ++g)
-    for (int i = 0; i < group_size; ++i)
-      tokens_per_group[g] += weight[g * group_size + i];
-  rc = balanced_packing(tokens_per_group, G, N, group_pack, group_rank);
-  if (rc) goto done;
-  for (int e = 0; e < E; ++e) {
-    int g = e / group_size;
-    log2mlog[e] = (group_pack[g] * groups_per_node + group_rank[g]) * group_size +
-                  e % group_size;
+  /* 1. groups over nodes */
+  for (int e = 0; e < E; ++e) group_load[e / gsize] += weight[e];
+  rc = balanced_packing(group_load, G, N, node_of_group, seat_of_group);
+  if (rc) goto out;
+  for (int g = 0; g < G; ++g) {
+    int first = node_of_group[g] * per_node + seat_of_group[g] * gsize;
+    for (int j = 0; j < gsize; ++j) member[first + j] = g * gsize + j;
   }
-  for (int e = 0; e < E; ++e) mlog2log[log2mlog[e]] = e; /* inverse */
 
   for (int n = 0; n < N; ++n) {
-    /* step 2: redundant experts inside node n */
-    for (int i = 0; i < lpn; ++i) tokens_per_mlog[i] = weight[mlog2log[n * lpn + i]];
-    replicate_experts(tokens_per_mlog, lpn, ppn, phy2mlog, rank, mlogcnt + n * lpn);
-    const int *cnt = mlogcnt + n * lpn;
+    const int *mine = member + n * per_node;
 
-    /* step 3: replicas -> GPUs of node n, load of replica j is
-       tokens_per_mlog[phy2mlog[j]] / cnt[phy2mlog[j]], scaled by LAMBDA.
-       With one replica per GPU balanced_packing returns the identity
-       without reading the loads, so they are not formed then.  A row whose
-       LAMBDA exceeds 2^62 cannot be held exactly and is rejected. */
-    for (int j = 0; j < ppn; ++j) tokens_per_phy[j] = 0;
-    if (ppg > 1) {
-      i128 lambda = 1;
-      for (int i = 0; i < lpn; ++i) {
-        lambda = lambda / gcd128(lambda, cnt[i]) * cnt[i];
-        if (lambda > ((i128)1 << 62)) { rc = ORACLE_ERR_RANGE; goto done; }
+    /* 2. copies inside node n */
+    for (int i = 0; i < per_node; ++i) node_w[i] = weight[mine[i]];
+    replicate_experts(node_w, per_node, slots_per_node, owner, copy_rank, copies);
+    for (int i = 0; i < per_node; ++i) logcnt[mine[i]] = copies[i];
+
+    /* 3. copies over node n's GPUs.  A copy carries w / copies; the packing
+       compares sums of these ratios exactly by scaling all of them by one
+       common multiple D of the copy counts (any D gives the same order).
+       With one copy per GPU the packing is the identity and reads no loads.
+       A row whose D would exceed 2^62 cannot be held exactly: rejected. */
+    for (int j = 0; j < slots_per_node; ++j) copy_w[j] = 0;
+    if (slots_per_gpu > 1) {
+      i128 D = 1;
+      for (int i = 0; i < per_node; ++i) {
+        D = D / gcd128(D, copies[i]) * copies[i];
+        if (D > ((i128)1 << 62)) { rc = ORACLE_ERR_RANGE; goto out; }
       }
-      for (int j = 0; j < ppn; ++j) {
-        int i = phy2mlog[j];
-        tokens_per_phy[j] = (i128)tokens_per_mlog[i] * (lambda / cnt[i]);
-      }
+      for (int j = 0; j < slots_per_node; ++j)
+        copy_w[j] = (i128)node_w[owner[j]] * (D / copies[owner[j]]);
     }
-    rc = balanced_packing(tokens_per_phy, ppn, gpus_per_node, pack, rank_in_pack);
-    if (rc) goto done;
-    for (int j = 0; j < ppn; ++j) pphy2phy[pack[j] * ppg + rank_in_pack[j]] = j;
-
-    /* index bookkeeping: pphy -> mlog -> log */
-    for (int pp = 0; pp < ppn; ++pp) {
-      int j = pphy2phy[pp];
-      phy2log[n * ppn + pp] = mlog2log[n * lpn + phy2mlog[j]];
-      phyrank[n * ppn + pp] = rank[j];
+    rc = balanced_packing(copy_w, slots_per_node, gpus_per_node, gpu_of_copy, seat_of_copy);
+    if (rc) goto out;
+    for (int j = 0; j < slots_per_node; ++j) {
+      int slot = n * slots_per_node + gpu_of_copy[j] * slots_per_gpu + seat_of_copy[j];
+      phy2log[slot] = mine[owner[j]];
+      phyrank[slot] = copy_rank[j];
     }
   }
-  for (int e = 0; e < E; ++e) logcnt[e] = mlogcnt[log2mlog[e]];
 
-done:
-  free(tokens_per_group); free(group_pack); free(group_rank); free(log2mlog);
-  free(mlog2log); free(tokens_per_mlog); free(phy2mlog); free(rank);
-  free(mlogcnt); free(tokens_per_phy); free(pack); free(rank_in_pack);
-  free(pphy2phy);
+out:
+  free(group_load); free(node_of_group); free(seat_of_group); free(member);
+  free(node_w); free(owner); free(copy_rank); free(copies); free(copy_w);
+  free(gpu_of_copy); free(seat_of_copy);
   return rc;
 }
 
@@ -314,7 +306,7 @@ int oracle_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P,
     for (int e = 0; e < E; ++e)
       if (w[e] < 0 || w[e] >= LOAD_LIMIT) return ORACLE_ERR_RANGE;
     int32_t *p2l = phy2log + r * P, *prk = phyrank + r * P, *cnt = logcnt + r * E;
-    int rc = rebalance_hierarchical_row(w, E, P, g, n, gpus, p2l, prk, cnt);
+    int rc = plan_row(w, E, P, g, n, gpus, p2l, prk, cnt);
     if (rc) return rc;
     int32_t *l2p = log2phy + r * (int64_t)E * X;
     for (int64_t i = 0; i < (int64_t)E * X; ++i) l2p[i] = -1;
