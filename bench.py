@@ -51,11 +51,19 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--clock-ms", type=float, default=400.0,
+                    help="repeat the timed region until the clock record spans about this long")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer e2e measurement")
     ap.add_argument("--no-fresh", action="store_true", help="skip the fresh-plan-order comparison")
     ap.add_argument("--fresh-only", action="store_true",
                     help="time only the fresh-plan order (for profiling its kernels)")
-    return ap.parse_args()
+    ap.add_argument("--legs", default="hbm_stream,global_policy,window_sweep",
+                    help="single-GPU legs on the other workloads, comma-separated ('' for none)")
+    ap.add_argument("--legs-only", action="store_true",
+                    help="run only the legs (no serving step): for profiling their kernels")
+    a = ap.parse_args()
+    a.legs = [x for x in a.legs.split(",") if x]
+    return a
 
 
 def _peaks():
@@ -84,7 +92,7 @@ class ClockSampler:
              0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
              0x10: "sync_boost", 0x100: "display_clock"}
 
-    def __init__(self, device: int, period: float = 0.02):
+    def __init__(self, device: int, period: float = 0.002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period, self._stop, self.ok = period, threading.Event(), False
         try:
@@ -112,9 +120,13 @@ class ClockSampler:
         nv = self.nv
         get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        self.t_first = self.t_last = None
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.t_last = time.perf_counter()
+                if self.t_first is None:
+                    self.t_first = self.t_last
                 r = get_r(self.h)
                 for bit, name in self.NAMES.items():
                     if r & bit:
@@ -138,7 +150,9 @@ class ClockSampler:
         if not self.ok or not self.samples:
             return None
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+                "sm_mhz_min": min(self.samples), "reasons": sorted(self.reasons),
+                "samples": len(self.samples),
+                "span_ms": round(1e3 * (self.t_last - self.t_first), 1) if self.t_first else 0.0}
 
 
 # --------------------------------------------------------------- profiles --
@@ -180,21 +194,26 @@ def _traffic(kernel_file: str, profile: str, scale: float):
 STAGES = ("count", "allreduce", "window", "rebalance", "redirect")
 
 
-def _timed_steps(step, idx, flush, K, group, dev, staged=False, scrub=None):
+def _timed_steps(step, idx, flush, K, group, dev, staged=False, scrub=None, clock_ms=0.0):
     """Runs K steps, each between a start and an end event (the L2 flush
-    before each step stays outside them); returns (total ms, max over ranks,
-    per-stage mean ms or None, clock summary).  With ``staged`` the step also
-    records events between its stages for the per-stage breakdown -- those
-    extra records cost time of their own, so the headline is taken without
-    them.  ``scrub`` (a buffer larger than L2): read after the flush write,
-    so that L2 holds clean lines and none of the flush's dirty lines is
-    written back inside the timed step."""
+    before each step stays outside them); returns (total ms of the K steps,
+    max over ranks; per-stage mean ms or None; clock summary; ms per step of
+    every repeat).  With ``staged`` the step also records events between its
+    stages for the per-stage breakdown -- those extra records cost time of
+    their own, so the headline is taken without them.  ``scrub`` (a buffer
+    larger than L2): read after the flush write, so that L2 holds clean
+    lines and none of the flush's dirty lines is written back inside the
+    timed step.  ``clock_ms``: the K-step region is then repeated (same
+    count on every rank) until the clock sampler, running throughout, has
+    seen about that many milliseconds; the first region is the one
+    returned as the total, the repeats only widen the clock record."""
     n_ev = 6 if staged else 2
-    marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
-    if group is not None:
-        torch.distributed.barrier(group=group)
-    torch.cuda.synchronize()
-    with ClockSampler(dev.index) as clocks:
+
+    def region():
+        marks = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
+        if group is not None:
+            torch.distributed.barrier(group=group)
+        torch.cuda.synchronize()
         for i in range(K):
             flush.fill_(i & 0xff)
             if scrub is not None:
@@ -206,17 +225,32 @@ def _timed_steps(step, idx, flush, K, group, dev, staged=False, scrub=None):
                 step(idx)
                 marks[i][1].record()
         torch.cuda.synchronize()
-    if group is not None:
-        torch.distributed.barrier(group=group)
+        if group is not None:
+            torch.distributed.barrier(group=group)
+        tot = torch.tensor([sum(m[0].elapsed_time(m[-1]) for m in marks)], dtype=torch.float64,
+                           device=dev)
+        if group is not None:
+            torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX, group=group)
+        return float(tot.item()), marks
+
+    with ClockSampler(dev.index) as clocks:
+        t_wall = time.perf_counter()
+        total, marks = region()
+        wall_ms = (time.perf_counter() - t_wall) * 1e3
+        # a repeat count every rank derives from the same all-reduced figure
+        reps = 0 if clock_ms <= 0 else min(2000, int(clock_ms / max(wall_ms, 1e-3)))
+        if group is not None and reps:
+            r = torch.tensor([reps], dtype=torch.int64, device=dev)
+            torch.distributed.all_reduce(r, op=torch.distributed.ReduceOp.MIN, group=group)
+            reps = int(r.item())
+        repeats = [total / K]
+        for _ in range(reps):
+            repeats.append(region()[0] / K)
     per_stage = None
     if staged:
         per_stage = {n: statistics.mean(m[k].elapsed_time(m[k + 1]) for m in marks)
                      for k, n in enumerate(STAGES)}
-    total = torch.tensor([sum(m[0].elapsed_time(m[-1]) for m in marks)], dtype=torch.float64,
-                         device=dev)
-    if group is not None:
-        torch.distributed.all_reduce(total, op=torch.distributed.ReduceOp.MAX, group=group)
-    return float(total.item()), per_stage, clocks.summary()
+    return total, per_stage, clocks.summary(), repeats
 
 
 def _stage_report(per_stage, fused, X, world, hbm_peak):
@@ -250,6 +284,143 @@ def _stage_report(per_stage, fused, X, world, hbm_peak):
     return stages
 
 
+# ------------------------------------------------- the other configurations --
+# Single-GPU legs on the pages' other workloads: the 16x larger routed batch
+# (HBM streaming), the global policy over 144 GPUs and the 1000-step window
+# sweep.  Each call is timed alone between CUDA events on the launching
+# stream, with the clock sampler running; median over the calls.
+
+def _time_calls(fn, n, dev, flush=None):
+    """Times n calls of fn (after 3 untimed ones), each between two events on
+    the current stream; ``flush`` is written before every call, outside the
+    events.  Returns (median ms, mean ms, clock summary)."""
+    for i in range(3):
+        if flush is not None:
+            flush.fill_(i & 0xff)
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clocks:
+        for i in range(n):
+            if flush is not None:
+                flush.fill_(i & 0xff)
+            ev[i][0].record()
+            fn()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    return statistics.median(ms), statistics.mean(ms), clocks.summary()
+
+
+def _hbm_entry(algo_bytes, med, mean, clocks, hbm_peak, extra=None):
+    gbs = algo_bytes / (med / 1e3) / 1e9
+    d = {"ms": round(med, 5), "ms_mean": round(mean, 5), "algo_bytes": algo_bytes,
+         "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm_peak, 4),
+         "frac_of_datasheet": round(gbs / DATASHEET_HBM_GBS, 4), "clocks": clocks}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def leg_hbm_stream(n, dev, hbm_peak):
+    """hbm_stream: 58 layers x 1,048,576 tokens x top-8 (486.5 M int32
+    indices, 1.95 GB).  count_loads, redirect and the fused count_redirect,
+    each on the whole batch, against the plan rebuilt from the batch's own
+    counts.  Inputs and outputs are 16x the L2, so no flush is needed."""
+    import moe_expert_load_eplb_b200 as eplb
+    c = W.HBM_STREAM
+    torch.cuda.empty_cache()
+    idx = W.routed_indices("hbm_stream", device=dev)
+    n_idx = idx.numel()
+    counts = eplb.count_loads(idx, c.E)
+    plan = eplb.rebalance(counts, c.P, c.G, c.N, c.gpus)
+    out = torch.empty_like(idx)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    res = {"workload": c.name, "layers": c.L, "tokens_per_layer": c.T, "top_k": c.K,
+           "indices": n_idx, "calls": n, "l2": "not flushed: 1.95 GB in (+1.95 GB out) per call"}
+    m = _time_calls(lambda: eplb.count_loads(idx, c.E, counts=counts), n, dev)
+    res["count"] = _hbm_entry(4.0 * n_idx, *m, hbm_peak,
+                              {"target_ms": round(4.0 * n_idx / (0.7 * hbm_peak * 1e9) * 1e3, 4)})
+    m = _time_calls(lambda: eplb.redirect(idx, plan.log2phy, plan.logcnt, out=out, status=st), n, dev)
+    res["redirect"] = _hbm_entry(8.0 * n_idx, *m, hbm_peak,
+                                 {"target_ms": round(8.0 * n_idx / (0.7 * hbm_peak * 1e9) * 1e3, 4)})
+    m = _time_calls(lambda: eplb.count_redirect(idx, c.E, plan.log2phy, plan.logcnt, counts=counts,
+                                                out=out, status=st), n, dev)
+    res["count_redirect"] = _hbm_entry(8.0 * n_idx + 8.0 * c.L * c.E, *m, hbm_peak)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the hbm_stream leg")
+    del idx, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def leg_global_policy(n, dev, flush):
+    """global_policy: rebalance_experts on 58 rows of 256 Pareto loads, 288
+    replicas, one group over 2 nodes (global policy), 144 GPUs (two replicas
+    each).  L2 flushed before every call."""
+    import moe_expert_load_eplb_b200 as eplb
+    c = W.GLOBAL_POLICY
+    loads = torch.from_numpy(W.global_policy_loads()).to(dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    plan = eplb.rebalance(loads, c.P, c.G, c.N, c.gpus, status=st)
+    med, mean, clocks = _time_calls(
+        lambda: eplb.rebalance(loads, c.P, c.G, c.N, c.gpus, out=plan, status=st), n, dev, flush)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the global_policy leg")
+    return {"workload": c.name, "rows": c.L, "experts": c.E, "replicas": c.P, "plan_gpus": c.gpus,
+            "policy": "global", "calls": n, "l2": "flushed before every call (512 MB write)",
+            "rebalance": {"us_per_call": round(med * 1e3, 2), "us_mean": round(mean * 1e3, 2),
+                          "rows_per_s": round(c.L / (med / 1e3), 1), "clocks": clocks}}
+
+
+def leg_window_sweep(n, dev, flush, hbm_peak):
+    """window_sweep: 1000 steps x 58 layers x 256 experts of per-step counts
+    (8,192 tokens x top-8 each); the W = 1000 window sum of every step
+    (running totals, int64 [1000, 58, 256] in and out), then rebalance_experts
+    on all 58,000 windowed rows.  L2 flushed before every call."""
+    import moe_expert_load_eplb_b200 as eplb
+    c = W.WINDOW_SWEEP
+    steps = W.window_sweep_steps(device=dev)
+    snaps = eplb.window_accumulate(steps, c.W)
+    loads = snaps.view(-1, c.E)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    plan = eplb.rebalance(loads, c.P, c.G, c.N, c.gpus, status=st)
+    elems = steps.numel()
+    res = {"workload": c.name, "steps": c.S, "layers": c.L, "experts": c.E, "window": c.W,
+           "calls": n, "l2": "flushed before every call (512 MB write)"}
+    m = _time_calls(lambda: eplb.window_accumulate(steps, c.W, out=snaps), n, dev, flush)
+    res["window"] = _hbm_entry(16.0 * elems, *m, hbm_peak)
+    med, mean, clocks = _time_calls(
+        lambda: eplb.rebalance(loads, c.P, c.G, c.N, c.gpus, out=plan, status=st), n, dev, flush)
+    res["rebalance"] = {"rows": loads.shape[0], "ms": round(med, 4), "ms_mean": round(mean, 4),
+                        "rows_per_s": round(loads.shape[0] / (med / 1e3), 1), "clocks": clocks}
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the window_sweep leg")
+    del steps, snaps, plan
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_legs(args, dev, legs):
+    """The single-GPU legs named in ``legs`` (one GPU only)."""
+    hbm_peak, _ = _peaks()
+    n = max(20, min(args.steps, 200))
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    out = {}
+    if "hbm_stream" in legs:
+        out["hbm_stream"] = leg_hbm_stream(n, dev, hbm_peak)
+    if "global_policy" in legs:
+        out["global_policy"] = leg_global_policy(n, dev, flush)
+    if "window_sweep" in legs:
+        out["window_sweep"] = leg_window_sweep(n, dev, flush, hbm_peak)
+    del flush
+    return out
+
+
 def run_ours(args, rank: int, world: int, group):
     import moe_expert_load_eplb_b200 as eplb
     from moe_expert_load_eplb_b200.pipeline import EplbStep
@@ -279,8 +450,8 @@ def run_ours(args, rank: int, world: int, group):
             flush.fill_(i & 0xff)
             fresh(idx)
         check(fresh, "fresh-order warm-up")
-        f_total, _, clocks = _timed_steps(fresh, idx, flush, args.steps, group, dev)
-        _, f_stage, _ = _timed_steps(fresh, idx, flush, min(args.steps, 500), group, dev, staged=True)
+        f_total, _, clocks, _ = _timed_steps(fresh, idx, flush, args.steps, group, dev)
+        _, f_stage, _, _ = _timed_steps(fresh, idx, flush, min(args.steps, 500), group, dev, staged=True)
         check(fresh, "fresh-order steps")
         return {"fresh_only": True, "steps": args.steps, "ms_per_step": round(f_total / args.steps, 5),
                 "stages": _stage_report(f_stage, False, fresh.X, world, hbm_peak), "clocks": clocks}
@@ -292,12 +463,17 @@ def run_ours(args, rank: int, world: int, group):
         step(idx)
     check(step, "warm-up")
     K = args.steps
-    total_ms, _, clocks = _timed_steps(step, idx, flush, K, group, dev)
+    total_ms, _, clocks, repeats = _timed_steps(step, idx, flush, K, group, dev,
+                                                clock_ms=args.clock_ms)
     check(step, "timed steps")
     ms_per_step = total_ms / K
+    if clocks is not None:
+        clocks["region"] = (f"the {K} timed steps, then {len(repeats) - 1} repeats of them "
+                            f"(sampled every 2 ms throughout)")
+        clocks["step_kcycles"] = round(ms_per_step * clocks["sm_mhz"], 2)
     value = c.L * K / (total_ms / 1e3)
     # per-stage breakdown: a separate pass with events between the stages
-    _, per_stage, _ = _timed_steps(step, idx, flush, max(3, min(K, 500)), group, dev, staged=True)
+    _, per_stage, _, _ = _timed_steps(step, idx, flush, max(3, min(K, 500)), group, dev, staged=True)
     check(step, "staged steps")
     stages = _stage_report(per_stage, True, step.X, world, hbm_peak)
     stages["count"]["traffic"] = _traffic("redirect.cu+redirect_chunk.cuh",
@@ -317,7 +493,9 @@ def run_ours(args, rank: int, world: int, group):
            "config": dict(_config(world), step_order=order),
            "gpu_launches": step.launches_per_step * K,
            "tokens_per_s": round(world * c.T * K / (total_ms / 1e3), 1),
-           "stages": stages, "roofline": roof, "clocks": clocks}
+           "stages": stages, "roofline": roof, "clocks": clocks,
+           "repeats_ms_per_step": {"n": len(repeats), "median": round(statistics.median(repeats), 5),
+                                   "min": round(min(repeats), 5), "max": round(max(repeats), 5)}}
 
     # ---- the same step after a clean flush, one GPU only --------------------
     # The headline's flush (a 512 MB write) leaves L2 full of dirty lines that
@@ -327,8 +505,8 @@ def run_ours(args, rank: int, world: int, group):
     if world == 1 and not args.no_fresh:
         scrub = torch.zeros(FLUSH_BYTES // 2, dtype=torch.uint8, device=dev)
         Kc = max(3, min(K, 500))
-        c_total, _, _ = _timed_steps(step, idx, flush, Kc, group, dev, scrub=scrub)
-        _, c_stage, _ = _timed_steps(step, idx, flush, Kc, group, dev, staged=True, scrub=scrub)
+        c_total, _, _, _ = _timed_steps(step, idx, flush, Kc, group, dev, scrub=scrub)
+        _, c_stage, _, _ = _timed_steps(step, idx, flush, Kc, group, dev, staged=True, scrub=scrub)
         check(step, "clean-flush steps")
         cst = _stage_report(c_stage, True, step.X, world, hbm_peak)
         out["clean_l2"] = {
@@ -347,7 +525,7 @@ def run_ours(args, rank: int, world: int, group):
             one(idx)
         check(one, "one-launch warm-up")
         Ko = max(3, min(K, 500))
-        o_total, _, _ = _timed_steps(one, idx, flush, Ko, group, dev)
+        o_total, _, _, _ = _timed_steps(one, idx, flush, Ko, group, dev)
         check(one, "one-launch steps")
         n_idx = c.L * c.T * c.K
         # indices in and out, count atomics, ring rows summed, cleared slot,
@@ -421,8 +599,8 @@ def run_ours(args, rank: int, world: int, group):
         fresh(idx)
     check(fresh, "fresh-order warm-up")
     Kf = max(3, min(K, 500))
-    f_total, _, _ = _timed_steps(fresh, idx, flush, Kf, group, dev)
-    _, f_stage, _ = _timed_steps(fresh, idx, flush, Kf, group, dev, staged=True)
+    f_total, _, _, _ = _timed_steps(fresh, idx, flush, Kf, group, dev)
+    _, f_stage, _, _ = _timed_steps(fresh, idx, flush, Kf, group, dev, staged=True)
     check(fresh, "fresh-order steps")
     fstages = _stage_report(f_stage, False, fresh.X, world, hbm_peak)
     out["fresh_order"] = {"steps": Kf, "ms_per_step": round(f_total / Kf, 5),
@@ -436,6 +614,8 @@ def run_ours(args, rank: int, world: int, group):
 def _finish(out, args, step, idx, hist, flush, group, dev, rank, world):
     c = CFG
     K = args.steps
+    if world == 1 and args.legs:
+        out.update(run_legs(args, dev, args.legs))
 
     def check(st, where):
         torch.cuda.synchronize()
@@ -644,6 +824,10 @@ def main():
     from moe_expert_load_eplb_b200.distributed import init_from_env
     rank, world, local, group = init_from_env("nccl" if world > 1 else None)
     torch.cuda.set_device(local)
+    if args.legs_only:
+        if world == 1:
+            print(json.dumps(run_legs(args, torch.device("cuda", local), args.legs)), flush=True)
+        return
     try:
         res = run_ours(args, rank, world, group)
         if rank == 0:

@@ -125,13 +125,20 @@ eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, i
  * log2phy  device int32 [R, E, X].  X = (P - E) / N + 1 (hierarchical) or
  *          P - E + 1 (global) always suffices; with a smaller X, replicas of
  *          rank >= X are left out of log2phy and *status = EPLB_ERR_SLOTS.
+ * gpu_load device double [R, gpus], nullable; stats device double [R, 4],
+ *          nullable: the plan quality of each row's new plan, computed in the
+ *          same launch while the plan is still on chip -- exactly the figures
+ *          of eplb_plan_stats(loads, phy2log, logcnt) (same fp64 operations in
+ *          the same order, so bit-identical).  Rows rejected with
+ *          EPLB_ERR_RANGE get NaN.
  * Limits:  1 <= E <= 1024, E <= P <= 2048, G | E, gpus | P, N | gpus (hierarchical),
  *          X >= 1, R >= 0.
  */
 eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P,
                            int32_t G, int32_t N, int32_t gpus, int32_t X,
                            int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
-                           int32_t *log2phy, int32_t *status, cudaStream_t stream);
+                           int32_t *log2phy, double *gpu_load, double *stats,
+                           int32_t *status, cudaStream_t stream);
 
 /*
  * S2 + S3/S4 for a serving ring -- rebalance from the window sum of a ring
@@ -139,7 +146,8 @@ eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P
  *   loads[r, e] = sum_{w < W} ring[w, r, e]     (the window of the last W
  *                 steps, row order irrelevant: eplb_window_accumulate with
  *                 S = W, s_first = W - 1)
- * then exactly eplb_rebalance on those loads (same outputs, limits, errors).
+ * then exactly eplb_rebalance on those loads (same outputs, plan quality,
+ * limits, errors).
  * ring       device int64 [W, R, E]; each window sum must lie in [0, 2^40).
  * zero_slot  -1, or the ring row to clear after it has been read (the slot
  *            the next step's counts go to, e.g. with eplb_count_redirect and
@@ -150,7 +158,8 @@ eplb_status eplb_rebalance_window(int64_t *ring, int64_t W, int64_t zero_slot, i
                                   int32_t E, int32_t P, int32_t G, int32_t N, int32_t gpus,
                                   int32_t X, int64_t *loads_out, int32_t *phy2log,
                                   int32_t *phyrank, int32_t *logcnt, int32_t *log2phy,
-                                  int32_t *status, cudaStream_t stream);
+                                  double *gpu_load, double *stats, int32_t *status,
+                                  cudaStream_t stream);
 
 /*
  * S5 -- redirect logical expert indices to physical replicas ([LPLB] usage
@@ -200,8 +209,9 @@ eplb_status eplb_count_redirect(const int32_t *idx, int64_t L, int64_t T, int32_
  *   2. then, for every layer l, exactly eplb_rebalance_window on row l of the
  *      ring [W, L, E] (the window sum over all W slots, this batch included)
  *      into next_phy2log / next_phyrank / next_logcnt / next_log2phy, writing
- *      loads_out (nullable) and clearing ring row zero_slot (-1: none) after
- *      the sum was read.
+ *      loads_out and the plan quality gpu_load [L, gpus] / stats [L, 4] (all
+ *      nullable) and clearing ring row zero_slot (-1: none) after the sum
+ *      was read.
  * A layer's plan is built by the CTA that finishes the layer's last chunk,
  * while other layers are still being redirected.
  * ring         device int64 [W, L, E]; ring[slot] must hold the counts that
@@ -222,7 +232,8 @@ eplb_status eplb_serve_step(const int32_t *idx, int64_t L, int64_t T, int32_t K,
                             int64_t slot, int64_t zero_slot, int32_t P, int32_t G, int32_t N,
                             int32_t gpus, int64_t *loads_out, int32_t *next_phy2log,
                             int32_t *next_phyrank, int32_t *next_logcnt, int32_t *next_log2phy,
-                            uint32_t *layer_done, int32_t *status, cudaStream_t stream);
+                            double *gpu_load, double *stats, uint32_t *layer_done,
+                            int32_t *status, cudaStream_t stream);
 
 /*
  * eplb_serve_step without the caller's layer_done array: the per-layer
@@ -245,8 +256,8 @@ eplb_status eplb_serve_step_noalloc(const int32_t *idx, int64_t L, int64_t T, in
                                     int64_t slot, int64_t zero_slot, int32_t P, int32_t G,
                                     int32_t N, int32_t gpus, int64_t *loads_out,
                                     int32_t *next_phy2log, int32_t *next_phyrank,
-                                    int32_t *next_logcnt, int32_t *next_log2phy, int32_t *status,
-                                    cudaStream_t stream);
+                                    int32_t *next_logcnt, int32_t *next_log2phy, double *gpu_load,
+                                    double *stats, int32_t *status, cudaStream_t stream);
 
 /*
  * Plan quality ([EPLB] box "От переводчика: что на рисунке": per-GPU load of

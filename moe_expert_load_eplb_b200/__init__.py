@@ -79,19 +79,19 @@ def load_library():
         "eplb_abi_version": ([], i32),
         "eplb_count_loads": ([p, i64, i64, i32, i32, p, i32, p, p], i32),
         "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, p], i32),
-        "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p], i32),
+        "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p], i32),
         "eplb_redirect": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, p], i32),
         "eplb_count_redirect": ([p, i64, i64, i32, i32, p, i32, p, i32, p, i64, p, p, p, p], i32),
         "eplb_plan_stats": ([p, p, p, i64, i32, i32, i32, p, p, p, p], i32),
-        "eplb_rebalance_window": ([p, i64, i64, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p, p],
-                                  i32),
+        "eplb_rebalance_window": ([p, i64, i64, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p,
+                                   p, p, p], i32),
         "eplb_fold_loads": ([p, p, i64, i32, i32, p, p, p], i32),
         "eplb_initial_map": ([i64, i32, i32, p, p, p], i32),
         "eplb_plan_diff": ([p, p, i64, i32, i32, i32, p, p, p, p], i32),
         "eplb_serve_step": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, i64, i64, i64,
-                             i32, i32, i32, i32, p, p, p, p, p, p, p, p], i32),
+                             i32, i32, i32, i32, p, p, p, p, p, p, p, p, p, p], i32),
         "eplb_serve_step_noalloc": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, i64, i64,
-                                     i64, i32, i32, i32, i32, p, p, p, p, p, p, p], i32),
+                                     i64, i32, i32, i32, i32, p, p, p, p, p, p, p, p, p], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -144,6 +144,20 @@ def _word(t: Optional[torch.Tensor], dtypes, name: str, device: torch.device):
 def _words(device: torch.device, bad=None, status=None):
     _word(bad, _BAD_DTYPES, "bad", device)
     _word(status, (torch.int32,), "status", device)
+
+
+def _check_quality(gpu_load: Optional[torch.Tensor], stats: Optional[torch.Tensor], R: int,
+                   gpus: int, device: torch.device):
+    """The optional plan-quality outputs: float64 gpu_load [R, gpus] and
+    stats [R, 4] (min, max, mean, mean / max of the GPU loads)."""
+    if gpu_load is not None:
+        _cuda(gpu_load, torch.float64, "gpu_load", device)
+        if tuple(gpu_load.shape) != (R, gpus):
+            raise ValueError(f"gpu_load must be {(R, gpus)}")
+    if stats is not None:
+        _cuda(stats, torch.float64, "stats", device)
+        if tuple(stats.shape) != (R, 4):
+            raise ValueError(f"stats must be {(R, 4)}")
 
 
 def _check_plan(plan, name: str, R: int, E: int, X: int, P: Optional[int],
@@ -247,9 +261,12 @@ def default_slots(num_logical: int, num_replicas: int, num_groups: int, num_node
 
 def rebalance(loads: torch.Tensor, num_replicas: int, num_groups: int, num_nodes: int,
               num_gpus: int, slots: Optional[int] = None, out: Optional[Plan] = None,
-              status: Optional[torch.Tensor] = None) -> Plan:
+              status: Optional[torch.Tensor] = None, gpu_load: Optional[torch.Tensor] = None,
+              stats: Optional[torch.Tensor] = None) -> Plan:
     """S3/S4: rebalance_experts for every row of int64 loads [R, E] (hierarchical
-    policy when num_groups % num_nodes == 0, else global)."""
+    policy when num_groups % num_nodes == 0, else global).  ``gpu_load``
+    (float64 [R, gpus]) and ``stats`` (float64 [R, 4]), if given, receive the
+    new plans' quality in the same launch (the figures of ``plan_stats``)."""
     _cuda(loads, torch.int64, "loads")
     if loads.dim() != 2:
         raise ValueError("loads must be [R, E]")
@@ -268,21 +285,24 @@ def rebalance(loads: torch.Tensor, num_replicas: int, num_groups: int, num_nodes
         if tuple(t.shape) != shape:
             raise ValueError(f"{name} must be {shape}")
     _words(dev, status=status)
+    _check_quality(gpu_load, stats, R, num_gpus, dev)
     with _on_device(dev):
         _check(load_library().eplb_rebalance(
             _ptr(loads), R, E, P, num_groups, num_nodes, num_gpus, X,
             _ptr(out.phy2log), _ptr(out.phyrank), _ptr(out.logcnt), _ptr(out.log2phy),
-            _ptr(status), _stream(dev)), "eplb_rebalance")
+            _ptr(gpu_load), _ptr(stats), _ptr(status), _stream(dev)), "eplb_rebalance")
     return out
 
 
 def rebalance_window(ring: torch.Tensor, num_replicas: int, num_groups: int, num_nodes: int,
                      num_gpus: int, zero_slot: int = -1, slots: Optional[int] = None,
                      out: Optional[Plan] = None, loads_out: Optional[torch.Tensor] = None,
-                     status: Optional[torch.Tensor] = None) -> Plan:
+                     status: Optional[torch.Tensor] = None, gpu_load: Optional[torch.Tensor] = None,
+                     stats: Optional[torch.Tensor] = None) -> Plan:
     """S2 + S3/S4 in one launch: rebalance_experts on the window sum of a ring of
     per-step counts (int64 [W, R, E]); zero_slot >= 0 clears that ring row after
-    reading it (the next step's counting slot)."""
+    reading it (the next step's counting slot).  ``gpu_load`` / ``stats`` as
+    for ``rebalance``."""
     _cuda(ring, torch.int64, "ring")
     if ring.dim() != 3:
         raise ValueError("ring must be [W, R, E]")
@@ -305,11 +325,12 @@ def rebalance_window(ring: torch.Tensor, num_replicas: int, num_groups: int, num
         _cuda(loads_out, torch.int64, "loads_out", dev)
         if tuple(loads_out.shape) not in ((R, E), (1, R, E)):
             raise ValueError("loads_out must be [R, E]")
+    _check_quality(gpu_load, stats, R, num_gpus, dev)
     with _on_device(dev):
         _check(load_library().eplb_rebalance_window(
             _ptr(ring), Wr, zero_slot, R, E, P, num_groups, num_nodes, num_gpus, X, _ptr(loads_out),
             _ptr(out.phy2log), _ptr(out.phyrank), _ptr(out.logcnt), _ptr(out.log2phy),
-            _ptr(status), _stream(dev)), "eplb_rebalance_window")
+            _ptr(gpu_load), _ptr(stats), _ptr(status), _stream(dev)), "eplb_rebalance_window")
     return out
 
 
@@ -410,11 +431,14 @@ def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, nex
                layer_done: torch.Tensor, num_groups: int, num_nodes: int, num_gpus: int,
                zero_slot: int = -1, token_offset: int = 0, out: Optional[torch.Tensor] = None,
                loads_out: Optional[torch.Tensor] = None, bad: Optional[torch.Tensor] = None,
-               status: Optional[torch.Tensor] = None) -> torch.Tensor:
+               status: Optional[torch.Tensor] = None, gpu_load: Optional[torch.Tensor] = None,
+               stats: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The serving step in one launch: count idx into ring[slot] and redirect it
     with ``plan`` (the plan in force), then rebuild every layer's plan from the
     window sum over the ring into ``next_plan`` (clearing ring[zero_slot]).
-    ``layer_done``: uint32 [L] work array, zero before and after.  Returns out."""
+    ``layer_done``: uint32 [L] work array, zero before and after;
+    ``gpu_load`` / ``stats``: the next plan's quality, as for ``rebalance``.
+    Returns out."""
     L, T, K, Wr, E, P, X, out = _serve_args(idx, plan, ring, next_plan, out, loads_out, bad,
                                             status)
     if not isinstance(layer_done, torch.Tensor) or not layer_done.is_cuda or \
@@ -422,13 +446,14 @@ def serve_step(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: int, nex
         raise TypeError("layer_done must be a CUDA uint32 tensor of L elements")
     if not layer_done.is_contiguous() or layer_done.device != idx.device:
         raise ValueError("layer_done must be contiguous and on the device of idx")
+    _check_quality(gpu_load, stats, L, num_gpus, idx.device)
     with _on_device(idx.device):
         _check(load_library().eplb_serve_step(
             _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
             _ptr(out), _ptr(bad), _ptr(ring), Wr, slot, zero_slot, P, num_groups, num_nodes,
             num_gpus, _ptr(loads_out), _ptr(next_plan.phy2log), _ptr(next_plan.phyrank),
-            _ptr(next_plan.logcnt), _ptr(next_plan.log2phy), _ptr(layer_done), _ptr(status),
-            _stream(idx.device)), "eplb_serve_step")
+            _ptr(next_plan.logcnt), _ptr(next_plan.log2phy), _ptr(gpu_load), _ptr(stats),
+            _ptr(layer_done), _ptr(status), _stream(idx.device)), "eplb_serve_step")
     return out
 
 
@@ -438,19 +463,22 @@ def serve_step_noalloc(idx: torch.Tensor, plan: Plan, ring: torch.Tensor, slot: 
                        out: Optional[torch.Tensor] = None,
                        loads_out: Optional[torch.Tensor] = None,
                        bad: Optional[torch.Tensor] = None,
-                       status: Optional[torch.Tensor] = None) -> torch.Tensor:
+                       status: Optional[torch.Tensor] = None,
+                       gpu_load: Optional[torch.Tensor] = None,
+                       stats: Optional[torch.Tensor] = None) -> torch.Tensor:
     """serve_step with the library's own per-layer counters (no work array;
     calls must not overlap on one device).  ``out`` must be given or is
     allocated here by torch, outside the call."""
     L, T, K, Wr, E, P, X, out = _serve_args(idx, plan, ring, next_plan, out, loads_out, bad,
                                             status)
+    _check_quality(gpu_load, stats, L, num_gpus, idx.device)
     with _on_device(idx.device):
         _check(load_library().eplb_serve_step_noalloc(
             _ptr(idx), L, T, K, E, _ptr(plan.log2phy), X, _ptr(plan.logcnt), int(token_offset),
             _ptr(out), _ptr(bad), _ptr(ring), Wr, slot, zero_slot, P, num_groups, num_nodes,
             num_gpus, _ptr(loads_out), _ptr(next_plan.phy2log), _ptr(next_plan.phyrank),
-            _ptr(next_plan.logcnt), _ptr(next_plan.log2phy), _ptr(status),
-            _stream(idx.device)), "eplb_serve_step_noalloc")
+            _ptr(next_plan.logcnt), _ptr(next_plan.log2phy), _ptr(gpu_load), _ptr(stats),
+            _ptr(status), _stream(idx.device)), "eplb_serve_step_noalloc")
     return out
 
 

@@ -40,21 +40,36 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _inputs())
 
 
+def _compile(cmd: list[str]) -> subprocess.CompletedProcess:
+    return subprocess.run(cmd, capture_output=True, text=True)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA source into one shared library (static cudart)."""
+    """Compile every CUDA source into one shared library (static cudart):
+    one nvcc per source file, in parallel, then one link."""
     if not force and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--use_fast_math",
-           "-Xcompiler", "-fPIC,-O3", "-shared", "-cudart", "static",
-           "-I", os.path.join(ROOT, "include"), "-o", tmp, *sources()]
+    import tempfile
+    from concurrent.futures import ThreadPoolExecutor
+    common = [_nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--use_fast_math",
+              "-Xcompiler", "-fPIC,-O3", "-I", os.path.join(ROOT, "include")]
     if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
-    if verbose:
-        sys.stderr.write(res.stdout + res.stderr)
+        common.insert(1, "-Xptxas=-v")
+    with tempfile.TemporaryDirectory(prefix="eplb_build_") as tmpdir:
+        objs = [os.path.join(tmpdir, os.path.basename(src) + ".o") for src in sources()]
+        cmds = [common + ["-c", src, "-o", obj] for src, obj in zip(sources(), objs)]
+        with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+            results = list(ex.map(_compile, cmds))
+        for cmd, res in zip(cmds, results):
+            if res.returncode != 0:
+                raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
+            if verbose:
+                sys.stderr.write(res.stdout + res.stderr)
+        tmp = LIB + f".tmp{os.getpid()}"
+        link = [_nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
+        res = _compile(link)
+        if res.returncode != 0:
+            raise RuntimeError("nvcc link failed:\n" + " ".join(link) + "\n" + res.stdout + res.stderr)
     os.replace(tmp, LIB)
     return LIB
 

@@ -207,29 +207,30 @@ static eplb_status rebalance_shape(int64_t R, int32_t E, int32_t P, int32_t G, i
 
 eplb_status eplb_rebalance(const int64_t *loads, int64_t R, int32_t E, int32_t P, int32_t G,
                            int32_t N, int32_t gpus, int32_t X, int32_t *phy2log,
-                           int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
-                           cudaStream_t stream) {
+                           int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, double *gpu_load,
+                           double *stats, int32_t *status, cudaStream_t stream) {
   RebalanceShape sh;
   const eplb_status st = rebalance_shape(R, E, P, G, N, gpus, X, &sh);
   if (st != EPLB_OK || R == 0) return st;
   if (!loads || !phy2log || !phyrank || !logcnt || !log2phy) return EPLB_ERR_NULL;
   // the kernel only reads the load array when no ring slot is cleared
   return launch_rebalance(const_cast<int64_t *>(loads), 1, -1, nullptr, R, sh, phy2log, phyrank,
-                          logcnt, log2phy, status, stream);
+                          logcnt, log2phy, gpu_load, stats, status, stream);
 }
 
 eplb_status eplb_rebalance_window(int64_t *ring, int64_t W, int64_t zero_slot, int64_t R,
                                   int32_t E, int32_t P, int32_t G, int32_t N, int32_t gpus,
                                   int32_t X, int64_t *loads_out, int32_t *phy2log,
                                   int32_t *phyrank, int32_t *logcnt, int32_t *log2phy,
-                                  int32_t *status, cudaStream_t stream) {
+                                  double *gpu_load, double *stats, int32_t *status,
+                                  cudaStream_t stream) {
   if (W < 1 || zero_slot < -1 || zero_slot >= W) return EPLB_ERR_SHAPE;
   RebalanceShape sh;
   const eplb_status st = rebalance_shape(R, E, P, G, N, gpus, X, &sh);
   if (st != EPLB_OK || R == 0) return st;
   if (!ring || !phy2log || !phyrank || !logcnt || !log2phy) return EPLB_ERR_NULL;
   return launch_rebalance(ring, W, zero_slot, loads_out, R, sh, phy2log, phyrank, logcnt, log2phy,
-                          status, stream);
+                          gpu_load, stats, status, stream);
 }
 
 eplb_status eplb_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
@@ -273,7 +274,8 @@ eplb_status eplb_serve_step(const int32_t *idx, int64_t L, int64_t T, int32_t K,
                             int64_t slot, int64_t zero_slot, int32_t P, int32_t G, int32_t N,
                             int32_t gpus, int64_t *loads_out, int32_t *next_phy2log,
                             int32_t *next_phyrank, int32_t *next_logcnt, int32_t *next_log2phy,
-                            uint32_t *layer_done, int32_t *status, cudaStream_t stream) {
+                            double *gpu_load, double *stats, uint32_t *layer_done,
+                            int32_t *status, cudaStream_t stream) {
   if (L < 0 || T < 0 || K < 1 || E < 1 || X < 1 || t0 < 0) return EPLB_ERR_SHAPE;
   if (W < 1 || slot < 0 || slot >= W || zero_slot < -1 || zero_slot >= W) return EPLB_ERR_SHAPE;
   if (E > 1024 || static_cast<int64_t>(E) * X > 32768) return EPLB_ERR_LIMIT;
@@ -290,7 +292,7 @@ eplb_status eplb_serve_step(const int32_t *idx, int64_t L, int64_t T, int32_t K,
   if (next_log2phy == log2phy || next_logcnt == logcnt) return EPLB_ERR_SHAPE;
   return launch_serve(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot, zero_slot,
                       loads_out, sh, next_phy2log, next_phyrank, next_logcnt, next_log2phy,
-                      layer_done, status, stream);
+                      gpu_load, stats, layer_done, status, stream);
 }
 
 eplb_status eplb_serve_step_noalloc(const int32_t *idx, int64_t L, int64_t T, int32_t K,
@@ -300,20 +302,20 @@ eplb_status eplb_serve_step_noalloc(const int32_t *idx, int64_t L, int64_t T, in
                                     int64_t slot, int64_t zero_slot, int32_t P, int32_t G,
                                     int32_t N, int32_t gpus, int64_t *loads_out,
                                     int32_t *next_phy2log, int32_t *next_phyrank,
-                                    int32_t *next_logcnt, int32_t *next_log2phy, int32_t *status,
-                                    cudaStream_t stream) {
+                                    int32_t *next_logcnt, int32_t *next_log2phy, double *gpu_load,
+                                    double *stats, int32_t *status, cudaStream_t stream) {
   if (L > kStaticLayers) return EPLB_ERR_LIMIT;
   if (L <= 0) {
     return eplb_serve_step(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot,
                            zero_slot, P, G, N, gpus, loads_out, next_phy2log, next_phyrank,
-                           next_logcnt, next_log2phy, nullptr, status, stream);
+                           next_logcnt, next_log2phy, gpu_load, stats, nullptr, status, stream);
   }
   uint32_t *counters = nullptr;
   const eplb_status cst = static_layer_done(&counters);
   if (cst != EPLB_OK) return cst;
   return eplb_serve_step(idx, L, T, K, E, log2phy, X, logcnt, t0, out, bad, ring, W, slot,
                          zero_slot, P, G, N, gpus, loads_out, next_phy2log, next_phyrank,
-                         next_logcnt, next_log2phy, counters, status, stream);
+                         next_logcnt, next_log2phy, gpu_load, stats, counters, status, stream);
 }
 
 eplb_status eplb_plan_stats(const int64_t *loads, const int32_t *phy2log, const int32_t *logcnt,

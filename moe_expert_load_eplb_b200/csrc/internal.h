@@ -68,8 +68,8 @@ struct RebalanceShape {
 // load array); zero_slot >= 0 clears that ring row after reading it.
 eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, int64_t *loads_out,
                              int64_t R, const RebalanceShape &sh, int32_t *phy2log,
-                             int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
-                             cudaStream_t stream);
+                             int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, double *gpu_load,
+                             double *stats, int32_t *status, cudaStream_t stream);
 
 // Redirect; with counts != nullptr the same pass also adds the load histogram.
 eplb_status launch_redirect(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
@@ -85,8 +85,9 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
                          int32_t *out, unsigned long long *bad, int64_t *ring, int64_t W,
                          int64_t slot, int64_t zero_slot, int64_t *loads_out,
                          const RebalanceShape &sh, int32_t *next_phy2log, int32_t *next_phyrank,
-                         int32_t *next_logcnt, int32_t *next_log2phy, uint32_t *layer_done,
-                         int32_t *status, cudaStream_t stream);
+                         int32_t *next_logcnt, int32_t *next_log2phy, double *gpu_load,
+                         double *stats, uint32_t *layer_done, int32_t *status,
+                         cudaStream_t stream);
 
 // Device address of the library-owned per-layer counters of
 // eplb_serve_step_noalloc (kStaticLayers of them) on the current device,

@@ -28,8 +28,8 @@ __global__ void __launch_bounds__(kMaxThreads) rebalance_kernel(RbArgs a) {
 
 eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, int64_t *loads_out,
                              int64_t R, const RebalanceShape &sh, int32_t *phy2log,
-                             int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, int32_t *status,
-                             cudaStream_t stream) {
+                             int32_t *phyrank, int32_t *logcnt, int32_t *log2phy, double *gpu_load,
+                             double *stats, int32_t *status, cudaStream_t stream) {
   DeviceInfo di;
   const eplb_status dst = device_info(&di);
   if (dst != EPLB_OK) return dst;
@@ -50,6 +50,8 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
   a.logcnt = logcnt;
   a.log2phy = log2phy;
   a.status = status;
+  a.gpu_load = gpu_load;
+  a.stats = stats;
   a.s = sh;
   a.x_magic = 0xffffffffu / static_cast<uint32_t>(sh.X);
   a.table_vec4 = ((static_cast<int64_t>(sh.E) * sh.X) % 4 == 0) &&

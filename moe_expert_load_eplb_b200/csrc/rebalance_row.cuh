@@ -87,6 +87,9 @@ struct RbArgs {
   int64_t ring_w, ring_stride, zero_slot;
   int64_t *loads_out;
   int32_t *phy2log, *phyrank, *logcnt, *log2phy, *status;
+  // plan quality (nullable): per-GPU load [R, gpus] and {min, max, mean,
+  // mean / max} [R, 4] of the plan just built, fp64
+  double *gpu_load, *stats;
   RebalanceShape s;
   uint32_t x_magic;
   int table_vec4;  // log2phy rows may be written as 16-byte vectors
@@ -656,16 +659,59 @@ __device__ EPLB_RB_COLD void replicate_smem(int lpn, int ppn, int n, const int64
   }
 }
 
-// The plan of a row that cannot be computed: no replicas, log2phy all -1.
-__device__ void write_error_row(int32_t *phy2log, int32_t *phyrank, int32_t *logcnt,
-                                             int32_t *log2phy, int P, int E, int X, int64_t row) {
+// The plan of a row that cannot be computed: no replicas, log2phy all -1,
+// plan quality NaN.
+__device__ void write_error_row(const RbArgs &a, int64_t row) {
+  const int P = a.s.P, E = a.s.E, X = a.s.X, gpus = a.s.gpus;
   for (int t = threadIdx.x; t < P; t += nthr()) {
-    phy2log[row * P + t] = -1;
-    phyrank[row * P + t] = -1;
+    a.phy2log[row * P + t] = -1;
+    a.phyrank[row * P + t] = -1;
   }
-  for (int e = threadIdx.x; e < E; e += nthr()) logcnt[row * E + e] = 0;
-  int32_t *gl = log2phy + row * static_cast<int64_t>(E) * X;
+  for (int e = threadIdx.x; e < E; e += nthr()) a.logcnt[row * E + e] = 0;
+  int32_t *gl = a.log2phy + row * static_cast<int64_t>(E) * X;
   for (int i = threadIdx.x; i < E * X; i += nthr()) gl[i] = -1;
+  const double nan = __longlong_as_double(0x7ff8000000000000LL);
+  if (a.gpu_load)
+    for (int g = threadIdx.x; g < gpus; g += nthr()) a.gpu_load[row * gpus + g] = nan;
+  if (a.stats)
+    for (int k = threadIdx.x; k < 4; k += nthr()) a.stats[row * 4 + k] = nan;
+}
+
+// Plan quality of the row just assembled, by one warp (page "DualPipe и
+// EPLB", Part 2, box "От переводчика: что на рисунке": per-GPU loads of the
+// worked example; exercise 2 of "что сделать руками": max against mean).
+// q[p] = w / logcnt of slot p's expert (fp64, rounded to nearest); GPU g's
+// load is the sum of its slots' q in slot order from 0.0, then min, max and
+// the mean of the GPU loads summed in GPU order, and balancedness = mean /
+// max (1 when max is 0).  Every operation is an explicitly rounded fp64 add
+// or divide in that fixed order, so the figures are bit-identical to the
+// same sums done sequentially on a CPU.
+// Operands are plain values: an out-of-line call given the kernel's
+// parameter block by reference needs a stack copy of it (it doubled the
+// kernel's registers).
+__device__ EPLB_RB_COLD void plan_quality(double *gpu_load, double *stats, int64_t row, int gpus,
+                                          int ppg, const double *q, double *gl) {
+  const int lane = threadIdx.x & 31;
+  for (int g = lane; g < gpus; g += 32) {
+    double acc = 0.0;
+    for (int k = 0; k < ppg; ++k) acc = __dadd_rn(acc, q[g * ppg + k]);
+    gl[g] = acc;
+    if (gpu_load) gpu_load[row * gpus + g] = acc;
+  }
+  __syncwarp();
+  if (lane == 0 && stats) {
+    double mn = gl[0], mx = gl[0], sum = 0.0;
+    for (int g = 0; g < gpus; ++g) {
+      mn = fmin(mn, gl[g]);
+      mx = fmax(mx, gl[g]);
+      sum = __dadd_rn(sum, gl[g]);
+    }
+    const double mean = __ddiv_rn(sum, static_cast<double>(gpus));
+    stats[row * 4 + 0] = mn;
+    stats[row * 4 + 1] = mx;
+    stats[row * 4 + 2] = mean;
+    stats[row * 4 + 3] = mx > 0.0 ? __ddiv_rn(mean, mx) : 1.0;
+  }
 }
 
 // Operands of step 3 as plain values (an out-of-line instance then needs no
@@ -791,7 +837,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     }
   }
   if (__syncthreads_or(bad)) {
-    write_error_row(a.phy2log, a.phyrank, a.logcnt, a.log2phy, s.P, s.E, s.X, row);
+    write_error_row(a, row);
     if (tid == 0) report(a.status, EPLB_ERR_RANGE);
     return;
   }
@@ -927,7 +973,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     __syncthreads();
   }
   if (flags[1]) {
-    write_error_row(a.phy2log, a.phyrank, a.logcnt, a.log2phy, s.P, s.E, s.X, row);
+    write_error_row(a, row);
     if (tid == 0) report(a.status, EPLB_ERR_RANGE);
     return;
   }
@@ -958,12 +1004,19 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
   const bool in_smem = table_in_smem(s);
   int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
+  // plan quality: slot quotients w / logcnt, in the sort keys' space (free
+  // after step 3)
+  const bool quality = a.gpu_load != nullptr || a.stats != nullptr;
+  double *qslot = reinterpret_cast<double *>(smem + lay.keys);
   bool slots = false;
   for (int t = tid; t < s.P; t += nthr()) {
     const int n = t / s.ppn;
     const int pphy = n * s.ppn + ipack[t] * s.ppg + irank[t];
-    const int e = mlog2log[n * s.lpn + p2m[t]];
+    const int m = n * s.lpn + p2m[t];
+    const int e = mlog2log[m];
     const int k = rrank[t];
+    if (quality)
+      qslot[pphy] = __ddiv_rn(static_cast<double>(w[e]), static_cast<double>(cnt[m]));
     a.phy2log[row * s.P + pphy] = e;
     a.phyrank[row * s.P + pphy] = k;
     if (in_smem) {
@@ -982,6 +1035,11 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     a.logcnt[row * s.E + e] = cnt[m];
   }
   __syncthreads();
+  // warp 0 sums the plan quality (pack weights' space, free after step 3)
+  // while the other warps start copying the table out
+  if (quality && tid < 32)
+    plan_quality(a.gpu_load, a.stats, row, s.gpus, s.ppg, qslot,
+                 reinterpret_cast<double *>(smem + lay.pw));
   if (in_smem) {
     if (a.table_vec4) {
       const int4 *src = reinterpret_cast<const int4 *>(tbl);

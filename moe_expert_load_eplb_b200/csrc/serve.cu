@@ -64,8 +64,9 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
                          int32_t *out, unsigned long long *bad, int64_t *ring, int64_t W,
                          int64_t slot, int64_t zero_slot, int64_t *loads_out,
                          const RebalanceShape &sh, int32_t *next_phy2log, int32_t *next_phyrank,
-                         int32_t *next_logcnt, int32_t *next_log2phy, uint32_t *layer_done,
-                         int32_t *status, cudaStream_t stream) {
+                         int32_t *next_logcnt, int32_t *next_log2phy, double *gpu_load,
+                         double *stats, uint32_t *layer_done, int32_t *status,
+                         cudaStream_t stream) {
   DeviceInfo di;
   const eplb_status dst = device_info(&di);
   if (dst != EPLB_OK) return dst;
@@ -89,6 +90,8 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
   a.b.logcnt = next_logcnt;
   a.b.log2phy = next_log2phy;
   a.b.status = status;
+  a.b.gpu_load = gpu_load;
+  a.b.stats = stats;
   a.b.s = sh;
   a.b.x_magic = 0xffffffffu / static_cast<uint32_t>(sh.X);
   a.b.table_vec4 = ((static_cast<int64_t>(sh.E) * sh.X) % 4 == 0) &&

@@ -6,12 +6,17 @@
 //   snaps[s - s_first, c] = sum_{u=max(0,s-W+1)}^{s} steps[u, c],  s >= s_first,
 // i.e. a prefix scan along s of d[u] = steps[u] - steps[u-W].
 //
-// HBM-streaming design: a CTA owns a strip of `cw` adjacent columns and walks
-// all S rows in blocks of rg*U rows.  Thread (g, col) loads U rows of its
-// column (U independent 8-byte loads in flight per thread, coalesced across
-// the strip), scans them in registers, and the rg row-group totals are
-// combined through shared memory into the strip's running carry.  The strip
-// width is chosen on the host so the strip count fills the SMs evenly.
+// HBM-streaming design: a CTA owns a strip of kCols = 32 adjacent columns
+// (one warp reads one 256-byte row segment: coalesced) and walks all S rows
+// in blocks of rg * kU rows (kU = 8, or 4 when rows s - W are read too).  Warp g of the CTA holds rows g*kU .. g*kU+kU-1
+// of the block for its 32 columns; it scans them in registers, the rg warp
+// totals are combined through shared memory into the strip's running carry.
+// The next block's kU loads per thread are issued before the current block
+// is scanned (two blocks in registers), so a thread keeps kU independent
+// 8-byte loads in flight while it waits on the barrier and writes; rows
+// s - W are loaded only in blocks that reach them (none when W >= S).  With
+// up to 16 warps per CTA and several CTAs per SM this keeps 64-128 KB of
+// reads in flight per SM, which HBM3e needs for its bandwidth.
 #include <algorithm>
 
 #include "common.cuh"
@@ -20,51 +25,81 @@
 namespace eplb {
 namespace {
 
-constexpr int kU = 8;  // rows per thread per block
+constexpr int kCols = 32;    // columns per strip: one warp-wide row segment
+constexpr int kMaxRg = 16;   // row groups (warps) per CTA
 
-__global__ void window_kernel(const int64_t *__restrict__ steps, int64_t S, int64_t C, int64_t W,
-                              int64_t s_first, int64_t *__restrict__ snaps, int cw, int rg) {
-  extern __shared__ int64_t part[];  // [rg][cw]
+// kU rows per thread per block; kSub: some row s has s - W >= 0 (W < S), so
+// blocks that reach row W also load rows s - W.  Without it a block is kU
+// loads per thread; with it 2 kU, so it takes half the rows per block.
+template <int kU, bool kSub>
+struct WinBlock {
+  int64_t add[kU];
+  int64_t sub[kSub ? kU : 1];
+
+  __device__ __forceinline__ void load(const int64_t *__restrict__ steps, int64_t S, int64_t C,
+                                       int64_t W, int64_t r0, int64_t c, bool col_ok) {
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t r = r0 + u;
+      add[u] = (col_ok && r < S) ? __ldcs(steps + r * C + c) : 0;
+    }
+    if (kSub) {
+      const bool any_sub = r0 + kU - 1 >= W;  // warp-uniform: r0 is the warp's first row
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t r = r0 + u;
+        sub[kSub ? u : 0] = (any_sub && col_ok && r < S && r >= W) ? __ldg(steps + (r - W) * C + c) : 0;
+      }
+    }
+  }
+  __device__ __forceinline__ int64_t d(int u) const { return kSub ? add[u] - sub[kSub ? u : 0] : add[u]; }
+};
+
+template <int kU, bool kSub>
+__global__ void __launch_bounds__(kCols * kMaxRg) window_kernel(
+    const int64_t *__restrict__ steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
+    int64_t *__restrict__ snaps) {
+  __shared__ int64_t part[kMaxRg][kCols];
   pdl_trigger();
   pdl_wait();
-  const int tid = threadIdx.x;
-  const int col = tid % cw;
-  const int g = tid / cw;
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * cw + col;
-  const bool active = (g < rg) && (c < C);
+  const int col = threadIdx.x;  // blockDim = (kCols, rg)
+  const int g = threadIdx.y;
+  const int rg = blockDim.y;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kCols + col;
+  const bool col_ok = c < C;
   const int64_t rows_per_blk = static_cast<int64_t>(rg) * kU;
 
+  WinBlock<kU, kSub> cur, nxt;
+  cur.load(steps, S, C, W, static_cast<int64_t>(g) * kU, c, col_ok);
   int64_t carry = 0;
   for (int64_t blk = 0; blk < S; blk += rows_per_blk) {
     const int64_t r0 = blk + static_cast<int64_t>(g) * kU;
-    int64_t add[kU], sub[kU];
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t r = r0 + u;
-      add[u] = (active && r < S) ? __ldcs(steps + r * C + c) : 0;
-      sub[u] = (active && r < S && r >= W) ? __ldg(steps + (r - W) * C + c) : 0;
-    }
+    // the next block's loads go out before this block is scanned
+    if (blk + rows_per_blk < S) nxt.load(steps, S, C, W, r0 + rows_per_blk, c, col_ok);
     int64_t acc = 0;
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
-      acc += add[u] - sub[u];
-      add[u] = acc;  // inclusive prefix within this thread's rows
+      acc += cur.d(u);
+      cur.add[u] = acc;  // inclusive prefix within this thread's rows
     }
-    if (g < rg) part[g * cw + col] = acc;
+    part[g][col] = acc;
     __syncthreads();
-    int64_t pre = carry, tot = 0;
+    int64_t before = carry, tot = 0;
     for (int h = 0; h < rg; ++h) {
-      const int64_t p = part[h * cw + col];
-      pre += (h < g) ? p : 0;
+      const int64_t p = part[h][col];
+      before += (h < g) ? p : 0;
       tot += p;
     }
+    if (col_ok && r0 + kU > s_first) {
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t r = r0 + u;
-      if (active && r < S && r >= s_first) __stcs(snaps + (r - s_first) * C + c, pre + add[u]);
+      for (int u = 0; u < kU; ++u) {
+        const int64_t r = r0 + u;
+        if (r < S && r >= s_first) __stcs(snaps + (r - s_first) * C + c, before + cur.add[u]);
+      }
     }
     carry += tot;
     __syncthreads();
+    cur = nxt;
   }
 }
 
@@ -75,36 +110,29 @@ eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W,
   DeviceInfo di;
   const eplb_status dst = device_info(&di);
   if (dst != EPLB_OK) return dst;
-  // Pick the strip width cw and row groups rg: rg never exceeds the row
-  // blocks there are (short rings), the strip count fills the SMs evenly
-  // (strips per SM rounded up cost the tail), and enough threads per SM keep
-  // loads in flight.
-  const int64_t max_rg = std::max<int64_t>(1, (S + kU - 1) / kU);
-  int best_cw = 32;
-  double best_score = -1.0;
-  for (int cw = 8; cw <= 256; ++cw) {
-    const int rg = static_cast<int>(std::min<int64_t>(std::max(1, 256 / cw), max_rg));
-    if (cw * rg > 1024) continue;
-    const int64_t strips = (C + cw - 1) / cw;
-    const int64_t waves = (strips + di.sms - 1) / di.sms;
-    const double balance = static_cast<double>(strips) / static_cast<double>(waves * di.sms);
-    const double per_sm_threads = static_cast<double>(std::min<int64_t>(strips, waves * di.sms)) /
-                                  di.sms * cw * rg;
-    const double inflight = std::min(1.0, per_sm_threads / 1024.0);
-    const double score = balance * inflight;
-    if (score > best_score + 1e-9) {
-      best_score = score;
-      best_cw = cw;
+  const bool sub = W < S;
+  const int u = sub ? 4 : 8;
+  const int64_t strips = (C + kCols - 1) / kCols;
+  if (strips > 0x7fffffffLL) return EPLB_ERR_LIMIT;
+  const void *fn = sub ? reinterpret_cast<const void *>(window_kernel<4, true>)
+                       : reinterpret_cast<const void *>(window_kernel<8, false>);
+  // row groups: no more warps than the rows fill (up to kMaxRg), and the
+  // most that still let every strip's CTA be resident at once (one wave:
+  // a second, partial wave would leave SMs idle while it runs)
+  const int rg_rows = static_cast<int>(std::min<int64_t>(kMaxRg, std::max<int64_t>(1, (S + u - 1) / u)));
+  int rg = rg_rows;
+  for (int cand = rg_rows; cand >= 1; --cand) {
+    int per_sm = 0;
+    const eplb_status pst = prepare_kernel(fn, kCols * cand, 0, &per_sm);
+    if (pst != EPLB_OK) return pst;
+    if (static_cast<int64_t>(per_sm) * di.sms >= strips) {
+      rg = cand;
+      break;
     }
   }
-  const int cw = static_cast<int>(std::min<int64_t>(best_cw, C));
-  const int rg = static_cast<int>(std::min<int64_t>(std::max(1, 256 / cw), max_rg));
-  const int64_t strips = (C + cw - 1) / cw;
-  const size_t smem = static_cast<size_t>(rg) * cw * sizeof(int64_t);
-  void *args[] = {&steps, &S, &C, &W, &s_first, &snaps, const_cast<int *>(&cw), const_cast<int *>(&rg)};
-  const cudaError_t err = launch_pdl(reinterpret_cast<const void *>(window_kernel),
-                                     dim3(static_cast<unsigned>(strips)), dim3(cw * rg), smem, stream,
-                                     args);
+  void *args[] = {&steps, &S, &C, &W, &s_first, &snaps};
+  const cudaError_t err = launch_pdl(fn, dim3(static_cast<unsigned>(strips)), dim3(kCols, rg), 0,
+                                     stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);
 }
 

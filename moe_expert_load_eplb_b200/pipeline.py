@@ -48,7 +48,7 @@ class EplbStep:
     def __init__(self, L: int, T: int, K: int, E: int, P: int, G: int, N: int, gpus: int,
                  window: int = 1, device="cuda", slots: Optional[int] = None,
                  token_offset: int = 0, group=None, fused: bool = True,
-                 single_launch: bool = False):
+                 single_launch: bool = False, quality: bool = True):
         self.L, self.T, self.K, self.E = L, T, K, E
         self.P, self.G, self.N, self.gpus = P, G, N, gpus
         self.W = window
@@ -69,6 +69,10 @@ class EplbStep:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.bad = torch.zeros(1, dtype=torch.int64, device=dev)
         self.layer_done = torch.zeros(L, dtype=torch.uint32, device=dev)
+        # quality of the newest plan, computed by the launch that builds it:
+        # per-GPU load [L, gpus] and {min, max, mean, mean / max} [L, 4]
+        self.gpu_load = torch.zeros((L, gpus), dtype=torch.float64, device=dev) if quality else None
+        self.stats = torch.zeros((L, 4), dtype=torch.float64, device=dev) if quality else None
         self.steps_done = 0
         self.primed = False
 
@@ -132,7 +136,7 @@ class EplbStep:
     def _plan_from_ring(self, plan: Plan):
         window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads)
         rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=plan,
-                  status=self.status)
+                  status=self.status, gpu_load=self.gpu_load, stats=self.stats)
 
     def __call__(self, idx: torch.Tensor, marks: Optional[Sequence] = None):
         """Run one step on idx (int32 [L, T, K]).
@@ -156,7 +160,7 @@ class EplbStep:
             serve_step(idx, used, self.ring, self.steps_done % self.W, nxt, self.layer_done, self.G,
                        self.N, self.gpus, zero_slot=(self.steps_done + 1) % self.W,
                        token_offset=self.token_offset, out=self.out, loads_out=self.loads,
-                       bad=self.bad, status=self.status)
+                       bad=self.bad, status=self.status, gpu_load=self.gpu_load, stats=self.stats)
             for k in range(1, 6):
                 rec(k)
             self.steps_done += 1
@@ -177,13 +181,14 @@ class EplbStep:
             nxt = self.plans[1 - self.cur]
             rebalance_window(self.ring, self.P, self.G, self.N, self.gpus,
                              zero_slot=(self.steps_done + 1) % self.W, slots=self.X, out=nxt,
-                             loads_out=self.loads, status=self.status)
+                             loads_out=self.loads, status=self.status, gpu_load=self.gpu_load,
+                             stats=self.stats)
         else:
             window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads)
             rec(3)
             nxt = used
             rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=nxt,
-                      status=self.status)
+                      status=self.status, gpu_load=self.gpu_load, stats=self.stats)
         rec(4)
         if not self.fused:
             redirect(idx, nxt.log2phy, nxt.logcnt, self.token_offset, out=self.out, bad=self.bad,

@@ -69,14 +69,14 @@ def test_host_argument_checks(lib):
     assert lib.eplb_window_accumulate(None, 4, 2, 3, 2, 0, one, None) == 1
     # rebalance: divisibility, shape, limits; R == 0 needs no device
     rb = lib.eplb_rebalance
-    assert rb(one, 1, 12, 16, 5, 2, 8, 5, one, one, one, one, None, None) == 3   # 12 % 5
-    assert rb(one, 1, 12, 18, 4, 2, 8, 5, one, one, one, one, None, None) == 3   # 18 % 8
-    assert rb(one, 1, 12, 8, 4, 2, 8, 5, one, one, one, one, None, None) == 2    # P < E
-    assert rb(one, 1, 12, 18, 4, 4, 6, 5, one, one, one, one, None, None) == 3   # hier: 6 % 4
-    assert rb(one, 1, 2048, 4096, 8, 4, 32, 5, one, one, one, one, None, None) == 9
-    assert rb(one, 1, 12, 16, 4, 2, 8, 0, one, one, one, one, None, None) == 2   # X < 1
-    assert rb(one, 0, 12, 18, 3, 2, 3, 7, None, None, None, None, None, None) == 0  # global, R = 0
-    assert rb(None, 1, 12, 16, 4, 2, 8, 5, one, one, one, one, None, None) == 1
+    assert rb(one, 1, 12, 16, 5, 2, 8, 5, one, one, one, one, None, None, None, None) == 3   # 12 % 5
+    assert rb(one, 1, 12, 18, 4, 2, 8, 5, one, one, one, one, None, None, None, None) == 3   # 18 % 8
+    assert rb(one, 1, 12, 8, 4, 2, 8, 5, one, one, one, one, None, None, None, None) == 2    # P < E
+    assert rb(one, 1, 12, 18, 4, 4, 6, 5, one, one, one, one, None, None, None, None) == 3   # hier: 6 % 4
+    assert rb(one, 1, 2048, 4096, 8, 4, 32, 5, one, one, one, one, None, None, None, None) == 9
+    assert rb(one, 1, 12, 16, 4, 2, 8, 0, one, one, one, one, None, None, None, None) == 2   # X < 1
+    assert rb(one, 0, 12, 18, 3, 2, 3, 7, None, None, None, None, None, None, None, None) == 0  # global, R = 0
+    assert rb(None, 1, 12, 16, 4, 2, 8, 5, one, one, one, one, None, None, None, None) == 1
     # redirect: shape, limits, alignment
     rd = lib.eplb_redirect
     assert rd(one, 1, 4, 2, 8, one, 0, one, 0, one, None, None, None) == 2

@@ -866,6 +866,109 @@ def test_plan_stats_worked_example_gpu():
     assert _np(st)[0, 0] == h["min"] and _np(st)[0, 1] == h["max"]
 
 
+def _quality_bufs(R, gpus):
+    return (torch.full((R, gpus), -7.0, dtype=torch.float64, device=DEV),
+            torch.full((R, 4), -7.0, dtype=torch.float64, device=DEV))
+
+
+@pytest.mark.parametrize("cfg", ["tiny", "dsv3_prefill", "global_policy"])
+def test_rebalance_fused_quality_matches_oracle(cfg, request):
+    """The plan quality written by the rebalance launch itself equals the
+    oracle's plan_stats of the oracle's plan, bit for bit (fp64, same order)."""
+    c = W.WORKLOADS[cfg]
+    if cfg == "global_policy":
+        loads_np = W.global_policy_loads()
+    else:
+        idx = request.getfixturevalue({"tiny": "tiny_idx", "dsv3_prefill": "dsv3_idx"}[cfg])
+        loads_np, _ = oracle.count_loads(_np(idx), c.E)
+    gl, st = _quality_bufs(loads_np.shape[0], c.gpus)
+    word = _status()
+    plan = eplb.rebalance(torch.from_numpy(loads_np).to(DEV), c.P, c.G, c.N, c.gpus, status=word,
+                          gpu_load=gl, stats=st)
+    torch.cuda.synchronize()
+    assert int(word.item()) == 0
+    ref = _plans_for(c, loads_np)
+    _assert_plan_equal(plan, ref)
+    ref_gl, ref_st = oracle.plan_stats(loads_np, ref[0], ref[2], c.gpus)
+    assert np.array_equal(_np(gl), ref_gl) and np.array_equal(_np(st), ref_st)
+    # either output alone
+    gl2, st2 = _quality_bufs(loads_np.shape[0], c.gpus)
+    eplb.rebalance(torch.from_numpy(loads_np).to(DEV), c.P, c.G, c.N, c.gpus, stats=st2)
+    eplb.rebalance(torch.from_numpy(loads_np).to(DEV), c.P, c.G, c.N, c.gpus, gpu_load=gl2)
+    assert np.array_equal(_np(gl2), ref_gl) and np.array_equal(_np(st2), ref_st)
+
+
+@pytest.mark.parametrize("shape", SHAPES[:12])
+def test_rebalance_fused_quality_shapes(shape):
+    E, G, P, N, gpus = shape
+    rng = np.random.default_rng(E * 7 + P)
+    loads_np = rng.integers(0, 1 << 30, (9, E)).astype(np.int64)
+    loads_np[3] = 0  # all-zero row: balancedness 1
+    gl, st = _quality_bufs(9, gpus)
+    plan = eplb.rebalance(torch.from_numpy(loads_np).to(DEV), P, G, N, gpus, gpu_load=gl, stats=st)
+    ref = oracle.rebalance(loads_np, P, G, N, gpus, slots=plan.log2phy.shape[2])
+    ref_gl, ref_st = oracle.plan_stats(loads_np, ref[0], ref[2], gpus)
+    assert np.array_equal(_np(gl), ref_gl) and np.array_equal(_np(st), ref_st)
+    assert _np(st)[3, 3] == 1.0
+
+
+def test_rebalance_fused_quality_worked_example():
+    # the per-GPU load range the page prints for layer 0 of its example
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "eplb_readme_example.json")) as f:
+        ex = json.load(f)
+    w = torch.from_numpy(np.array(ex["weight"], dtype=np.int64)).to(DEV)
+    for G, key in ((4, "layer0_gpu_load_hierarchical"), (3, "layer0_gpu_load_global_groups3")):
+        gl, st = _quality_bufs(2, 8)
+        eplb.rebalance(w, 16, G, 2, 8, gpu_load=gl, stats=st)
+        assert _np(st)[0, 0] == ex[key]["min"] and _np(st)[0, 1] == ex[key]["max"]
+
+
+def test_rebalance_fused_quality_error_rows_are_nan():
+    loads_np = np.full((3, 12), 5, dtype=np.int64)
+    loads_np[1, 4] = 1 << 41  # outside [0, 2^40): the row is rejected
+    gl, st = _quality_bufs(3, 8)
+    word = _status()
+    eplb.rebalance(torch.from_numpy(loads_np).to(DEV), 16, 4, 2, 8, status=word, gpu_load=gl,
+                   stats=st)
+    torch.cuda.synchronize()
+    assert int(word.item()) == oracle.ERR_RANGE
+    assert np.isnan(_np(gl)[1]).all() and np.isnan(_np(st)[1]).all()
+    ref = oracle.rebalance(loads_np[[0, 2]], 16, 4, 2, 8)
+    ref_gl, ref_st = oracle.plan_stats(loads_np[[0, 2]], ref[0], ref[2], 8)
+    assert np.array_equal(_np(gl)[[0, 2]], ref_gl) and np.array_equal(_np(st)[[0, 2]], ref_st)
+
+
+@pytest.mark.parametrize("single", [True, False])
+def test_serving_step_reports_the_next_plans_quality(dsv3_idx, single):
+    """The serving step (one launch or two) writes the quality of the plan it
+    builds: the oracle's plan_stats on the window sums and the oracle's plan."""
+    from moe_expert_load_eplb_b200.pipeline import EplbStep
+    c = W.DSV3_PREFILL
+    W_ = 4
+    hist = W.histogram_steps(W_ - 1, c.L, c.E, c.T * c.K, c.stream, device=DEV)
+    step = EplbStep(c.L, c.T, c.K, c.E, c.P, c.G, c.N, c.gpus, window=W_, device=DEV,
+                    single_launch=single)
+    step.fill_history(hist)
+    ring = np.concatenate([_np(hist), np.zeros((1, c.L, c.E), np.int64)], axis=0)
+
+    def check():
+        loads = oracle.window(ring, W_, W_ - 1)[0]
+        ref = oracle.rebalance(loads, c.P, c.G, c.N, c.gpus, slots=step.X)
+        ref_gl, ref_st = oracle.plan_stats(loads, ref[0], ref[2], c.gpus)
+        assert np.array_equal(_np(step.gpu_load), ref_gl)
+        assert np.array_equal(_np(step.stats), ref_st)
+
+    check()  # the plan fill_history built
+    for s_i, idx in enumerate([dsv3_idx, dsv3_idx.flip(1).contiguous()]):
+        step(idx)
+        torch.cuda.synchronize()
+        assert int(step.status.item()) == 0
+        ring[(W_ - 1 + s_i) % W_] = oracle.count_loads(_np(idx), c.E)[0]
+        check()
+
+
 @pytest.mark.parametrize("shape", [(58, 256, 288), (3, 12, 16), (1000, 64, 96), (2, 1, 1)])
 def test_fold_loads_matches_oracle(shape):
     R, E, P = shape

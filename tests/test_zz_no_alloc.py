@@ -18,7 +18,7 @@ def test_noalloc_rejects_too_many_layers_before_touching_anything():
     # null pointers everywhere: the layer limit is checked first
     rc = lib.eplb_serve_step_noalloc(None, 4097, 16, 4, 24, None, 17, None, 0, None, None, None,
                                      2, 0, -1, 40, 6, 2, 4, None, None, None, None, None, None,
-                                     None)
+                                     None, None, None)
     assert rc == 9  # EPLB_ERR_LIMIT
 
 
