@@ -744,7 +744,10 @@ __device__ void step3(const Step3Ops &o) {
     if (j < ppn) {
       const int m = n * lpn + p2m[n * ppn + j];
       const uint32_t c = static_cast<uint32_t>(cnt[m]);
-      const uint64_t scale = c == 1 ? lam[n] : lam[n] / c;
+      const uint64_t lm = lam[n];
+      // Lambda / c exactly; a 32-bit divide when Lambda fits (lcm(1..9) =
+      // 2520 on the DeepSeek-V3 shape), the 64-bit routine otherwise
+      const uint64_t scale = c == 1 ? lm : (lm >> 32 ? lm / c : static_cast<uint32_t>(lm) / c);
       key = ((K(static_cast<uint64_t>(wm[m])) * K(scale)) << kIdxBits) | (imask - K(j));
     }
     keys[n * npad + j] = key;
