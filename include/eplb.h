@@ -49,7 +49,9 @@ typedef enum eplb_status {
   EPLB_ERR_CUDA = 6,          /* a CUDA runtime call or launch failed */
   EPLB_ERR_TIMEOUT = 7,       /* reserved: an in-kernel wait gave up (no current kernel waits) */
   EPLB_ERR_ALIGN = 8,         /* a pointer lacks the alignment stated below */
-  EPLB_ERR_LIMIT = 9          /* a size beyond the limits stated in this header */
+  EPLB_ERR_LIMIT = 9,         /* a size beyond the limits stated in this header */
+  EPLB_ERR_INTERNAL = 10      /* checking build only: an internal index check failed (the
+                                 access it guards was skipped); never from a normal build */
 } eplb_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -60,6 +62,12 @@ const char *eplb_last_cuda_error(void);
 
 /* ABI version of this library: (major << 16) | minor. */
 int32_t eplb_abi_version(void);
+
+/* 1 if this library is the checking build (internal index checks compiled
+ * in, built with `python -m moe_expert_load_eplb_b200.build --checks` as
+ * libeplb_checks.so), else 0.  The checking build has the same ABI and
+ * results; it is slower and meant for tests. */
+int32_t eplb_checking_build(void);
 
 /*
  * S1 -- load counting.  [EPLB] "От переводчика: термины": the load of an

@@ -31,12 +31,16 @@ __all__ = [
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_PKG, "libeplb.so")
+# EPLB_LIBRARY=checks selects the checking build (internal index checks that
+# report EPLB_ERR_INTERNAL; same ABI and results), built with
+# `python -m moe_expert_load_eplb_b200.build --checks`
+_LIB_PATH = os.path.join(_PKG, "libeplb_checks.so" if os.environ.get("EPLB_LIBRARY") == "checks"
+                         else "libeplb.so")
 
 STATUS = {
     0: "EPLB_OK", 1: "EPLB_ERR_NULL", 2: "EPLB_ERR_SHAPE", 3: "EPLB_ERR_DIVISIBILITY",
     4: "EPLB_ERR_RANGE", 5: "EPLB_ERR_SLOTS", 6: "EPLB_ERR_CUDA", 7: "EPLB_ERR_TIMEOUT",
-    8: "EPLB_ERR_ALIGN", 9: "EPLB_ERR_LIMIT",
+    8: "EPLB_ERR_ALIGN", 9: "EPLB_ERR_LIMIT", 10: "EPLB_ERR_INTERNAL",
 }
 
 
@@ -70,13 +74,15 @@ def load_library():
         return _lib
     if not os.path.exists(_LIB_PATH):
         raise ImportError(f"{_LIB_PATH} is missing: build it with "
-                          "`python -m moe_expert_load_eplb_b200.build` (nvcc, sm_100a)")
+                          "`python -m moe_expert_load_eplb_b200.build` (nvcc, sm_100a; "
+                          "--checks for the checking build)")
     lib = ctypes.CDLL(_LIB_PATH)
     p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32
     sig = {
         "eplb_status_string": ([i32], ctypes.c_char_p),
         "eplb_last_cuda_error": ([], ctypes.c_char_p),
         "eplb_abi_version": ([], i32),
+        "eplb_checking_build": ([], i32),
         "eplb_count_loads": ([p, i64, i64, i32, i32, p, i32, p, p], i32),
         "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, p], i32),
         "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p], i32),

@@ -116,6 +116,7 @@ const char *eplb_status_string(int32_t status) {
     case EPLB_ERR_TIMEOUT: return "EPLB_ERR_TIMEOUT";
     case EPLB_ERR_ALIGN: return "EPLB_ERR_ALIGN";
     case EPLB_ERR_LIMIT: return "EPLB_ERR_LIMIT";
+    case EPLB_ERR_INTERNAL: return "EPLB_ERR_INTERNAL";
     default: return "EPLB_ERR_UNKNOWN";
   }
 }
@@ -123,6 +124,14 @@ const char *eplb_status_string(int32_t status) {
 const char *eplb_last_cuda_error(void) { return g_last_error; }
 
 int32_t eplb_abi_version(void) { return (2 << 16) | 0; }
+
+int32_t eplb_checking_build(void) {
+#ifdef EPLB_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K, int32_t E,
                              int64_t *counts, int32_t accumulate, unsigned long long *bad,

@@ -17,6 +17,21 @@ __device__ __forceinline__ void report(int32_t *status, int32_t code) {
   if (status != nullptr) atomicCAS(status, 0, code);
 }
 
+// Checking build (-DEPLB_CHECKS): EPLB_IN(cond, status) states an index
+// bound the kernel relies on (a shared-memory row or slot, an output
+// position derived from data); when it does not hold, the access it guards
+// is skipped and EPLB_ERR_INTERNAL goes to the call's status word.  In the
+// normal build it is the constant true and the guard compiles away.
+#ifdef EPLB_CHECKS
+__device__ __forceinline__ bool check_in(bool cond, int32_t *status) {
+  if (!cond) report(status, EPLB_ERR_INTERNAL);
+  return cond;
+}
+#define EPLB_IN(cond, status) (::eplb::check_in((cond), (status)))
+#else
+#define EPLB_IN(cond, status) true
+#endif
+
 // Shared-memory access by 32-bit shared-window address: one multiply-add
 // per address, no generic-pointer arithmetic.
 __device__ __forceinline__ void red_shared_inc(uint32_t addr) {

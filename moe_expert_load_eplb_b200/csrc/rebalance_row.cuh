@@ -723,6 +723,7 @@ struct Step3Ops {
   const int32_t *cnt, *p2m;
   int32_t *pc, *ipack, *irank;
   int N, npad, lpn, ppn, mpn, ppg;
+  int32_t *status;  // the checking build's reports
 };
 
 template <typename K, bool kCap2>
@@ -741,7 +742,7 @@ __device__ void step3(const Step3Ops &o) {
     const int n = t / per;
     const int j = t - n * per;
     K key = 0;
-    if (j < ppn) {
+    if (j < ppn && EPLB_IN(p2m[n * ppn + j] >= 0 && p2m[n * ppn + j] < lpn, o.status)) {
       const int m = n * lpn + p2m[n * ppn + j];
       const uint32_t c = static_cast<uint32_t>(cnt[m]);
       const uint64_t lm = lam[n];
@@ -773,9 +774,9 @@ __device__ void step3_wide(unsigned char *keys, unsigned char *sorted, unsigned 
                                         const int64_t *wm, const uint64_t *lam, const int32_t *cnt,
                                         const int32_t *p2m, int32_t *pc, int32_t *ipack,
                                         int32_t *irank, int N, int npad, int lpn, int ppn, int mpn,
-                                        int ppg) {
+                                        int ppg, int32_t *status) {
   step3<u128, kCap2>(Step3Ops{keys, sorted, pw, wm, lam, cnt, p2m, pc, ipack, irank, N, npad, lpn,
-                              ppn, mpn, ppg});
+                              ppn, mpn, ppg, status});
 }
 
 // One row of rebalance_experts, by the whole CTA, in `smem` (Layout(a.s).total
@@ -886,6 +887,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   for (int e = tid; e < s.E; e += nthr()) {
     const int g = e / s.gs;
     const int m = (gpack[g] * s.gpn + grank[g]) * s.gs + (e - g * s.gs);
+    if (!EPLB_IN(m >= 0 && m < s.E, a.status)) continue;
     mlog2log[m] = e;
     wm[m] = w[e];
     cnt[m] = 1;
@@ -924,7 +926,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     __syncthreads();
     for (int t = tid; t < s.N * nc; t += nthr()) {
       const int n = t / nc;
-      cnt[n * s.lpn + cand_i[t]] = cand_c[t];
+      if (EPLB_IN(cand_i[t] >= 0 && cand_i[t] < s.lpn, a.status)) cnt[n * s.lpn + cand_i[t]] = cand_c[t];
     }
   } else if (nc > 32) {
     for (int n = tid >> 5; n < s.N; n += nwarps()) replicate_smem(s.lpn, s.ppn, n, wm, cnt, p2m, rrank);
@@ -991,11 +993,11 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   } else if (flags[0] == 0) {
     step3<uint64_t, kCap2>(Step3Ops{smem + lay.keys, smem + lay.sorted, smem + lay.pw, wm, lam, cnt,
                                     p2m, reinterpret_cast<int32_t *>(smem + lay.pc), ipack, irank,
-                                    s.N, s.npad, s.lpn, s.ppn, s.mpn, s.ppg});
+                                    s.N, s.npad, s.lpn, s.ppn, s.mpn, s.ppg, a.status});
   } else {
     step3_wide<kCap2>(smem + lay.keys, smem + lay.sorted, smem + lay.pw, wm, lam, cnt, p2m,
                       reinterpret_cast<int32_t *>(smem + lay.pc), ipack, irank, s.N, s.npad, s.lpn,
-                      s.ppn, s.mpn, s.ppg);
+                      s.ppn, s.mpn, s.ppg, a.status);
   }
   __syncthreads();
 
@@ -1018,6 +1020,10 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     const int m = n * s.lpn + p2m[t];
     const int e = mlog2log[m];
     const int k = rrank[t];
+    if (!EPLB_IN(pphy >= n * s.ppn && pphy < (n + 1) * s.ppn && e >= 0 && e < s.E && k >= 0 &&
+                     m >= n * s.lpn && m < (n + 1) * s.lpn,
+                 a.status))
+      continue;
     if (quality)
       qslot[pphy] = __ddiv_rn(static_cast<double>(w[e]), static_cast<double>(cnt[m]));
     a.phy2log[row * s.P + pphy] = e;
@@ -1054,6 +1060,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   } else {
     for (int t = tid; t < s.P; t += nthr()) {
       const int k = outr[t];
+      if (!EPLB_IN(outp[t] >= 0 && outp[t] < s.E && k >= 0, a.status)) continue;
       if (k < s.X)
         gl[outp[t] * s.X + k] = t;
       else

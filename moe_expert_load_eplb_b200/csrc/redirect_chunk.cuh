@@ -314,9 +314,13 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
     const uint32_t c = static_cast<uint32_t>(d >> 37) & 0xffffu;
     if (c == 0) return -1;
     const uint32_t r = mod_magic(ctx.y, c, static_cast<uint32_t>(d >> 5));
+    if (!EPLB_IN(r < c && c <= static_cast<uint32_t>(a.X) && ee < E, a.status)) return -1;
     return __ldg(l2p_layer + ee * static_cast<uint32_t>(a.X) + r);
   };
-  auto ctx_fast = [&](uint32_t tok) -> uint32_t { return tab_addr + 2u * mod_magic(tok, M, a.m_magic); };
+  auto ctx_fast = [&](uint32_t tok) -> uint32_t {
+    const uint32_t r = mod_magic(tok, M, a.m_magic);
+    return tab_addr + 2u * (EPLB_IN(r < M, a.status) ? r : 0u);
+  };
   auto ctx_desc = [&](uint32_t tok) -> uint2 { return make_uint2(selector(tok), tok); };
 
   auto stream = [&](auto ctx_of, auto map1) {
