@@ -605,8 +605,8 @@ def run_ours(args, rank: int, world: int, group):
     fstages = _stage_report(f_stage, False, fresh.X, world, hbm_peak)
     out["fresh_order"] = {"steps": Kf, "ms_per_step": round(f_total / Kf, 5),
                           "value": round(c.L * Kf / (f_total / 1e3), 1), "stages": fstages}
-    out["load_count_gbs"] = fstages["count"]["gbs"]
-    out["load_count_frac_hbm"] = fstages["count"]["frac_hbm"]
+    out["load_count_c2"] = {"gbs": fstages["count"]["gbs"], "frac_hbm": fstages["count"]["frac_hbm"],
+                            "stage": "fresh-order count stage on the 121.6 MB batch"}
     del fresh
     return _finish(out, args, step, idx, hist, flush, group, dev, rank, world)
 
@@ -616,6 +616,16 @@ def _finish(out, args, step, idx, hist, flush, group, dev, rank, world):
     K = args.steps
     if world == 1 and args.legs:
         out.update(run_legs(args, dev, args.legs))
+    # load-count GB/s: on the 1.95 GB stream (the workload the HBM target is
+    # set on) when that leg ran, else on the timed batch
+    if "hbm_stream" in out:
+        out["load_count_gbs"] = out["hbm_stream"]["count"]["gbs"]
+        out["load_count_frac_hbm"] = out["hbm_stream"]["count"]["frac_hbm"]
+        out["load_count_workload"] = "hbm_stream"
+    elif "load_count_c2" in out:
+        out["load_count_gbs"] = out["load_count_c2"]["gbs"]
+        out["load_count_frac_hbm"] = out["load_count_c2"]["frac_hbm"]
+        out["load_count_workload"] = "dsv3_prefill"
 
     def check(st, where):
         torch.cuda.synchronize()

@@ -97,14 +97,18 @@ eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K
  *
  * steps    device int64 [S, L, E].
  * snaps    device int64 [S - s_first, L, E]; must not overlap steps.
- * W >= 1 (W >= S gives running totals); 0 <= s_first < S.
+ * zero_row -1, or a row of steps to clear after it has been read (with a
+ *          ring of per-step counts: the slot the next step counts into, so
+ *          that eplb_count_loads can add to it with accumulate = 1 and no
+ *          separate clearing launch).
+ * W >= 1 (W >= S gives running totals); 0 <= s_first < S; -1 <= zero_row < S.
  * Sums are exact; wrap-around of int64 is the caller's concern.  No
  * data-dependent error exists, so the call takes no status word.
  * With a ring buffer of the last W per-step counts, s_first = S - 1 = W - 1
  * returns the current window sum (row order does not change a full sum).
  */
-eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, int32_t E,
-                                   int64_t W, int64_t s_first, int64_t *snaps,
+eplb_status eplb_window_accumulate(int64_t *steps, int64_t S, int64_t L, int32_t E,
+                                   int64_t W, int64_t s_first, int64_t *snaps, int64_t zero_row,
                                    cudaStream_t stream);
 
 /*

@@ -84,7 +84,7 @@ def load_library():
         "eplb_abi_version": ([], i32),
         "eplb_checking_build": ([], i32),
         "eplb_count_loads": ([p, i64, i64, i32, i32, p, i32, p, p], i32),
-        "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, p], i32),
+        "eplb_window_accumulate": ([p, i64, i64, i32, i64, i64, p, i64, p], i32),
         "eplb_rebalance": ([p, i64, i32, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p], i32),
         "eplb_redirect": ([p, i64, i64, i32, i32, p, i32, p, i64, p, p, p, p], i32),
         "eplb_count_redirect": ([p, i64, i64, i32, i32, p, i32, p, i32, p, i64, p, p, p, p], i32),
@@ -241,8 +241,9 @@ def count_loads(idx: torch.Tensor, num_experts: int, counts: Optional[torch.Tens
 
 
 def window_accumulate(steps: torch.Tensor, window: int, s_first: int = 0,
-                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """S2: out[s - s_first] = sum of steps[max(0, s-window+1) .. s] (int64 [S, L, E])."""
+                      out: Optional[torch.Tensor] = None, zero_row: int = -1) -> torch.Tensor:
+    """S2: out[s - s_first] = sum of steps[max(0, s-window+1) .. s] (int64 [S, L, E]);
+    zero_row >= 0 clears that row of ``steps`` after it has been read."""
     _cuda(steps, torch.int64, "steps")
     if steps.dim() != 3:
         raise ValueError("steps must be [S, L, E]")
@@ -254,7 +255,7 @@ def window_accumulate(steps: torch.Tensor, window: int, s_first: int = 0,
         raise ValueError("out must be [S - s_first, L, E]")
     with _on_device(steps.device):
         _check(load_library().eplb_window_accumulate(
-            _ptr(steps), S, L, E, window, s_first, _ptr(out), _stream(steps.device)),
+            _ptr(steps), S, L, E, window, s_first, _ptr(out), int(zero_row), _stream(steps.device)),
             "eplb_window_accumulate")
     return out
 

@@ -151,16 +151,17 @@ eplb_status eplb_count_loads(const int32_t *idx, int64_t L, int64_t T, int32_t K
   return launch_count_loads(idx, L, T * K, E, counts, bad, stream);
 }
 
-eplb_status eplb_window_accumulate(const int64_t *steps, int64_t S, int64_t L, int32_t E,
-                                   int64_t W, int64_t s_first, int64_t *snaps,
+eplb_status eplb_window_accumulate(int64_t *steps, int64_t S, int64_t L, int32_t E,
+                                   int64_t W, int64_t s_first, int64_t *snaps, int64_t zero_row,
                                    cudaStream_t stream) {
   if (S < 0 || L < 0 || E < 1 || W < 1 || s_first < 0) return EPLB_ERR_SHAPE;
+  if (zero_row < -1 || (zero_row >= S && S > 0)) return EPLB_ERR_SHAPE;
   if (S == 0 || L == 0) return s_first == 0 ? EPLB_OK : EPLB_ERR_SHAPE;
   if (s_first >= S) return EPLB_ERR_SHAPE;
   if (steps == nullptr || snaps == nullptr) return EPLB_ERR_NULL;
   const int64_t C = L * E;
   if (C > (int64_t(1) << 34)) return EPLB_ERR_LIMIT;
-  return launch_window(steps, S, C, W, s_first, snaps, stream);
+  return launch_window(steps, S, C, W, s_first, snaps, zero_row, stream);
 }
 
 static eplb_status rebalance_shape(int64_t R, int32_t E, int32_t P, int32_t G, int32_t N,

@@ -52,8 +52,8 @@ eplb_status cuda_fail(cudaError_t err);
 eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer, int32_t E,
                                int64_t *counts, unsigned long long *bad, cudaStream_t stream);
 
-eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
-                          int64_t *snaps, cudaStream_t stream);
+eplb_status launch_window(int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
+                          int64_t *snaps, int64_t zero_row, cudaStream_t stream);
 
 struct RebalanceShape {
   int32_t E, P, G, N, gpus, X;   // G, N after the policy choice

@@ -57,8 +57,8 @@ struct WinBlock {
 
 template <int kU, bool kSub>
 __global__ void __launch_bounds__(kCols * kMaxRg) window_kernel(
-    const int64_t *__restrict__ steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
-    int64_t *__restrict__ snaps) {
+    int64_t *__restrict__ steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
+    int64_t *__restrict__ snaps, int64_t zero_row) {
   __shared__ int64_t part[kMaxRg][kCols];
   pdl_trigger();
   pdl_wait();
@@ -101,12 +101,15 @@ __global__ void __launch_bounds__(kCols * kMaxRg) window_kernel(
     __syncthreads();
     cur = nxt;
   }
+  // every row of this strip's columns has been read (the last block's loads
+  // were consumed above): clear the requested row of them
+  if (zero_row >= 0 && g == 0 && col_ok) steps[zero_row * C + c] = 0;
 }
 
 }  // namespace
 
-eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
-                          int64_t *snaps, cudaStream_t stream) {
+eplb_status launch_window(int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
+                          int64_t *snaps, int64_t zero_row, cudaStream_t stream) {
   DeviceInfo di;
   const eplb_status dst = device_info(&di);
   if (dst != EPLB_OK) return dst;
@@ -130,7 +133,7 @@ eplb_status launch_window(const int64_t *steps, int64_t S, int64_t C, int64_t W,
       break;
     }
   }
-  void *args[] = {&steps, &S, &C, &W, &s_first, &snaps};
+  void *args[] = {&steps, &S, &C, &W, &s_first, &snaps, &zero_row};
   const cudaError_t err = launch_pdl(fn, dim3(static_cast<unsigned>(strips)), dim3(kCols, rg), 0,
                                      stream, args);
   return err == cudaSuccess ? EPLB_OK : cuda_fail(err);

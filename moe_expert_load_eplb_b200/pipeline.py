@@ -171,7 +171,9 @@ class EplbStep:
             count_redirect(idx, self.E, used.log2phy, used.logcnt, self.token_offset, counts=row,
                            accumulate=True, out=self.out, bad=self.bad, status=self.status)
         else:
-            count_loads(idx, self.E, counts=row, bad=self.bad)
+            # the ring row was cleared by the previous step's window launch
+            # (fill_history clears it for the first step)
+            count_loads(idx, self.E, counts=row, accumulate=True, bad=self.bad)
         rec(1)
         if self.group is not None:
             allreduce_loads(row, self.group)
@@ -184,7 +186,8 @@ class EplbStep:
                              loads_out=self.loads, status=self.status, gpu_load=self.gpu_load,
                              stats=self.stats)
         else:
-            window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads)
+            window_accumulate(self.ring, self.W, s_first=self.W - 1, out=self.loads,
+                              zero_row=(self.steps_done + 1) % self.W)
             rec(3)
             nxt = used
             rebalance(self.loads[0], self.P, self.G, self.N, self.gpus, slots=self.X, out=nxt,

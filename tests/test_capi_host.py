@@ -64,9 +64,11 @@ def test_host_argument_checks(lib):
     assert lib.eplb_count_loads(p(20), 1, 4, 2, 8, one, 1, None, None) == 8
     assert lib.eplb_count_loads(one, 0, 4, 2, 8, None, 0, None, None) == 0  # nothing to do
     # window
-    assert lib.eplb_window_accumulate(one, 4, 2, 3, 0, 0, one, None) == 2
-    assert lib.eplb_window_accumulate(one, 4, 2, 3, 2, 4, one, None) == 2
-    assert lib.eplb_window_accumulate(None, 4, 2, 3, 2, 0, one, None) == 1
+    assert lib.eplb_window_accumulate(one, 4, 2, 3, 0, 0, one, -1, None) == 2
+    assert lib.eplb_window_accumulate(one, 4, 2, 3, 2, 4, one, -1, None) == 2
+    assert lib.eplb_window_accumulate(one, 4, 2, 3, 2, 0, one, 4, None) == 2   # zero_row >= S
+    assert lib.eplb_window_accumulate(one, 4, 2, 3, 2, 0, one, -2, None) == 2
+    assert lib.eplb_window_accumulate(None, 4, 2, 3, 2, 0, one, -1, None) == 1
     # rebalance: divisibility, shape, limits; R == 0 needs no device
     rb = lib.eplb_rebalance
     assert rb(one, 1, 12, 16, 5, 2, 8, 5, one, one, one, one, None, None, None, None) == 3   # 12 % 5

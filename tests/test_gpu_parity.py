@@ -160,6 +160,21 @@ def test_window_shapes(S, L, E, window, s_first):
     assert np.array_equal(_np(snaps), ref)
 
 
+@pytest.mark.parametrize("S,W_,zero_row", [(16, 16, 3), (16, 16, 15), (1, 1, 0), (1000, 1000, 999),
+                                            (300, 40, 0), (7, 2, 6)])
+def test_window_zero_row(S, W_, zero_row):
+    """The window sum is taken before the row is cleared; only that row changes."""
+    g = torch.Generator(device=DEV).manual_seed(S + zero_row)
+    L, E = 3, 77
+    steps = torch.randint(0, 1 << 30, (S, L, E), generator=g, device=DEV, dtype=torch.int64)
+    before = _np(steps).copy()
+    snaps = eplb.window_accumulate(steps, W_, s_first=S - 1, zero_row=zero_row)
+    assert np.array_equal(_np(snaps), oracle.window(before, W_, S - 1))
+    after = before.copy()
+    after[zero_row] = 0
+    assert np.array_equal(_np(steps), after)
+
+
 # -------------------------------------------------------------- rebalance --
 
 def test_rebalance_readme_example():
