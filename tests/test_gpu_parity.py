@@ -515,8 +515,10 @@ def test_pipeline_serving_order_dsv3_prefill(dsv3_idx, single):
 @pytest.mark.parametrize("single", [True, False])
 @pytest.mark.parametrize("steps_done", [2, 7, 13])
 def test_pipeline_history_with_a_step_count(tiny_idx, single, steps_done):
-    """A step primed with history at any step count keeps the last W - 1
-    steps in its window: the oracle, given the same per-step counts in step
+    """A step primed with history at any step count keeps the right steps in
+    its window: the plan fill_history builds covers the history rows kept
+    (at most W - 1), and the plan each step builds covers the last W steps,
+    that step included.  The oracle, given the same per-step counts in step
     order, sums the same window before and after each new step."""
     from moe_expert_load_eplb_b200.pipeline import EplbStep
     c = W.TINY
@@ -528,7 +530,7 @@ def test_pipeline_history_with_a_step_count(tiny_idx, single, steps_done):
     steps = [_np(hist[0]), _np(hist[1])]  # per-step counts in step order
 
     def ref_plan():
-        win = np.stack(steps[-(W_ - 1):] + [np.zeros((c.L, c.E), np.int64)], axis=0)
+        win = np.stack(steps[-W_:], axis=0)
         return _oracle_plan_from_ring(win, c, step.X)
 
     plan_ref = ref_plan()
