@@ -65,6 +65,7 @@ def _rebalance_both(loads_np, P, G, N, gpus, slots=None):
 def _assert_plan_equal(plan, ref):
     for name, got, want in zip(("phy2log", "phyrank", "logcnt", "log2phy"), plan, ref):
         g = _np(got)
+        assert g.shape == want.shape, f"{name}: shape {g.shape}, oracle {want.shape}"
         if not np.array_equal(g, want):
             bad = np.argwhere(g != want)
             raise AssertionError(f"{name} differs at {len(bad)} places, first {bad[:5].tolist()}")
@@ -905,7 +906,7 @@ def test_rebalance_fused_quality_matches_oracle(cfg, request):
                           gpu_load=gl, stats=st)
     torch.cuda.synchronize()
     assert int(word.item()) == 0
-    ref = _plans_for(c, loads_np)
+    ref = oracle.rebalance(loads_np, c.P, c.G, c.N, c.gpus, slots=plan.log2phy.shape[2])
     _assert_plan_equal(plan, ref)
     ref_gl, ref_st = oracle.plan_stats(loads_np, ref[0], ref[2], c.gpus)
     assert np.array_equal(_np(gl), ref_gl) and np.array_equal(_np(st), ref_st)
