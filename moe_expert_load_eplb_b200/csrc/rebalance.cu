@@ -1,7 +1,8 @@
 // rebalance.cu -- S3/S4 (and, in ring mode, S2): rebalance_experts over R
 // rows, one CTA per row.  The row's work is rebalance_row (rebalance_row.cuh),
 // shared with the serving-step kernel.
-#define EPLB_RB_COLD __noinline__  // cold paths out of line (rebalance_row.cuh)
+#define EPLB_RB_COLD __noinline__    // cold paths out of line (rebalance_row.cuh)
+#define EPLB_RB_SHARED __noinline__  // one copy of the shared building blocks
 #include "rebalance_row.cuh"
 
 namespace eplb {

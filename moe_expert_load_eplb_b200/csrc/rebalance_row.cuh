@@ -56,6 +56,14 @@
 #ifndef EPLB_RB_COLD
 #define EPLB_RB_COLD
 #endif
+// The building blocks several steps use (the rank sort, the packing greedy)
+// carry EPLB_RB_SHARED: one out-of-line copy serves every call site in the
+// rebalance kernel, so the instruction cache holds it after its first use
+// (separate inlined copies are each fetched cold; sharing them made the
+// 58-row DeepSeek-V3 rebalance 2 us faster, measured).
+#ifndef EPLB_RB_SHARED
+#define EPLB_RB_SHARED
+#endif
 
 namespace eplb {
 namespace {
@@ -281,6 +289,13 @@ __device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit em
     rank_pass<4, K>(key, stride, nseg, n, tps, emit);
 }
 
+// Descending ranks written out: out[g * stride + rank] = key (the stable
+// (value desc, index asc) order of the composite keys).
+template <typename K>
+__device__ EPLB_RB_SHARED void rank_sort(const K *key, int stride, int nseg, int n, K *out) {
+  rank_segments<K>(key, stride, nseg, n, [&](int g, int, int r, K k) { out[g * stride + r] = k; });
+}
+
 // CTA-wide bitonic sort, descending, of nseg segments of npad (power of two)
 // keys each, in place; padding keys must be 0.
 template <typename K>
@@ -470,7 +485,7 @@ __device__ EPLB_RB_COLD void pack_segments_wide(const K *skey, int stride, int n
                                                 int32_t *irank, int out_stride);
 
 template <typename K, bool kCap2>
-__device__ void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
+__device__ EPLB_RB_SHARED void pack_segments(const K *skey, int stride, int nseg, int n, int m, int cap, K *pw,
                               int32_t *pc, int32_t *ipack, int32_t *irank, int out_stride) {
   if (n <= 0) return;
   if constexpr (kCap2) {
@@ -677,21 +692,31 @@ __device__ void write_error_row(const RbArgs &a, int64_t row) {
     for (int k = threadIdx.x; k < 4; k += nthr()) a.stats[row * 4 + k] = nan;
 }
 
-// Plan quality of the row just assembled, by one warp (page "DualPipe и
-// EPLB", Part 2, box "От переводчика: что на рисунке": per-GPU loads of the
-// worked example; exercise 2 of "что сделать руками": max against mean).
-// q[p] = w / logcnt of slot p's expert (fp64, rounded to nearest); GPU g's
-// load is the sum of its slots' q in slot order from 0.0, then min, max and
-// the mean of the GPU loads summed in GPU order, and balancedness = mean /
-// max (1 when max is 0).  Every operation is an explicitly rounded fp64 add
-// or divide in that fixed order, so the figures are bit-identical to the
-// same sums done sequentially on a CPU.
+// Plan quality of the row just assembled, by one warp while the others copy
+// log2phy out (page "DualPipe и EPLB", Part 2, box "От переводчика: что на
+// рисунке": per-GPU loads of the worked example; exercise 2 of "что сделать
+// руками": max against mean).  q[p] = w / logcnt of slot p's expert (fp64,
+// rounded to nearest); GPU g's load is the sum of its slots' q in slot order
+// from 0.0, then min, max and the mean of the GPU loads summed in GPU order,
+// and balancedness = mean / max (1 when max is 0).  Every operation is an
+// explicitly rounded fp64 add or divide in that fixed order, so the figures
+// are bit-identical to the same sums done sequentially on a CPU.
 // Operands are plain values: an out-of-line call given the kernel's
 // parameter block by reference needs a stack copy of it (it doubled the
-// kernel's registers).
+// kernel's registers).  p2l: slot -> expert; w, lc: load and replicas by
+// expert; q: P doubles and gl: gpus doubles of scratch.
 __device__ EPLB_RB_COLD void plan_quality(double *gpu_load, double *stats, int64_t row, int gpus,
-                                          int ppg, const double *q, double *gl) {
+                                          int ppg, int P, int E, const int32_t *p2l,
+                                          const int64_t *w, const int32_t *lc, double *q,
+                                          double *gl) {
   const int lane = threadIdx.x & 31;
+#pragma unroll 4
+  for (int p = lane; p < P; p += 32) {
+    const int e = p2l[p];
+    q[p] = e >= 0 && e < E ? __ddiv_rn(static_cast<double>(w[e]), static_cast<double>(lc[e]))
+                           : __longlong_as_double(0x7ff8000000000000LL);
+  }
+  __syncwarp();
   for (int g = lane; g < gpus; g += 32) {
     double acc = 0.0;
     for (int k = 0; k < ppg; ++k) acc = __dadd_rn(acc, q[g * ppg + k]);
@@ -756,8 +781,7 @@ __device__ void step3(const Step3Ops &o) {
   __syncthreads();
   const K *skeys = keys;
   if (ranked) {
-    rank_segments<K>(keys, npad, N, ppn,
-                     [&](int g, int, int r, K k) { sorted[g * npad + r] = k; });
+    rank_sort<K>(keys, npad, N, ppn, sorted);
     skeys = sorted;
     __syncthreads();
   } else {
@@ -869,8 +893,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     __syncthreads();
     const uint64_t *gs_keys = gsorted;
     if (s.gpad <= kRankSortMax) {
-      rank_segments<uint64_t>(gkey, s.gpad, 1, s.G,
-                              [&](int, int, int r, uint64_t k) { gsorted[r] = k; });
+      rank_sort<uint64_t>(gkey, s.gpad, 1, s.G, gsorted);
     } else {
       for (int g = s.G + tid; g < s.gpad; g += nthr()) gkey[g] = 0;
       __syncthreads();
@@ -908,12 +931,15 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       ckey[m] = (static_cast<uint64_t>(wm[m]) << kIdxBits) | (kIdxMask - (m - n * s.lpn));
     }
     __syncthreads();
-    rank_segments<uint64_t>(ckey, s.lpn, s.N, s.lpn, [&](int g, int j, int r, uint64_t) {
-      if (r < nc) {
-        cand_w[g * nc + r] = wm[g * s.lpn + j];
-        cand_i[g * nc + r] = j;
-      }
-    });
+    uint64_t *csorted = reinterpret_cast<uint64_t *>(smem + lay.sorted);
+    rank_sort<uint64_t>(ckey, s.lpn, s.N, s.lpn, csorted);
+    __syncthreads();
+    for (int t = tid; t < s.N * nc; t += nthr()) {  // the nc heaviest of each node
+      const int g = t / nc;
+      const int j = static_cast<int>(kIdxMask - (csorted[g * s.lpn + (t - g * nc)] & kIdxMask));
+      cand_w[t] = wm[g * s.lpn + j];
+      cand_i[t] = j;
+    }
     __syncthreads();
     if (nc * (s.ppn - s.lpn) <= 256) {
       for (int t = tid; t < s.N * nc; t += nthr()) cand_c[t] = 1;
@@ -1009,10 +1035,9 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
   const bool in_smem = table_in_smem(s);
   int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
-  // plan quality: slot quotients w / logcnt, in the sort keys' space (free
-  // after step 3)
+  // plan quality: the slot -> expert map is kept in outp (unused by the
+  // shared-table path) for the quality warp
   const bool quality = a.gpu_load != nullptr || a.stats != nullptr;
-  double *qslot = reinterpret_cast<double *>(smem + lay.keys);
   bool slots = false;
   for (int t = tid; t < s.P; t += nthr()) {
     const int n = t / s.ppn;
@@ -1024,8 +1049,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
                      m >= n * s.lpn && m < (n + 1) * s.lpn,
                  a.status))
       continue;
-    if (quality)
-      qslot[pphy] = __ddiv_rn(static_cast<double>(w[e]), static_cast<double>(cnt[m]));
+    if (quality) outp[pphy] = e;
     a.phy2log[row * s.P + pphy] = e;
     a.phyrank[row * s.P + pphy] = k;
     if (in_smem) {
@@ -1044,18 +1068,24 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     a.logcnt[row * s.E + e] = cnt[m];
   }
   __syncthreads();
-  // warp 0 sums the plan quality (pack weights' space, free after step 3)
-  // while the other warps start copying the table out
+  // warp 0 computes the plan quality (scratch in the sort keys' and pack
+  // weights' space, free after step 3) while the other warps copy the
+  // table out
   if (quality && tid < 32)
-    plan_quality(a.gpu_load, a.stats, row, s.gpus, s.ppg, qslot,
+    plan_quality(a.gpu_load, a.stats, row, s.gpus, s.ppg, s.P, s.E, outp, w, lc,
+                 reinterpret_cast<double *>(smem + lay.keys),
                  reinterpret_cast<double *>(smem + lay.pw));
   if (in_smem) {
-    if (a.table_vec4) {
-      const int4 *src = reinterpret_cast<const int4 *>(tbl);
-      int4 *dst = reinterpret_cast<int4 *>(gl);
-      for (int i = tid; i < (EX >> 2); i += nthr()) dst[i] = src[i];
-    } else {
-      for (int i = tid; i < EX; i += nthr()) gl[i] = tbl[i];
+    const int t0 = quality ? 32 : 0;
+    if (tid >= t0) {
+      const int nt = nthr() - t0;
+      if (a.table_vec4) {
+        const int4 *src = reinterpret_cast<const int4 *>(tbl);
+        int4 *dst = reinterpret_cast<int4 *>(gl);
+        for (int i = tid - t0; i < (EX >> 2); i += nt) dst[i] = src[i];
+      } else {
+        for (int i = tid - t0; i < EX; i += nt) gl[i] = tbl[i];
+      }
     }
   } else {
     for (int t = tid; t < s.P; t += nthr()) {
