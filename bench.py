@@ -392,7 +392,9 @@ def leg_window_sweep(n, dev, flush, hbm_peak):
     res = {"workload": c.name, "steps": c.S, "layers": c.L, "experts": c.E, "window": c.W,
            "calls": n, "l2": "flushed before every call (512 MB write)"}
     m = _time_calls(lambda: eplb.window_accumulate(steps, c.W, out=snaps), n, dev, flush)
-    res["window"] = _hbm_entry(16.0 * elems, *m, hbm_peak)
+    res["window"] = _hbm_entry(16.0 * elems, *m, hbm_peak,
+                               {"kernel": "window_kernel",
+                                "traffic": _traffic("window.cu", "window_window_sweep.md", 1.0)})
     med, mean, clocks = _time_calls(
         lambda: eplb.rebalance(loads, c.P, c.G, c.N, c.gpus, out=plan, status=st), n, dev, flush)
     res["rebalance"] = {"rows": loads.shape[0], "ms": round(med, 4), "ms_mean": round(mean, 4),

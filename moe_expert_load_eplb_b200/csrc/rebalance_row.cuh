@@ -697,18 +697,18 @@ __device__ void write_error_row(const RbArgs &a, int64_t row) {
 // рисунке": per-GPU loads of the worked example; exercise 2 of "что сделать
 // руками": max against mean).  q[p] = w / logcnt of slot p's expert (fp64,
 // rounded to nearest); GPU g's load is the sum of its slots' q in slot order
-// from 0.0, then min, max and the mean of the GPU loads summed in GPU order,
-// and balancedness = mean / max (1 when max is 0).  Every operation is an
-// explicitly rounded fp64 add or divide in that fixed order, so the figures
-// are bit-identical to the same sums done sequentially on a CPU.
-// Operands are plain values: an out-of-line call given the kernel's
-// parameter block by reference needs a stack copy of it (it doubled the
-// kernel's registers).  p2l: slot -> expert; w, lc: load and replicas by
-// expert; q: P doubles and gl: gpus doubles of scratch.
-__device__ EPLB_RB_COLD void plan_quality(double *gpu_load, double *stats, int64_t row, int gpus,
-                                          int ppg, int P, int E, const int32_t *p2l,
-                                          const int64_t *w, const int32_t *lc, double *q,
-                                          double *gl) {
+// from 0.0; min and max of the GPU loads (exact in any order: a warp
+// butterfly); their mean summed in GPU order from 0.0 divided by gpus; and
+// balancedness = mean / max (1 when max is 0).  Every add and divide is an
+// explicitly rounded fp64 operation in that fixed order, so the figures are
+// bit-identical to the same sums done sequentially on a CPU.  Inline: out of
+// line, and with a serial min / max loop, it cost 4 us of the 58-row step
+// (measured).  p2l: slot -> expert; w, lc: load and replicas by expert; q: P
+// doubles and gl: gpus doubles of scratch.
+__device__ __forceinline__ void plan_quality(double *gpu_load, double *stats, int64_t row,
+                                             int gpus, int ppg, int P, int E, const int32_t *p2l,
+                                             const int64_t *w, const int32_t *lc, double *q,
+                                             double *gl) {
   const int lane = threadIdx.x & 31;
 #pragma unroll 4
   for (int p = lane; p < P; p += 32) {
@@ -717,20 +717,34 @@ __device__ EPLB_RB_COLD void plan_quality(double *gpu_load, double *stats, int64
                            : __longlong_as_double(0x7ff8000000000000LL);
   }
   __syncwarp();
+  double mn = __longlong_as_double(0x7ff0000000000000LL), mx = 0.0;  // +inf, 0
   for (int g = lane; g < gpus; g += 32) {
     double acc = 0.0;
+#pragma unroll 4
     for (int k = 0; k < ppg; ++k) acc = __dadd_rn(acc, q[g * ppg + k]);
     gl[g] = acc;
     if (gpu_load) gpu_load[row * gpus + g] = acc;
+    mn = fmin(mn, acc);
+    mx = fmax(mx, acc);
+  }
+  if (stats == nullptr) return;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   }
   __syncwarp();
-  if (lane == 0 && stats) {
-    double mn = gl[0], mx = gl[0], sum = 0.0;
-    for (int g = 0; g < gpus; ++g) {
-      mn = fmin(mn, gl[g]);
-      mx = fmax(mx, gl[g]);
-      sum = __dadd_rn(sum, gl[g]);
+  if (lane == 0) {
+    double sum = 0.0;
+    int g = 0;
+    for (; g + 8 <= gpus; g += 8) {  // loads ahead of the ordered adds
+      double v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = gl[g + j];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) sum = __dadd_rn(sum, v[j]);
     }
+    for (; g < gpus; ++g) sum = __dadd_rn(sum, gl[g]);
     const double mean = __ddiv_rn(sum, static_cast<double>(gpus));
     stats[row * 4 + 0] = mn;
     stats[row * 4 + 1] = mx;

@@ -9,7 +9,8 @@
 // HBM-bound gather, streamed like the count kernel: each CTA owns one chunk
 // of one layer (a contiguous run of the flattened index array whose interior
 // is 16-byte aligned); every thread keeps U = 4 independent 16-byte
-// streaming loads in flight and writes 16-byte streaming stores.
+// streaming loads in flight, the next U vectors requested into L2 by
+// prefetches, and writes 16-byte streaming stores.
 // The per-index work decides the speed, so the common case is cut to a
 // handful of instructions:
 //
@@ -245,12 +246,17 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
   int32_t p0[kStage];
   int32_t c0 = tid < E1 ? load_expert(tid, p0) : 0;
 
-  // first vectors in flight while the tables are built
+  // first vectors in flight while the tables are built, and the batch after
+  // them requested into L2 (a prefetch holds no register): twice the bytes
+  // in flight while the plan loads are outstanding
   int i = tid;
   int4 x[kU];
 #pragma unroll
   for (int u = 0; u < kU; ++u)
     x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
+#pragma unroll
+  for (int u = 0; u < kU; ++u)
+    if (i + (kU + u) * kThreads < nvec) prefetch_l2(pin + i + (kU + u) * kThreads);
 
   if (tid < E1) vote_expert(tid, c0, p0);
   for (int e = tid + kThreads; e < E1; e += kThreads) {
@@ -359,6 +365,11 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
 #pragma unroll
       for (int u = 0; u < kU; ++u)
         x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
+      // one batch ahead into L2 (measured: -3 us on the 121.6 MB batch,
+      // even on the 1.95 GB stream; two batches ahead was slower)
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (i + (kU + u) * kThreads < nvec) prefetch_l2(pin + i + (kU + u) * kThreads);
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u)
