@@ -701,22 +701,14 @@ __device__ void write_error_row(const RbArgs &a, int64_t row) {
 // butterfly); their mean summed in GPU order from 0.0 divided by gpus; and
 // balancedness = mean / max (1 when max is 0).  Every add and divide is an
 // explicitly rounded fp64 operation in that fixed order, so the figures are
-// bit-identical to the same sums done sequentially on a CPU.  Inline: out of
-// line, and with a serial min / max loop, it cost 4 us of the 58-row step
-// (measured).  p2l: slot -> expert; w, lc: load and replicas by expert; q: P
-// doubles and gl: gpus doubles of scratch.
+// bit-identical to the same sums done sequentially on a CPU.  The quotients
+// q come from the assembly pass (one divide per thread: nine per lane here
+// took 1.4 us); inline: out of line, and with a serial min / max loop, it
+// cost 4 us of the 58-row step (measured).  q: P slot quotients, gl: gpus
+// doubles of scratch.
 __device__ __forceinline__ void plan_quality(double *gpu_load, double *stats, int64_t row,
-                                             int gpus, int ppg, int P, int E, const int32_t *p2l,
-                                             const int64_t *w, const int32_t *lc, double *q,
-                                             double *gl) {
+                                             int gpus, int ppg, const double *q, double *gl) {
   const int lane = threadIdx.x & 31;
-#pragma unroll 4
-  for (int p = lane; p < P; p += 32) {
-    const int e = p2l[p];
-    q[p] = e >= 0 && e < E ? __ddiv_rn(static_cast<double>(w[e]), static_cast<double>(lc[e]))
-                           : __longlong_as_double(0x7ff8000000000000LL);
-  }
-  __syncwarp();
   double mn = __longlong_as_double(0x7ff0000000000000LL), mx = 0.0;  // +inf, 0
   for (int g = lane; g < gpus; g += 32) {
     double acc = 0.0;
@@ -1049,9 +1041,10 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
   const bool in_smem = table_in_smem(s);
   int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
-  // plan quality: the slot -> expert map is kept in outp (unused by the
-  // shared-table path) for the quality warp
+  // plan quality: each slot's quotient w / logcnt, in the sort keys' space
+  // (free after step 3)
   const bool quality = a.gpu_load != nullptr || a.stats != nullptr;
+  double *qslot = reinterpret_cast<double *>(smem + lay.keys);
   bool slots = false;
   for (int t = tid; t < s.P; t += nthr()) {
     const int n = t / s.ppn;
@@ -1063,7 +1056,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
                      m >= n * s.lpn && m < (n + 1) * s.lpn,
                  a.status))
       continue;
-    if (quality) outp[pphy] = e;
+    if (quality) qslot[pphy] = __ddiv_rn(static_cast<double>(w[e]), static_cast<double>(cnt[m]));
     a.phy2log[row * s.P + pphy] = e;
     a.phyrank[row * s.P + pphy] = k;
     if (in_smem) {
@@ -1086,8 +1079,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   // weights' space, free after step 3) while the other warps copy the
   // table out
   if (quality && tid < 32)
-    plan_quality(a.gpu_load, a.stats, row, s.gpus, s.ppg, s.P, s.E, outp, w, lc,
-                 reinterpret_cast<double *>(smem + lay.keys),
+    plan_quality(a.gpu_load, a.stats, row, s.gpus, s.ppg, qslot,
                  reinterpret_cast<double *>(smem + lay.pw));
   if (in_smem) {
     const int t0 = quality ? 32 : 0;

@@ -931,6 +931,25 @@ def test_rebalance_fused_quality_shapes(shape):
     assert _np(st)[3, 3] == 1.0
 
 
+@pytest.mark.parametrize("shape", [(256, 8, 288, 4, 32), (256, 1, 288, 2, 144), (12, 4, 16, 2, 8),
+                                   (64, 32, 128, 16, 32), (300, 5, 602, 7, 7)])
+def test_rebalance_many_rows(shape):
+    """More rows than two per SM take the 128-thread many-row kernel: the same
+    plans and plan quality as the oracle's."""
+    E, G, P, N, gpus = shape
+    R = 2 * torch.cuda.get_device_properties(0).multi_processor_count + 11
+    rng = np.random.default_rng(E + P + R)
+    loads_np = (rng.pareto(1.3, (R, E)) * 1000).astype(np.int64)
+    loads_np[5] = 0
+    gl, st = _quality_bufs(R, gpus)
+    plan = eplb.rebalance(torch.from_numpy(loads_np).to(DEV), P, G, N, gpus, gpu_load=gl, stats=st)
+    ref, ref_status = _oracle_rows(loads_np, P, G, N, gpus, plan.log2phy.shape[2])
+    assert ref_status == 0
+    _assert_plan_equal(plan, ref)
+    ref_gl, ref_st = oracle.plan_stats(loads_np, ref[0], ref[2], gpus)
+    assert np.array_equal(_np(gl), ref_gl) and np.array_equal(_np(st), ref_st)
+
+
 def test_rebalance_fused_quality_worked_example():
     # the per-GPU load range the page prints for layer 0 of its example
     import json
