@@ -402,6 +402,38 @@ def test_redirect_arbitrary_tables(E, X, K, fused):
     assert int(bad.item()) == nbad and int(st.item()) == 0
 
 
+@pytest.mark.parametrize("fused", [False, True])
+def test_redirect_mixed_table_periods(fused):
+    """Layers whose replica counts all divide 24 take the short table, layers
+    with a count of 5 the 120-entry one, a count of 7 the descriptors: all in
+    one call, each equal to the oracle."""
+    L, T, K, E, X = 4, 5003, 8, 256, 9
+    rng = np.random.default_rng(77)
+    cnt = np.empty((L, E), np.int32)
+    cnt[0] = rng.choice([1, 2, 3, 4, 6, 8], E)   # period 24
+    cnt[1] = rng.choice([1, 2, 3, 4], E)
+    cnt[1, 17] = 5                                  # period 120
+    cnt[2] = 1
+    cnt[2, 200] = 7                                 # descriptors
+    cnt[3] = rng.choice([1, 2, 4, 8], E)            # period 24
+    l2p = np.full((L, E, X), -1, np.int32)
+    for l in range(L):
+        for e in range(E):
+            l2p[l, e, :cnt[l, e]] = rng.integers(0, 288, cnt[l, e])
+    idx = rng.integers(-1, E + 1, (L, T, K)).astype(np.int32)
+    d = lambda a: torch.from_numpy(a).to(DEV)
+    st = _status()
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    if fused:
+        counts, out = eplb.count_redirect(d(idx), E, d(l2p), d(cnt), 11, bad=bad, status=st)
+        assert np.array_equal(_np(counts), oracle.count_loads(idx, E)[0])
+    else:
+        out = eplb.redirect(d(idx), d(l2p), d(cnt), 11, bad=bad, status=st)
+    ref, nbad = oracle.redirect(idx, l2p, cnt, 11)
+    assert np.array_equal(_np(out), ref)
+    assert int(bad.item()) == nbad and int(st.item()) == 0
+
+
 def test_redirect_sharded_equals_whole(dsv3_idx):
     c = W.DSV3_PREFILL
     counts = eplb.count_loads(dsv3_idx, c.E)
