@@ -64,6 +64,11 @@
 #ifndef EPLB_RB_SHARED
 #define EPLB_RB_SHARED
 #endif
+// Loops strided by the CTA or a warp run once or twice per thread; they carry
+// `#pragma unroll 1`, since the compiler's default unrolling only adds code
+// that is fetched cold (the kernel 227 -> 171 KB of code; the 58-row
+// DeepSeek-V3 rebalance with plan quality 28.8 -> 25.5 us and the 58,000-row
+// sweep 4.6% faster, measured).
 
 namespace eplb {
 namespace {
@@ -303,6 +308,7 @@ __device__ EPLB_RB_COLD void bitonic_desc(K *key, int npad, int nseg) {
   const int half = (npad * nseg) >> 1;
   for (int k = 2; k <= npad; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll 1
       for (int t = threadIdx.x; t < half; t += nthr()) {
         const int i = ((t & ~(j - 1)) << 1) | (t & (j - 1));
         const int p = i | j;
@@ -403,6 +409,7 @@ __device__ EPLB_RB_COLD void pack_warp(const K *skey, int n, int m, int cap, K *
   const int lane = threadIdx.x & 31;
   const K imask = K(kIdxMask);
   const K kmax = ~K(0);
+#pragma unroll 1
   for (int q = lane; q < m; q += 32) {
     pw[q] = 0;
     pc[q] = 0;
@@ -424,6 +431,7 @@ __device__ EPLB_RB_COLD void pack_warp(const K *skey, int n, int m, int cap, K *
       ipack[item] = q;
       irank[item] = rk;
       K nb = kmax;
+#pragma unroll 1
       for (int qq = lane; qq < m; qq += 32)
         if (pc[qq] < cap) nb = kmin(nb, pw[qq] | K(qq));
       best = nb;
@@ -452,6 +460,7 @@ template <typename K>
 __device__ EPLB_RB_COLD void pack_cap2(const K *skey_base, int stride, int nseg, int m, int32_t *ipack,
                           int32_t *irank, int out_stride) {
   const K imask = K(kIdxMask);
+#pragma unroll 1
   for (int t = threadIdx.x; t < nseg * m; t += nthr()) {
     const int g = t / m;
     const int p = t - g * m;
@@ -493,6 +502,7 @@ __device__ EPLB_RB_SHARED void pack_segments(const K *skey, int stride, int nseg
     // nodes) the vote cost more than the short greedy it replaces (measured)
     if (cap == 2 && n == 2 * m && m >= kCap2MinPacks) {  // every segment has this shape
       bool ok = true;
+#pragma unroll 1
       for (int g = threadIdx.x; g < nseg; g += nthr())
         ok &= (skey[g * stride + m - 1] >> kIdxBits) != K(0);
       if (__syncthreads_and(ok)) {
@@ -519,6 +529,7 @@ __device__ EPLB_RB_COLD void pack_segments_wide(const K *skey, int stride, int n
   } else if (m <= 256 && sizeof(K) == 8) {
     pack_seg<K, 8>(skey, stride, nseg, n, m, cap, ipack, irank, out_stride);
   } else {
+#pragma unroll 1
     for (int g = threadIdx.x >> 5; g < nseg; g += nwarps())
       pack_warp<K>(skey + g * stride, n, m, cap, pw + g * m, pc + g * m, ipack + g * out_stride,
                    irank + g * out_stride);
@@ -551,6 +562,7 @@ __device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
   // D2 cross-multiplied compares.
   const int R = s.ppn - s.lpn, nc = num_cand(s);
   const int grid = nc * R;
+#pragma unroll 1
   for (int t = threadIdx.x; t < s.N * grid; t += nthr()) {
     const int n = t / grid;
     const int p = t - n * grid;
@@ -641,6 +653,7 @@ __device__ EPLB_RB_COLD void replicate_smem(int lpn, int ppn, int n, const int64
     bw = 0;
     bc = 1;
     bi = 0x7fffffff;
+#pragma unroll 1
     for (int i = lane; i < lpn; i += 32)
       if (rep_better(wm[bm + i], cnt[bm + i], i, bw, bc, bi)) {
         bw = wm[bm + i];
@@ -678,18 +691,22 @@ __device__ EPLB_RB_COLD void replicate_smem(int lpn, int ppn, int n, const int64
 // plan quality NaN.
 __device__ void write_error_row(const RbArgs &a, int64_t row) {
   const int P = a.s.P, E = a.s.E, X = a.s.X, gpus = a.s.gpus;
+#pragma unroll 1
   for (int t = threadIdx.x; t < P; t += nthr()) {
     a.phy2log[row * P + t] = -1;
     a.phyrank[row * P + t] = -1;
   }
+#pragma unroll 1
   for (int e = threadIdx.x; e < E; e += nthr()) a.logcnt[row * E + e] = 0;
   int32_t *gl = a.log2phy + row * static_cast<int64_t>(E) * X;
+#pragma unroll 1
   for (int i = threadIdx.x; i < E * X; i += nthr()) gl[i] = -1;
   const double nan = __longlong_as_double(0x7ff8000000000000LL);
-  if (a.gpu_load)
+  if (a.gpu_load) {
+#pragma unroll 1
     for (int g = threadIdx.x; g < gpus; g += nthr()) a.gpu_load[row * gpus + g] = nan;
-  if (a.stats)
-    for (int k = threadIdx.x; k < 4; k += nthr()) a.stats[row * 4 + k] = nan;
+  }
+  if (a.stats && threadIdx.x < 4) a.stats[row * 4 + threadIdx.x] = nan;
 }
 
 // Plan quality of the row just assembled, by one warp while the others copy
@@ -710,6 +727,7 @@ __device__ __forceinline__ void plan_quality(double *gpu_load, double *stats, in
                                              int gpus, int ppg, const double *q, double *gl) {
   const int lane = threadIdx.x & 31;
   double mn = __longlong_as_double(0x7ff0000000000000LL), mx = 0.0;  // +inf, 0
+#pragma unroll 1
   for (int g = lane; g < gpus; g += 32) {
     double acc = 0.0;
 #pragma unroll 4
@@ -769,6 +787,7 @@ __device__ void step3(const Step3Ops &o) {
   const K imask = K(kIdxMask);
   const bool ranked = npad <= kRankSortMax;
   const int per = ranked ? ppn : npad;
+#pragma unroll 1
   for (int t = threadIdx.x; t < N * per; t += nthr()) {
     const int n = t / per;
     const int j = t - n * per;
@@ -850,6 +869,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   {
     const int lane = tid & 31;
     const int64_t half = (a.ring_w + 1) >> 1;
+#pragma unroll 1
     for (int t = tid; t - lane < 2 * s.E; t += nthr()) {  // warp-uniform for the shuffle
       const bool live = t < 2 * s.E;
       const int e = t >> 1;
@@ -878,19 +898,23 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
 
   if (table_in_smem(s)) {  // the log2phy table starts all -1 (filled while step 1 runs)
     int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
+#pragma unroll 1
     for (int i = tid; i < s.E * s.X; i += nthr()) tbl[i] = -1;
   }
 
   // ---- step 1: groups -> nodes ---------------------------------------------
   if (s.gpn == 1) {  // one group per node: the pages' identity short-cut
+#pragma unroll 1
     for (int g = tid; g < s.G; g += nthr()) {
       gpack[g] = g;
       grank[g] = 0;
     }
   } else {
+#pragma unroll 1
     for (int g = tid >> 5; g < s.G; g += nwarps()) {  // one warp per group
       const int lane = tid & 31;
       uint64_t sum = 0;
+#pragma unroll 1
       for (int i = lane; i < s.gs; i += 32) sum += static_cast<uint64_t>(w[g * s.gs + i]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
@@ -901,6 +925,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     if (s.gpad <= kRankSortMax) {
       rank_sort<uint64_t>(gkey, s.gpad, 1, s.G, gsorted);
     } else {
+#pragma unroll 1
       for (int g = s.G + tid; g < s.gpad; g += nthr()) gkey[g] = 0;
       __syncthreads();
       bitonic_desc<uint64_t>(gkey, s.gpad, 1);
@@ -913,6 +938,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   }
   __syncthreads();
   // mlog = logical order after the node permutation; replicate's initial state
+#pragma unroll 1
   for (int e = tid; e < s.E; e += nthr()) {
     const int g = e / s.gs;
     const int m = (gpack[g] * s.gpn + grank[g]) * s.gs + (e - g * s.gs);
@@ -932,6 +958,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   if (nc > 0 && nc <= 32) {
     // candidates: the nc heaviest experts of each node (ties by index)
     uint64_t *ckey = reinterpret_cast<uint64_t *>(smem + lay.keys);
+#pragma unroll 1
     for (int m = tid; m < s.E; m += nthr()) {
       const int n = m / s.lpn;
       ckey[m] = (static_cast<uint64_t>(wm[m]) << kIdxBits) | (kIdxMask - (m - n * s.lpn));
@@ -940,6 +967,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     uint64_t *csorted = reinterpret_cast<uint64_t *>(smem + lay.sorted);
     rank_sort<uint64_t>(ckey, s.lpn, s.N, s.lpn, csorted);
     __syncthreads();
+#pragma unroll 1
     for (int t = tid; t < s.N * nc; t += nthr()) {  // the nc heaviest of each node
       const int g = t / nc;
       const int j = static_cast<int>(kIdxMask - (csorted[g * s.lpn + (t - g * nc)] & kIdxMask));
@@ -948,25 +976,30 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     }
     __syncthreads();
     if (nc * (s.ppn - s.lpn) <= 256) {
+#pragma unroll 1
       for (int t = tid; t < s.N * nc; t += nthr()) cand_c[t] = 1;
       __syncthreads();
       replicate_pairs(s, cand_w, cand_i, cand_c, p2m, rrank);
     } else {
+#pragma unroll 1
       for (int n = tid >> 5; n < s.N; n += nwarps())
         replicate_warp(nc, s.lpn, s.ppn, n, cand_w, cand_i, cand_c, p2m, rrank);
     }
     __syncthreads();
+#pragma unroll 1
     for (int t = tid; t < s.N * nc; t += nthr()) {
       const int n = t / nc;
       if (EPLB_IN(cand_i[t] >= 0 && cand_i[t] < s.lpn, a.status)) cnt[n * s.lpn + cand_i[t]] = cand_c[t];
     }
   } else if (nc > 32) {
+#pragma unroll 1
     for (int n = tid >> 5; n < s.N; n += nwarps()) replicate_smem(s.lpn, s.ppn, n, wm, cnt, p2m, rrank);
   }
   __syncthreads();
 
   // ---- Lambda and key width per node (one thread per node) ----------------
   if (s.ppg > 1) {
+#pragma unroll 1
     for (int n = tid; n < s.N; n += nthr()) {
       int64_t wmax = 0;
       if (nc > 0 && nc <= 32) {
@@ -1017,6 +1050,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
 
   // ---- step 3: replicas -> GPUs of each node ------------------------------
   if (s.ppg == 1) {  // one replica per GPU: identity short-cut
+#pragma unroll 1
     for (int t = tid; t < s.P; t += nthr()) {
       const int n = t / s.ppn;
       ipack[t] = t - n * s.ppn;
@@ -1046,6 +1080,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   const bool quality = a.gpu_load != nullptr || a.stats != nullptr;
   double *qslot = reinterpret_cast<double *>(smem + lay.keys);
   bool slots = false;
+#pragma unroll 1
   for (int t = tid; t < s.P; t += nthr()) {
     const int n = t / s.ppn;
     const int pphy = n * s.ppn + ipack[t] * s.ppg + irank[t];
@@ -1069,6 +1104,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       outr[pphy] = k;
     }
   }
+#pragma unroll 1
   for (int m = tid; m < s.E; m += nthr()) {
     const int e = mlog2log[m];
     lc[e] = cnt[m];
@@ -1088,12 +1124,15 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
       if (a.table_vec4) {
         const int4 *src = reinterpret_cast<const int4 *>(tbl);
         int4 *dst = reinterpret_cast<int4 *>(gl);
+#pragma unroll 1
         for (int i = tid - t0; i < (EX >> 2); i += nt) dst[i] = src[i];
       } else {
+#pragma unroll 1
         for (int i = tid - t0; i < EX; i += nt) gl[i] = tbl[i];
       }
     }
   } else {
+#pragma unroll 1
     for (int t = tid; t < s.P; t += nthr()) {
       const int k = outr[t];
       if (!EPLB_IN(outp[t] >= 0 && outp[t] < s.E && k >= 0, a.status)) continue;
@@ -1103,6 +1142,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
         slots = true;
     }
     const uint32_t X = static_cast<uint32_t>(s.X);
+#pragma unroll 1
     for (int i = tid; i < EX; i += nthr()) {
       const uint32_t e = div_magic(static_cast<uint32_t>(i), X, a.x_magic);
       if (static_cast<int>(i - e * X) >= lc[e]) gl[i] = -1;
