@@ -37,6 +37,14 @@ __device__ __forceinline__ bool check_in(bool cond, int32_t *status) {
 __device__ __forceinline__ void red_shared_inc(uint32_t addr) {
   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr));
 }
+__device__ __forceinline__ uint64_t ld_shared_u64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void ld_shared_u64x2(uint32_t addr, uint64_t &x, uint64_t &y) {
+  asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(x), "=l"(y) : "r"(addr));
+}
 __device__ __forceinline__ int32_t ld_shared_s16(uint32_t addr) {
   int32_t v;
   asm volatile("ld.shared.s16 %0, [%1];" : "=r"(v) : "r"(addr));

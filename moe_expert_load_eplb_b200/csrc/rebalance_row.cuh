@@ -218,6 +218,45 @@ __device__ __forceinline__ bool lcm_into(uint64_t &lam, uint32_t c) {
 }
 
 // ---------------------------------------------------------------------------
+// r[q] += the number of keys in [i0, i1) of a segment greater than me[q].
+// 64-bit keys are read by 32-bit shared address, two per 16-byte load: the
+// rank sort runs out of line, where the compiler cannot tell that the keys
+// are in shared memory, and its generic single-key loads measured 1.6-2.3x
+// slower on 8-288 keys.  128-bit keys (a rare path) keep the plain loop.
+template <int Q, typename K>
+__device__ __forceinline__ void count_greater(const K *seg, int i0, int i1, const K (&me)[Q],
+                                              int (&r)[Q]) {
+  if constexpr (sizeof(K) == 8) {
+    const uint32_t base = smem_u32(seg);
+    int i = i0;
+    if (i < i1 && ((base + 8u * i) & 15u) != 0) {
+      const uint64_t x = ld_shared_u64(base + 8u * i);
+#pragma unroll
+      for (int q = 0; q < Q; ++q) r[q] += x > me[q] ? 1 : 0;
+      ++i;
+    }
+#pragma unroll 4
+    for (; i + 1 < i1; i += 2) {
+      uint64_t x, y;
+      ld_shared_u64x2(base + 8u * i, x, y);
+#pragma unroll
+      for (int q = 0; q < Q; ++q) r[q] += (x > me[q] ? 1 : 0) + (y > me[q] ? 1 : 0);
+    }
+    if (i < i1) {
+      const uint64_t x = ld_shared_u64(base + 8u * i);
+#pragma unroll
+      for (int q = 0; q < Q; ++q) r[q] += x > me[q] ? 1 : 0;
+    }
+  } else {
+#pragma unroll 4
+    for (int i = i0; i < i1; ++i) {
+      const K kk = seg[i];
+#pragma unroll
+      for (int q = 0; q < Q; ++q) r[q] += kk > me[q] ? 1 : 0;
+    }
+  }
+}
+
 // Descending ranks of n distinct keys in each of nseg segments (segment g at
 // key + g * stride).  Threads are grouped by segment (nthr() / nseg per
 // segment); each ranks Q keys per pass (Q = 1, 2 or 4, the fewest that cover
@@ -240,12 +279,7 @@ __device__ void rank_pass(const K *key, int stride, int nseg, int n, int tps, Em
         me[q] = j < n ? seg[j] : ~K(0);
         r[q] = 0;
       }
-#pragma unroll 4
-      for (int i = 0; i < n; ++i) {
-        const K kk = seg[i];
-#pragma unroll
-        for (int q = 0; q < Q; ++q) r[q] += kk > me[q] ? 1 : 0;
-      }
+      count_greater<Q, K>(seg, 0, n, me, r);
 #pragma unroll
       for (int q = 0; q < Q; ++q) {
         const int j = j0 + q * tps;
@@ -270,14 +304,11 @@ __device__ void rank_pass_split(const K *key, int stride, int nseg, int n, int t
     const int g = g0 + gl;
     const bool live = gl < segs_per_pass && g < nseg && j < n;
     const K *seg = key + (live ? g : 0) * stride;
-    const K me = live ? seg[j] : K(0);
-    int r = 0;
-    if (live) {
-#pragma unroll 4
-      for (int i = i0; i < i1; ++i) r += seg[i] > me ? 1 : 0;
-    }
-    r += __shfl_xor_sync(0xffffffffu, r, 1);
-    if (live && half == 0) emit(g, j, r, me);
+    const K me[1] = {live ? seg[j] : K(0)};
+    int r[1] = {0};
+    if (live) count_greater<1, K>(seg, i0, i1, me, r);
+    r[0] += __shfl_xor_sync(0xffffffffu, r[0], 1);
+    if (live && half == 0) emit(g, j, r[0], me[0]);
   }
 }
 
@@ -294,11 +325,43 @@ __device__ void rank_segments(const K *key, int stride, int nseg, int n, Emit em
     rank_pass<4, K>(key, stride, nseg, n, tps, emit);
 }
 
+// The general passes, out of line: the common shapes below never fetch them.
+template <typename K>
+__device__ EPLB_RB_COLD void rank_sort_general(const K *key, int stride, int nseg, int n, K *out) {
+  rank_segments<K>(key, stride, nseg, n, [&](int g, int, int r, K k) { out[g * stride + r] = k; });
+}
+
 // Descending ranks written out: out[g * stride + rank] = key (the stable
 // (value desc, index asc) order of the composite keys).
 template <typename K>
 __device__ EPLB_RB_SHARED void rank_sort(const K *key, int stride, int nseg, int n, K *out) {
-  rank_segments<K>(key, stride, nseg, n, [&](int g, int, int r, K k) { out[g * stride + r] = k; });
+  if constexpr (sizeof(K) == 8) {
+    // one key per thread: a warp per segment when it holds one (lanes are
+    // keys, no index arithmetic), else nthr() / nseg threads per segment.
+    // These two shapes cover the 8-, 64- and 72-key sorts of the DeepSeek-V3
+    // row; the general passes cost 0.4-0.9 us more there in their index
+    // arithmetic (measured).
+    int g = -1, j = 0;
+    if (n <= 32 && nseg <= nwarps()) {
+      g = threadIdx.x >> 5;
+      j = threadIdx.x & 31;
+    } else if (nseg <= nthr() && n <= nthr() / nseg) {
+      const int tps = nthr() / nseg;
+      g = threadIdx.x / tps;
+      j = threadIdx.x - g * tps;
+    }
+    if (g >= 0) {
+      if (g < nseg && j < n) {
+        const K *seg = key + g * stride;
+        const K me[1] = {seg[j]};
+        int r[1] = {0};
+        count_greater<1, K>(seg, 0, n, me, r);
+        out[g * stride + r[0]] = me[0];
+      }
+      return;
+    }
+  }
+  rank_sort_general<K>(key, stride, nseg, n, out);
 }
 
 // CTA-wide bitonic sort, descending, of nseg segments of npad (power of two)
@@ -719,10 +782,16 @@ __device__ void write_error_row(const RbArgs &a, int64_t row) {
 // balancedness = mean / max (1 when max is 0).  Every add and divide is an
 // explicitly rounded fp64 operation in that fixed order, so the figures are
 // bit-identical to the same sums done sequentially on a CPU.  The quotients
-// q come from the assembly pass (one divide per thread: nine per lane here
-// took 1.4 us); inline: out of line, and with a serial min / max loop, it
-// cost 4 us of the 58-row step (measured).  q: P slot quotients, gl: gpus
-// doubles of scratch.
+// q are divided while step 3 packs (one per expert, by the idle warps: nine
+// per lane here took 1.4 us) and placed by the assembly pass; inline: out of
+// line, and with a serial min / max loop, it cost 4 us of the 58-row step
+// (measured).  q: P slot quotients, gl: gpus doubles of scratch.
+// one out-of-line copy of the correctly rounded fp64 divide, off the row's
+// straight-line code
+__device__ EPLB_RB_COLD double qdiv(double a, double b) { return __ddiv_rn(a, b); }
+
+constexpr int kQualityRegs = 12;  // replicas per GPU summed from registers
+
 __device__ __forceinline__ void plan_quality(double *gpu_load, double *stats, int64_t row,
                                              int gpus, int ppg, const double *q, double *gl) {
   const int lane = threadIdx.x & 31;
@@ -730,8 +799,17 @@ __device__ __forceinline__ void plan_quality(double *gpu_load, double *stats, in
 #pragma unroll 1
   for (int g = lane; g < gpus; g += 32) {
     double acc = 0.0;
+    if (ppg <= kQualityRegs) {  // every load issued before the ordered adds
+      double v[kQualityRegs];
+#pragma unroll
+      for (int k = 0; k < kQualityRegs; ++k) v[k] = k < ppg ? q[g * ppg + k] : 0.0;
+#pragma unroll
+      for (int k = 0; k < kQualityRegs; ++k)
+        if (k < ppg) acc = __dadd_rn(acc, v[k]);
+    } else {
 #pragma unroll 4
-    for (int k = 0; k < ppg; ++k) acc = __dadd_rn(acc, q[g * ppg + k]);
+      for (int k = 0; k < ppg; ++k) acc = __dadd_rn(acc, q[g * ppg + k]);
+    }
     gl[g] = acc;
     if (gpu_load) gpu_load[row * gpus + g] = acc;
     mn = fmin(mn, acc);
@@ -755,11 +833,11 @@ __device__ __forceinline__ void plan_quality(double *gpu_load, double *stats, in
       for (int j = 0; j < 8; ++j) sum = __dadd_rn(sum, v[j]);
     }
     for (; g < gpus; ++g) sum = __dadd_rn(sum, gl[g]);
-    const double mean = __ddiv_rn(sum, static_cast<double>(gpus));
+    const double mean = qdiv(sum, static_cast<double>(gpus));
     stats[row * 4 + 0] = mn;
     stats[row * 4 + 1] = mx;
     stats[row * 4 + 2] = mean;
-    stats[row * 4 + 3] = mx > 0.0 ? __ddiv_rn(mean, mx) : 1.0;
+    stats[row * 4 + 3] = mx > 0.0 ? qdiv(mean, mx) : 1.0;
   }
 }
 
@@ -1065,6 +1143,16 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
                       reinterpret_cast<int32_t *>(smem + lay.pc), ipack, irank, s.N, s.npad, s.lpn,
                       s.ppn, s.mpn, s.ppg, a.status);
   }
+  // plan quality: every logical expert's slot value w / logcnt, by the warps
+  // the packing chain leaves idle (the highest thread ids take the first
+  // experts), into the raw loads' space (free after step 1)
+  const bool quality = a.gpu_load != nullptr || a.stats != nullptr;
+  double *qm = reinterpret_cast<double *>(smem + lay.w);
+  if (quality) {
+#pragma unroll 1
+    for (int m = nthr() - 1 - tid; m < s.E; m += nthr())
+      qm[m] = qdiv(static_cast<double>(wm[m]), static_cast<double>(cnt[m]));
+  }
   __syncthreads();
 
   // ---- assembly: pphy = node*ppn + gpu*ppg + rank -------------------------
@@ -1075,9 +1163,8 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   int32_t *gl = a.log2phy + row * static_cast<int64_t>(EX);
   const bool in_smem = table_in_smem(s);
   int32_t *tbl = reinterpret_cast<int32_t *>(smem + lay.table);
-  // plan quality: each slot's quotient w / logcnt, in the sort keys' space
-  // (free after step 3)
-  const bool quality = a.gpu_load != nullptr || a.stats != nullptr;
+  // plan quality: each slot's quotient, in the sort keys' space (free after
+  // step 3)
   double *qslot = reinterpret_cast<double *>(smem + lay.keys);
   bool slots = false;
 #pragma unroll 1
@@ -1091,7 +1178,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
                      m >= n * s.lpn && m < (n + 1) * s.lpn,
                  a.status))
       continue;
-    if (quality) qslot[pphy] = __ddiv_rn(static_cast<double>(w[e]), static_cast<double>(cnt[m]));
+    if (quality) qslot[pphy] = qm[m];
     a.phy2log[row * s.P + pphy] = e;
     a.phyrank[row * s.P + pphy] = k;
     if (in_smem) {
