@@ -504,9 +504,9 @@ __device__ EPLB_RB_COLD void pack_warp(const K *skey, int n, int m, int cap, K *
 }
 
 // The greedy in closed form when every pack takes exactly two items
-// (n == 2m) and the m heaviest items all weigh more than zero.  Round 1:
+// (n == 2m) and the m heaviest items all weigh more than zero.  First items:
 // item j (sorted, 0-based) finds packs 0..j-1 heavier than the empty ones,
-// so it opens pack j.  Round 2: no pack changes weight until it is full, so
+// so it opens pack j.  Second items: no pack changes weight until it is full, so
 // the packs take their second item lightest first -- ascending (weight,
 // index) of their first item -- and pack p takes item m + pos(p).  One
 // thread per pack, no dependent chain.
