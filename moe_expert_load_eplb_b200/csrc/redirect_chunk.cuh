@@ -188,27 +188,24 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
   uint32_t m_magic = a.m_magic;
   uint64_t div_mask = a.div_mask;
 
-  // this CTA: chunk j of layer l, elements [g, g1); chunk boundaries inside
-  // a layer are rounded down to 4 elements so the interior stays 16-byte
-  // aligned
+  // this CTA: part j of layer l.  The layer's 16-byte aligned interior
+  // [b0, b1) is cut into blocks of kThreads * kU vectors and part j takes
+  // blocks j, j + chunks, j + 2 * chunks, ...: the layer's CTAs sweep it
+  // side by side, so the DRAM pages they read and write are few at a time
+  // (the same copy traffic with one contiguous range per CTA measured 2 us
+  // slower behind the step's dirty L2).  Part 0 also takes the up to 3
+  // elements before b0 and after b1.
   const int64_t layer = cta / a.chunks;
   const int64_t j = cta - layer * a.chunks;
   const int64_t lbase = layer * a.per_layer;
-  auto bound = [&](int64_t q) -> int64_t {
-    if (q == 0) return lbase;
-    if (q == a.chunks) return lbase + a.per_layer;
-    const int64_t b = (lbase + a.per_layer * q / a.chunks) & ~int64_t(3);
-    return min(max(b, lbase), lbase + a.per_layer);
-  };
-  const int64_t g = bound(j);
-  const int64_t g1 = bound(j + 1);
-  // [g, b0) head, [b0, b1) 16-byte aligned interior, [b1, g1) tail
+  const int64_t g = lbase, g1 = lbase + a.per_layer;
   const int64_t b0 = min((g + 3) & ~int64_t(3), g1);
   const int64_t b1 = max(g1 & ~int64_t(3), b0);
   const int4 *pin = reinterpret_cast<const int4 *>(a.idx) + (b0 >> 2);
   int4 *pout = reinterpret_cast<int4 *>(a.out) + (b0 >> 2);
   const int nvec = static_cast<int>((b1 - b0) >> 2);
   const uint32_t pos0 = static_cast<uint32_t>(b0 - lbase);
+  const int step = static_cast<int>(a.chunks) * (kThreads * kU);  // vectors between blocks
 
   const int32_t *l2p_layer = a.log2phy + layer * static_cast<int64_t>(a.E) * a.X;
   const int32_t *cnt = a.logcnt + layer * a.E;
@@ -254,14 +251,14 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
   // first vectors in flight while the tables are built, and the batch after
   // them requested into L2 (a prefetch holds no register): twice the bytes
   // in flight while the plan loads are outstanding
-  int i = tid;
+  int i = static_cast<int>(j) * (kThreads * kU) + tid;
   int4 x[kU];
 #pragma unroll
   for (int u = 0; u < kU; ++u)
     x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
 #pragma unroll
   for (int u = 0; u < kU; ++u)
-    if (i + (kU + u) * kThreads < nvec) prefetch_l2(pin + i + (kU + u) * kThreads);
+    if (i + step + u * kThreads < nvec) prefetch_l2(pin + i + step + u * kThreads);
 
   // a layer whose replica counts all divide 24 (1..4, 6, 8, 12, 24) gets the
   // 24-entry period: a fifth of the table to build before streaming
@@ -350,12 +347,12 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
   auto ctx_desc = [&](uint32_t tok) -> uint2 { return make_uint2(selector(tok), tok); };
 
   auto stream = [&](auto ctx_of, auto map1) {
-    if (tid < b0 - g) {
+    if (j == 0 && tid < b0 - g) {
       const int64_t p = g + tid;
       const uint32_t tok = a.t0 + div_magic(static_cast<uint32_t>(p - lbase), a.K, a.k_magic);
       a.out[p] = map1(__ldg(a.idx + p), ctx_of(tok));
     }
-    if (tid >= 32 && tid - 32 < g1 - b1) {
+    if (j == 0 && tid >= 32 && tid - 32 < g1 - b1) {
       const int64_t p = b1 + (tid - 32);
       const uint32_t tok = a.t0 + div_magic(static_cast<uint32_t>(p - lbase), a.K, a.k_magic);
       a.out[p] = map1(__ldg(a.idx + p), ctx_of(tok));
@@ -378,10 +375,12 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
       __stcs(pout + v, y);
     };
     // whole batches without per-vector range checks, then the guarded rest
+    // (a batch that is not whole is the thread's last: the next one starts
+    // a whole block further on)
     while (i + (kU - 1) * kThreads < nvec) {
 #pragma unroll
       for (int u = 0; u < kU; ++u) vector(i + u * kThreads, x[u]);
-      i += kThreads * kU;
+      i += step;
 #pragma unroll
       for (int u = 0; u < kU; ++u)
         x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
@@ -389,7 +388,7 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
       // even on the 1.95 GB stream; two batches ahead was slower)
 #pragma unroll
       for (int u = 0; u < kU; ++u)
-        if (i + (kU + u) * kThreads < nvec) prefetch_l2(pin + i + (kU + u) * kThreads);
+        if (i + step + u * kThreads < nvec) prefetch_l2(pin + i + step + u * kThreads);
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u)
