@@ -5,9 +5,11 @@
 //   counts[l, e] += #{(t, k) : idx[l, t, k] == e}.
 //
 // HBM-bound streaming design for B200:
-//   * one 512-thread CTA per chunk of one layer: the grid is just under a
-//     whole number of waves (up to 8), so the block scheduler gives the
-//     chunks of slow SMs to fast ones and no thin last wave is left;
+//   * a layer's work is split over several 512-thread CTAs, which take its
+//     blocks of 4096 vectors in turn (they sweep the layer side by side);
+//     the grid is just under a whole number of waves (up to 8), so the
+//     block scheduler gives the parts of slow SMs to fast ones and no thin
+//     last wave is left;
 //   * every thread keeps U independent 16-byte streaming loads
 //     (ld.global.cs) in flight -- on a B200 this measured faster than
 //     staging the same bytes through shared memory with cp.async.bulk (4- to
@@ -51,26 +53,22 @@ __global__ void __launch_bounds__(kThreads) count_loads_kernel(CountArgs a) {
   const int E1 = a.E + 1;
   uint32_t *hist_lane = hist + lane;
 
-  // chunk j of layer l: elements [g, g1), inner boundaries rounded down to 4
+  // part j of layer l: blocks j, j + chunks, ... of kThreads * kU vectors
+  // of the layer's 16-byte aligned interior [b0, b1), so that the layer's
+  // CTAs sweep it side by side (as in the redirect kernel); part 0 also
+  // takes the up to 3 elements before b0 and after b1
   const int64_t layer = blockIdx.x / a.chunks;
   const int64_t j = blockIdx.x - layer * a.chunks;
   const int64_t lbase = layer * a.per_layer;
-  auto bound = [&](int64_t q) -> int64_t {
-    if (q == 0) return lbase;
-    if (q == a.chunks) return lbase + a.per_layer;
-    const int64_t b = (lbase + a.per_layer * q / a.chunks) & ~int64_t(3);
-    return min(max(b, lbase), lbase + a.per_layer);
-  };
-  const int64_t g = bound(j);
-  const int64_t g1 = bound(j + 1);
-  // [g, b0) head, [b0, b1) 16-byte aligned interior, [b1, g1) tail
+  const int64_t g = lbase, g1 = lbase + a.per_layer;
   const int64_t b0 = min((g + 3) & ~int64_t(3), g1);
   const int64_t b1 = max(g1 & ~int64_t(3), b0);
   const int4 *pin = reinterpret_cast<const int4 *>(a.idx) + (b0 >> 2);
   const int nvec = static_cast<int>((b1 - b0) >> 2);
+  const int step = static_cast<int>(a.chunks) * (kThreads * kU);
 
   // first vectors in flight while the histogram is cleared
-  int i = tid;
+  int i = static_cast<int>(j) * (kThreads * kU) + tid;
   int4 x[kU];
 #pragma unroll
   for (int u = 0; u < kU; ++u)
@@ -79,8 +77,8 @@ __global__ void __launch_bounds__(kThreads) count_loads_kernel(CountArgs a) {
   __syncthreads();
 
   auto add = [&](int32_t e) { atomicAdd(hist_lane + min(static_cast<uint32_t>(e), E) * 32u, 1u); };
-  if (tid < b0 - g) add(__ldg(a.idx + g + tid));
-  if (tid >= 32 && tid - 32 < g1 - b1) add(__ldg(a.idx + b1 + (tid - 32)));
+  if (j == 0 && tid < b0 - g) add(__ldg(a.idx + g + tid));
+  if (j == 0 && tid >= 32 && tid - 32 < g1 - b1) add(__ldg(a.idx + b1 + (tid - 32)));
   while (i < nvec) {
 #pragma unroll
     for (int u = 0; u < kU; ++u) {
@@ -91,7 +89,7 @@ __global__ void __launch_bounds__(kThreads) count_loads_kernel(CountArgs a) {
         add(x[u].w);
       }
     }
-    i += kThreads * kU;
+    i += step;
 #pragma unroll
     for (int u = 0; u < kU; ++u)
       x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
