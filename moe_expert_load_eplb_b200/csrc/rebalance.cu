@@ -74,6 +74,7 @@ eplb_status launch_rebalance(int64_t *ring, int64_t ring_w, int64_t zero_slot, i
   a.stats = stats;
   a.s = sh;
   a.x_magic = 0xffffffffu / static_cast<uint32_t>(sh.X);
+  set_row_magics(a);
   a.table_vec4 = ((static_cast<int64_t>(sh.E) * sh.X) % 4 == 0) &&
                  (reinterpret_cast<uintptr_t>(log2phy) % 16 == 0);
   const int threads = many ? kManyRowThreads : kFewRowThreads;

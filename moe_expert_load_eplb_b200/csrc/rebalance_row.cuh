@@ -106,6 +106,11 @@ struct RbArgs {
   RebalanceShape s;
   uint32_t x_magic;
   int table_vec4;  // log2phy rows may be written as 16-byte vectors
+  // multiply-high divisors (floor((2^32 - 1) / d), 0 for d = 0) of the row's
+  // index arithmetic: gs, lpn, ppn, the candidates nc, the extra replicas
+  // R = ppn - lpn, nc * R, and step 3's keys per node; a 32-bit divide by a
+  // run-time value is a long dependent sequence on the row's critical path
+  uint32_t m_gs, m_lpn, m_ppn, m_nc, m_r, m_grid, m_per;
 };
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
@@ -116,6 +121,23 @@ __host__ __device__ inline bool table_in_smem(const RebalanceShape &s) {
 // experts per node that can receive extra replicas
 __host__ __device__ inline int num_cand(const RebalanceShape &s) {
   return min(s.ppn - s.lpn, s.lpn);
+}
+
+// x / d for 0 <= x < 2^31 by the magic m of d (common.cuh's div_magic)
+__device__ __forceinline__ int qdivm(int x, int d, uint32_t m) {
+  return static_cast<int>(div_magic(static_cast<uint32_t>(x), static_cast<uint32_t>(d), m));
+}
+inline uint32_t row_magic(int32_t d) { return d > 0 ? 0xffffffffu / static_cast<uint32_t>(d) : 0u; }
+inline void set_row_magics(RbArgs &a) {
+  const RebalanceShape &s = a.s;
+  const int nc = num_cand(s), R = s.ppn - s.lpn;
+  a.m_gs = row_magic(s.gs);
+  a.m_lpn = row_magic(s.lpn);
+  a.m_ppn = row_magic(s.ppn);
+  a.m_nc = row_magic(nc);
+  a.m_r = row_magic(R);
+  a.m_grid = row_magic(nc * R);
+  a.m_per = row_magic(s.npad <= kRankSortMax ? s.ppn : s.npad);  // step 3's keys per node
 }
 
 // Shared-memory carve-up of one row (byte offsets), identical on host and device.
@@ -346,9 +368,15 @@ __device__ EPLB_RB_SHARED void rank_sort(const K *key, int stride, int nseg, int
       g = threadIdx.x >> 5;
       j = threadIdx.x & 31;
     } else if (nseg <= nthr() && n <= nthr() / nseg) {
-      const int tps = nthr() / nseg;
-      g = threadIdx.x / tps;
-      j = threadIdx.x - g * tps;
+      if ((nseg & (nseg - 1)) == 0) {  // nthr() is a power of two too: shifts
+        const int ls = (__ffs(nthr()) - 1) - (__ffs(nseg) - 1);
+        g = threadIdx.x >> ls;
+        j = threadIdx.x - (g << ls);
+      } else {
+        const int tps = nthr() / nseg;
+        g = threadIdx.x / tps;
+        j = threadIdx.x - g * tps;
+      }
     }
     if (g >= 0) {
       if (g < nseg && j < n) {
@@ -411,9 +439,10 @@ __device__ void pack_seg(const K *skey_base, int stride, int nseg, int n, int m,
   if (PL > 1) ms = 32;
   const int lane = threadIdx.x & 31;
   const int li = lane & (ms - 1);            // lane within the segment
-  const int slot = static_cast<int>(threadIdx.x) / ms;
-  const int slots = nthr() / ms;
-  const int warp_first_slot = (static_cast<int>(threadIdx.x) & ~31) / ms;
+  const int lms = __ffs(ms) - 1;  // ms is a power of two
+  const int slot = static_cast<int>(threadIdx.x) >> lms;
+  const int slots = nthr() >> lms;
+  const int warp_first_slot = (static_cast<int>(threadIdx.x) & ~31) >> lms;
   for (int g0 = 0; g0 < nseg; g0 += slots) {
     if (g0 + warp_first_slot >= nseg) continue;  // no segment of this warp is live: skip the chain
     const int g = g0 + slot;
@@ -616,7 +645,7 @@ __device__ __forceinline__ bool rep_better(int64_t aw, int ac, int ai, int64_t b
 // pairs of all nodes are ranked in parallel; the picks need no serial chain.
 __device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
                                 const int32_t *cand_i, int32_t *cand_c, int32_t *p2m,
-                                int32_t *rrank) {
+                                int32_t *rrank, uint32_t m_grid, uint32_t m_r) {
   // Pair (k, d) -- candidate k's d-th extra replica, value w_k / d -- ranks
   // after every pair of greater value, and after equal-valued pairs of a
   // lower expert index (same expert: lower d).  Candidate k2 has D2 = R - k2
@@ -627,9 +656,9 @@ __device__ void replicate_pairs(const RebalanceShape &s, const int64_t *cand_w,
   const int grid = nc * R;
 #pragma unroll 1
   for (int t = threadIdx.x; t < s.N * grid; t += nthr()) {
-    const int n = t / grid;
+    const int n = qdivm(t, grid, m_grid);
     const int p = t - n * grid;
-    const int k = p / R;
+    const int k = qdivm(p, R, m_r);
     const int d = p - k * R + 1;
     if (d > R - k) continue;
     const int64_t w = cand_w[n * nc + k];
@@ -851,6 +880,7 @@ struct Step3Ops {
   int32_t *pc, *ipack, *irank;
   int N, npad, lpn, ppn, mpn, ppg;
   int32_t *status;  // the checking build's reports
+  uint32_t m_per;   // magic of the keys per node
 };
 
 template <typename K, bool kCap2>
@@ -867,7 +897,7 @@ __device__ void step3(const Step3Ops &o) {
   const int per = ranked ? ppn : npad;
 #pragma unroll 1
   for (int t = threadIdx.x; t < N * per; t += nthr()) {
-    const int n = t / per;
+    const int n = qdivm(t, per, o.m_per);
     const int j = t - n * per;
     K key = 0;
     if (j < ppn && EPLB_IN(p2m[n * ppn + j] >= 0 && p2m[n * ppn + j] < lpn, o.status)) {
@@ -901,9 +931,9 @@ __device__ void step3_wide(unsigned char *keys, unsigned char *sorted, unsigned 
                                         const int64_t *wm, const uint64_t *lam, const int32_t *cnt,
                                         const int32_t *p2m, int32_t *pc, int32_t *ipack,
                                         int32_t *irank, int N, int npad, int lpn, int ppn, int mpn,
-                                        int ppg, int32_t *status) {
+                                        int ppg, int32_t *status, uint32_t m_per) {
   step3<u128, kCap2>(Step3Ops{keys, sorted, pw, wm, lam, cnt, p2m, pc, ipack, irank, N, npad, lpn,
-                              ppn, mpn, ppg, status});
+                              ppn, mpn, ppg, status, m_per});
 }
 
 // One row of rebalance_experts, by the whole CTA, in `smem` (Layout(a.s).total
@@ -1018,13 +1048,13 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   // mlog = logical order after the node permutation; replicate's initial state
 #pragma unroll 1
   for (int e = tid; e < s.E; e += nthr()) {
-    const int g = e / s.gs;
+    const int g = qdivm(e, s.gs, a.m_gs);
     const int m = (gpack[g] * s.gpn + grank[g]) * s.gs + (e - g * s.gs);
     if (!EPLB_IN(m >= 0 && m < s.E, a.status)) continue;
     mlog2log[m] = e;
     wm[m] = w[e];
     cnt[m] = 1;
-    const int n = m / s.lpn;
+    const int n = qdivm(m, s.lpn, a.m_lpn);
     const int i = m - n * s.lpn;
     p2m[n * s.ppn + i] = i;
     rrank[n * s.ppn + i] = 0;
@@ -1038,7 +1068,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     uint64_t *ckey = reinterpret_cast<uint64_t *>(smem + lay.keys);
 #pragma unroll 1
     for (int m = tid; m < s.E; m += nthr()) {
-      const int n = m / s.lpn;
+      const int n = qdivm(m, s.lpn, a.m_lpn);
       ckey[m] = (static_cast<uint64_t>(wm[m]) << kIdxBits) | (kIdxMask - (m - n * s.lpn));
     }
     __syncthreads();
@@ -1047,7 +1077,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     __syncthreads();
 #pragma unroll 1
     for (int t = tid; t < s.N * nc; t += nthr()) {  // the nc heaviest of each node
-      const int g = t / nc;
+      const int g = qdivm(t, nc, a.m_nc);
       const int j = static_cast<int>(kIdxMask - (csorted[g * s.lpn + (t - g * nc)] & kIdxMask));
       cand_w[t] = wm[g * s.lpn + j];
       cand_i[t] = j;
@@ -1057,7 +1087,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
 #pragma unroll 1
       for (int t = tid; t < s.N * nc; t += nthr()) cand_c[t] = 1;
       __syncthreads();
-      replicate_pairs(s, cand_w, cand_i, cand_c, p2m, rrank);
+      replicate_pairs(s, cand_w, cand_i, cand_c, p2m, rrank, a.m_grid, a.m_r);
     } else {
 #pragma unroll 1
       for (int n = tid >> 5; n < s.N; n += nwarps())
@@ -1066,7 +1096,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
     __syncthreads();
 #pragma unroll 1
     for (int t = tid; t < s.N * nc; t += nthr()) {
-      const int n = t / nc;
+      const int n = qdivm(t, nc, a.m_nc);
       if (EPLB_IN(cand_i[t] >= 0 && cand_i[t] < s.lpn, a.status)) cnt[n * s.lpn + cand_i[t]] = cand_c[t];
     }
   } else if (nc > 32) {
@@ -1130,18 +1160,18 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   if (s.ppg == 1) {  // one replica per GPU: identity short-cut
 #pragma unroll 1
     for (int t = tid; t < s.P; t += nthr()) {
-      const int n = t / s.ppn;
+      const int n = qdivm(t, s.ppn, a.m_ppn);
       ipack[t] = t - n * s.ppn;
       irank[t] = 0;
     }
   } else if (flags[0] == 0) {
     step3<uint64_t, kCap2>(Step3Ops{smem + lay.keys, smem + lay.sorted, smem + lay.pw, wm, lam, cnt,
                                     p2m, reinterpret_cast<int32_t *>(smem + lay.pc), ipack, irank,
-                                    s.N, s.npad, s.lpn, s.ppn, s.mpn, s.ppg, a.status});
+                                    s.N, s.npad, s.lpn, s.ppn, s.mpn, s.ppg, a.status, a.m_per});
   } else {
     step3_wide<kCap2>(smem + lay.keys, smem + lay.sorted, smem + lay.pw, wm, lam, cnt, p2m,
                       reinterpret_cast<int32_t *>(smem + lay.pc), ipack, irank, s.N, s.npad, s.lpn,
-                      s.ppn, s.mpn, s.ppg, a.status);
+                      s.ppn, s.mpn, s.ppg, a.status, a.m_per);
   }
   // plan quality: every logical expert's slot value w / logcnt, by the warps
   // the packing chain leaves idle (the highest thread ids take the first
@@ -1169,7 +1199,7 @@ __device__ __forceinline__ void rebalance_row(const RbArgs &a, int64_t row, unsi
   bool slots = false;
 #pragma unroll 1
   for (int t = tid; t < s.P; t += nthr()) {
-    const int n = t / s.ppn;
+    const int n = qdivm(t, s.ppn, a.m_ppn);
     const int pphy = n * s.ppn + ipack[t] * s.ppg + irank[t];
     const int m = n * s.lpn + p2m[t];
     const int e = mlog2log[m];

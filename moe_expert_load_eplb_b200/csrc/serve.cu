@@ -94,6 +94,7 @@ eplb_status launch_serve(const int32_t *idx, int64_t L, int64_t T, int32_t K, in
   a.b.stats = stats;
   a.b.s = sh;
   a.b.x_magic = 0xffffffffu / static_cast<uint32_t>(sh.X);
+  set_row_magics(a.b);
   a.b.table_vec4 = ((static_cast<int64_t>(sh.E) * sh.X) % 4 == 0) &&
                    (reinterpret_cast<uintptr_t>(next_log2phy) % 16 == 0);
   a.layer_done = layer_done;
