@@ -189,12 +189,13 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
   uint64_t div_mask = a.div_mask;
 
   // this CTA: part j of layer l.  The layer's 16-byte aligned interior
-  // [b0, b1) is cut into blocks of kThreads * kU vectors and part j takes
-  // blocks j, j + chunks, j + 2 * chunks, ...: the layer's CTAs sweep it
-  // side by side, so the DRAM pages they read and write are few at a time
-  // (the same copy traffic with one contiguous range per CTA measured 2 us
-  // slower behind the step's dirty L2).  Part 0 also takes the up to 3
-  // elements before b0 and after b1.
+  // [b0, b1) is cut into slices of kThreads vectors and part j takes slices
+  // j, j + chunks, j + 2 * chunks, ... (a thread's kU loads of a batch are
+  // kU of them): the layer's CTAs sweep it side by side, so the DRAM pages
+  // they read and write are few at a time (the same copy traffic with one
+  // contiguous range per CTA measured 2 us slower behind the step's dirty
+  // L2; blocks of 2 or 4 batches were slower than single slices).  Part 0
+  // also takes the up to 3 elements before b0 and after b1.
   const int64_t layer = cta / a.chunks;
   const int64_t j = cta - layer * a.chunks;
   const int64_t lbase = layer * a.per_layer;
@@ -205,7 +206,8 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
   int4 *pout = reinterpret_cast<int4 *>(a.out) + (b0 >> 2);
   const int nvec = static_cast<int>((b1 - b0) >> 2);
   const uint32_t pos0 = static_cast<uint32_t>(b0 - lbase);
-  const int step = static_cast<int>(a.chunks) * (kThreads * kU);  // vectors between blocks
+  const int sl = static_cast<int>(a.chunks) * kThreads;  // vectors between a part's slices
+  const int step = sl * kU;                                // between its batches
 
   const int32_t *l2p_layer = a.log2phy + layer * static_cast<int64_t>(a.E) * a.X;
   const int32_t *cnt = a.logcnt + layer * a.E;
@@ -251,14 +253,14 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
   // first vectors in flight while the tables are built, and the batch after
   // them requested into L2 (a prefetch holds no register): twice the bytes
   // in flight while the plan loads are outstanding
-  int i = static_cast<int>(j) * (kThreads * kU) + tid;
+  int i = static_cast<int>(j) * kThreads + tid;
   int4 x[kU];
 #pragma unroll
   for (int u = 0; u < kU; ++u)
-    x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
+    x[u] = i + u * sl < nvec ? __ldcs(pin + i + u * sl) : make_int4(0, 0, 0, 0);
 #pragma unroll
   for (int u = 0; u < kU; ++u)
-    if (i + step + u * kThreads < nvec) prefetch_l2(pin + i + step + u * kThreads);
+    if (i + step + u * sl < nvec) prefetch_l2(pin + i + step + u * sl);
 
   // a layer whose replica counts all divide 24 (1..4, 6, 8, 12, 24) gets the
   // 24-entry period: a fifth of the table to build before streaming
@@ -376,23 +378,23 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
     };
     // whole batches without per-vector range checks, then the guarded rest
     // (a batch that is not whole is the thread's last: the next one starts
-    // a whole block further on)
-    while (i + (kU - 1) * kThreads < nvec) {
+    // past its last slice)
+    while (i + (kU - 1) * sl < nvec) {
 #pragma unroll
-      for (int u = 0; u < kU; ++u) vector(i + u * kThreads, x[u]);
+      for (int u = 0; u < kU; ++u) vector(i + u * sl, x[u]);
       i += step;
 #pragma unroll
       for (int u = 0; u < kU; ++u)
-        x[u] = i + u * kThreads < nvec ? __ldcs(pin + i + u * kThreads) : make_int4(0, 0, 0, 0);
+        x[u] = i + u * sl < nvec ? __ldcs(pin + i + u * sl) : make_int4(0, 0, 0, 0);
       // one batch ahead into L2 (measured: -3 us on the 121.6 MB batch,
       // even on the 1.95 GB stream; two batches ahead was slower)
 #pragma unroll
       for (int u = 0; u < kU; ++u)
-        if (i + step + u * kThreads < nvec) prefetch_l2(pin + i + step + u * kThreads);
+        if (i + step + u * sl < nvec) prefetch_l2(pin + i + step + u * sl);
     }
 #pragma unroll
     for (int u = 0; u < kU; ++u)
-      if (i + u * kThreads < nvec) vector(i + u * kThreads, x[u]);
+      if (i + u * sl < nvec) vector(i + u * sl, x[u]);
   };
   if (fast)
     stream(ctx_fast, map_fast);
