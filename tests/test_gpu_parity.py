@@ -256,6 +256,31 @@ def test_rebalance_shapes(shape, dist):
     _assert_plan_equal(plan, ref)
 
 
+@pytest.mark.parametrize("shape", [(256, 8, 288, 4, 32), (64, 8, 96, 4, 16), (24, 6, 36, 3, 6)])
+@pytest.mark.parametrize("edge", [-1, 0])
+def test_rebalance_replica_ranking_widths(shape, edge):
+    """The replica ranking takes 32-bit arithmetic while a node's heaviest
+    candidate times R + 1 stays below 2^31 and 64-bit arithmetic from there:
+    loads at that edge (one below it, and at it), many of them exact
+    multiples of each other so that w_k2 * d == w_k * d2 ties are common,
+    give the oracle's plans on both sides."""
+    E, G, P, N, gpus = shape
+    R = P // N - E // N
+    top = (1 << 31) // (R + 1) + edge  # heaviest load of every node
+    rng = np.random.default_rng(R * 7 + edge)
+    rows = []
+    for _ in range(6):
+        base = top // 12
+        w = base * rng.choice([12, 6, 4, 3, 2, 1], E)  # exact ratios among the loads
+        w[rng.integers(0, E, E // 8)] = rng.integers(0, base, E // 8)
+        for n in range(N):
+            w[n * (E // N) + rng.integers(0, E // N)] = top
+        rows.append(w)
+    plan, ref, st = _rebalance_both(np.stack(rows).astype(np.int64), P, G, N, gpus)
+    assert st == 0
+    _assert_plan_equal(plan, ref)
+
+
 def _random_shape(rng):
     while True:
         N = int(rng.choice([1, 2, 3, 4, 5, 8]))
