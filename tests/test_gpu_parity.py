@@ -493,6 +493,31 @@ def test_count_redirect_workloads(cfg, request):
     assert int(bad.item()) == nb == nb2 == 0 and int(st.item()) == 0
 
 
+@pytest.mark.parametrize("shape", [(1, 200003, 8), (2, 333331, 3), (3, 65537, 7)])
+def test_count_redirect_many_parts_per_layer(shape):
+    """Layers split over many CTAs that take the layer's slices in turn, with
+    a ragged layer length (not a multiple of 4): every index counted and
+    redirected once, as the oracle does."""
+    L, T, K = shape
+    E, P, G, N, gpus = 256, 288, 8, 4, 32
+    rng = np.random.default_rng(L * 13 + T)
+    ref_plan = oracle.rebalance(rng.integers(0, 100000, (L, E)), P, G, N, gpus)
+    l2p = torch.from_numpy(ref_plan[3]).to(DEV)
+    cnt = torch.from_numpy(ref_plan[2]).to(DEV)
+    g = torch.Generator(device=DEV).manual_seed(T)
+    idx = torch.randint(-1, E + 1, (L, T, K), generator=g, device=DEV, dtype=torch.int32)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    counts, out = eplb.count_redirect(idx, E, l2p, cnt, token_offset=5, bad=bad)
+    idx_h = _np(idx)
+    ref_c, nb = oracle.count_loads(idx_h, E)
+    ref_o, _ = oracle.redirect(idx_h, ref_plan[3], ref_plan[2], 5)
+    assert np.array_equal(_np(counts), ref_c)
+    assert np.array_equal(_np(out), ref_o)
+    assert int(bad.item()) == nb
+    only = eplb.count_loads(idx, E)
+    assert np.array_equal(_np(only), ref_c)
+
+
 @pytest.mark.parametrize("shape", [(1, 1, 1), (3, 1001, 3), (2, 4097, 8), (5, 3, 7), (2, 70001, 5),
                                    (4, 2048, 6), (7, 12345, 2)])
 @pytest.mark.parametrize("t0", [0, 19, (1 << 31) - 80000])
