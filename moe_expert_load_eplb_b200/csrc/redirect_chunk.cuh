@@ -10,7 +10,10 @@
 // of one layer (a contiguous run of the flattened index array whose interior
 // is 16-byte aligned); every thread keeps U = 4 independent 16-byte
 // streaming loads in flight, the next U vectors requested into L2 by
-// prefetches, and writes 16-byte streaming stores.
+// prefetches, and writes 16-byte stores with the default cache policy (the
+// evict-first `.cs` stores measured 0.6-0.8% slower on the 1.95 GB stream
+// and 1.2 us slower for count+redirect on the 121.6 MB batch; the default
+// also leaves the output in L2 for the kernel that reads it next).
 // The per-index work decides the speed, so the common case is cut to a
 // handful of instructions:
 //
@@ -374,7 +377,7 @@ __device__ __forceinline__ void redirect_chunk(const RedirectArgs &a, unsigned c
         y.z = map1(xv.z, ctx_of(a.t0 + div_magic(pos + 2, a.K, a.k_magic)));
         y.w = map1(xv.w, ctx_of(a.t0 + div_magic(pos + 3, a.K, a.k_magic)));
       }
-      __stcs(pout + v, y);
+      pout[v] = y;
     };
     // whole batches without per-vector range checks, then the guarded rest
     // (a batch that is not whole is the thread's last: the next one starts
