@@ -1165,6 +1165,38 @@ def test_rebalance_window_matches_window_then_rebalance(W_, zero):
             assert np.array_equal(after[k], ring_h[k])
 
 
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("dist", ["uniform", "huge"])
+def test_rebalance_window_rotating_ring_shapes(shape, dist):
+    """A rotating ring (zero_slot >= 0: the serving step's call, which runs
+    the instruction warm-up on shapes with room for its scratch) and a fixed
+    one give the same plan, the oracle's for the summed rows; the cleared
+    slot is all zero afterwards."""
+    E, G, P, N, gpus = shape
+    rng = np.random.default_rng(abs(hash((E, G, P, N, gpus, dist))) % (1 << 31))
+    R = 5
+    if dist == "uniform":
+        w = rng.integers(0, 5000, (R, E))
+    else:
+        w = rng.integers((1 << 40) - 100000, 1 << 40, (R, E))
+    w = w.astype(np.int64)
+    ring_h = np.stack([w // 3, w // 3, w - 2 * (w // 3)])
+    plans, statuses = [], []
+    for zero in (-1, 1):
+        ring = torch.from_numpy(ring_h.copy()).to(DEV)
+        st = _status()
+        plans.append(eplb.rebalance_window(ring, P, G, N, gpus, zero_slot=zero, status=st))
+        torch.cuda.synchronize()
+        after = _np(ring)
+        assert np.array_equal(after[0], ring_h[0]) and np.array_equal(after[2], ring_h[2])
+        assert np.array_equal(after[1], ring_h[1] if zero < 0 else np.zeros_like(ring_h[1]))
+        statuses.append(int(st.item()))
+    ref, ref_status = _oracle_rows(w, P, G, N, gpus, plans[0].log2phy.shape[2])
+    assert statuses == [ref_status, ref_status]
+    for plan in plans:
+        _assert_plan_equal(plan, ref)
+
+
 def test_rebalance_window_range_error():
     ring = torch.full((2, 3, 12), 1 << 39, dtype=torch.int64, device=DEV)  # sums reach 2^40
     ring[:, 1] = 5
