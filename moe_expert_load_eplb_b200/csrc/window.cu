@@ -36,19 +36,33 @@ struct WinBlock {
   int64_t add[kU];
   int64_t sub[kSub ? kU : 1];
 
+  // Rows r0 .. r0+kU-1 of column c: one pointer stepped by C through a
+  // whole group of rows, per-row checks only where the group is cut.
   __device__ __forceinline__ void load(const int64_t *__restrict__ steps, int64_t S, int64_t C,
                                        int64_t W, int64_t r0, int64_t c, bool col_ok) {
+    if (col_ok && r0 + kU <= S) {
+      const int64_t *p = steps + r0 * C + c;
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t r = r0 + u;
-      add[u] = (col_ok && r < S) ? __ldcs(steps + r * C + c) : 0;
-    }
-    if (kSub) {
-      const bool any_sub = r0 + kU - 1 >= W;  // warp-uniform: r0 is the warp's first row
+      for (int u = 0; u < kU; ++u, p += C) add[u] = __ldcs(p);
+    } else {
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int64_t r = r0 + u;
-        sub[kSub ? u : 0] = (any_sub && col_ok && r < S && r >= W) ? __ldg(steps + (r - W) * C + c) : 0;
+        add[u] = (col_ok && r < S) ? __ldcs(steps + r * C + c) : 0;
+      }
+    }
+    if (kSub) {
+      if (col_ok && r0 >= W && r0 + kU <= S) {
+        const int64_t *p = steps + (r0 - W) * C + c;
+#pragma unroll
+        for (int u = 0; u < kU; ++u, p += C) sub[kSub ? u : 0] = __ldg(p);
+      } else {
+        const bool any_sub = r0 + kU - 1 >= W;  // warp-uniform: r0 is the warp's first row
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int64_t r = r0 + u;
+          sub[kSub ? u : 0] = (any_sub && col_ok && r < S && r >= W) ? __ldg(steps + (r - W) * C + c) : 0;
+        }
       }
     }
   }
@@ -90,7 +104,11 @@ __global__ void __launch_bounds__(kCols * kMaxRg) window_kernel(
       before += (h < g) ? p : 0;
       tot += p;
     }
-    if (col_ok && r0 + kU > s_first) {
+    if (col_ok && r0 >= s_first && r0 + kU <= S) {
+      int64_t *p = snaps + (r0 - s_first) * C + c;
+#pragma unroll
+      for (int u = 0; u < kU; ++u, p += C) __stcs(p, before + cur.add[u]);
+    } else if (col_ok && r0 + kU > s_first) {
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
         const int64_t r = r0 + u;
