@@ -190,7 +190,10 @@ static eplb_status rebalance_shape(int64_t R, int32_t E, int32_t P, int32_t G, i
   sh.ppn = P / sh.N;
   sh.ppg = P / gpus;
   sh.mpn = gpus / sh.N;
-  sh.npad = next_pow2(sh.ppn);
+  // the rank sort needs no padding (the stride is ppn: the key areas, sized
+  // by npad, hold 4 x 72 instead of 4 x 128 keys on the DeepSeek-V3 shape,
+  // so 6 rows share an SM instead of 5); the bitonic network does
+  sh.npad = sh.ppn <= kRankSortMax ? sh.ppn : next_pow2(sh.ppn);
   sh.gpad = next_pow2(sh.G);
   sh.ibits = bit_width(sh.ppn);
   sh.qbits = bit_width(sh.mpn - 1);

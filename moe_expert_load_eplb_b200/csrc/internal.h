@@ -55,10 +55,15 @@ eplb_status launch_count_loads(const int32_t *idx, int64_t L, int64_t per_layer,
 eplb_status launch_window(int64_t *steps, int64_t S, int64_t C, int64_t W, int64_t s_first,
                           int64_t *snaps, int64_t zero_row, cudaStream_t stream);
 
+// Segments up to this many keys are sorted by rank counting; longer ones by
+// a bitonic network over a power-of-two padding.
+constexpr int kRankSortMax = 512;
+
 struct RebalanceShape {
   int32_t E, P, G, N, gpus, X;   // G, N after the policy choice
   int32_t gs, gpn, lpn, ppn, ppg, mpn;
-  int32_t npad, gpad;
+  int32_t npad;                  // step 3's key stride per node: ppn, or next_pow2(ppn) above kRankSortMax
+  int32_t gpad;
   int32_t ibits, qbits, gibits, nqbits;
   int32_t cmax;                  // most replicas one expert can get: ppn - lpn + 1
   uint64_t lam_fixed;            // lcm(1..cmax) when <= 2^62, else 0

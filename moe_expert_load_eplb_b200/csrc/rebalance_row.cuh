@@ -83,7 +83,6 @@ constexpr int kManyRowThreads = 128;
 __device__ __forceinline__ int nthr() { return static_cast<int>(blockDim.x); }
 __device__ __forceinline__ int nwarps() { return static_cast<int>(blockDim.x) >> 5; }
 constexpr int64_t kLoadLimit = int64_t(1) << 40;
-constexpr int kRankSortMax = 512;        // longer segments use the bitonic network
 constexpr int kTableMaxEntries = 16384;  // log2phy rows up to this size are built in smem
 // Every composite key keeps an index (item, pack, group or expert, all < 4096)
 // in its low kIdxBits bits, so keys are combined with constant shifts only.
