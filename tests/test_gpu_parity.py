@@ -1014,22 +1014,34 @@ def test_rebalance_fused_quality_shapes(shape):
 
 
 @pytest.mark.parametrize("shape", [(256, 8, 288, 4, 32), (256, 1, 288, 2, 144), (12, 4, 16, 2, 8),
-                                   (64, 32, 128, 16, 32), (300, 5, 602, 7, 7)])
-def test_rebalance_many_rows(shape):
-    """More rows than two per SM take the 128-thread many-row kernel: the same
-    plans and plan quality as the oracle's."""
+                                   (64, 32, 128, 16, 32), (300, 5, 602, 7, 7),
+                                   (96, 3, 2048, 2, 8), (1024, 32, 2048, 8, 64)])
+@pytest.mark.parametrize("dist", ["pareto", "huge"])
+def test_rebalance_many_rows(shape, dist):
+    """More rows than two per SM take the 128-thread many-row kernel and its
+    compact shared-memory layout (step 3's outputs in a key area; the
+    staging arrays in the table's place): the same plans and plan quality as
+    the oracle's, with the bitonic path (1,024 replicas a node), a log2phy
+    table outside shared memory and 128-bit keys among the cases."""
     E, G, P, N, gpus = shape
     R = 2 * torch.cuda.get_device_properties(0).multi_processor_count + 11
-    rng = np.random.default_rng(E + P + R)
-    loads_np = (rng.pareto(1.3, (R, E)) * 1000).astype(np.int64)
+    rng = np.random.default_rng(E + P + R + len(dist))
+    if dist == "pareto":
+        loads_np = (rng.pareto(1.3, (R, E)) * 1000).astype(np.int64)
+    else:
+        loads_np = rng.integers((1 << 40) - 100000, 1 << 40, (R, E)).astype(np.int64)
     loads_np[5] = 0
     gl, st = _quality_bufs(R, gpus)
-    plan = eplb.rebalance(torch.from_numpy(loads_np).to(DEV), P, G, N, gpus, gpu_load=gl, stats=st)
+    status = _status()
+    plan = eplb.rebalance(torch.from_numpy(loads_np).to(DEV), P, G, N, gpus, gpu_load=gl, stats=st,
+                          status=status)
+    torch.cuda.synchronize()
     ref, ref_status = _oracle_rows(loads_np, P, G, N, gpus, plan.log2phy.shape[2])
-    assert ref_status == 0
+    assert int(status.item()) == ref_status
     _assert_plan_equal(plan, ref)
-    ref_gl, ref_st = oracle.plan_stats(loads_np, ref[0], ref[2], gpus)
-    assert np.array_equal(_np(gl), ref_gl) and np.array_equal(_np(st), ref_st)
+    if ref_status == 0:
+        ref_gl, ref_st = oracle.plan_stats(loads_np, ref[0], ref[2], gpus)
+        assert np.array_equal(_np(gl), ref_gl) and np.array_equal(_np(st), ref_st)
 
 
 def test_rebalance_fused_quality_worked_example():
